@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Throughput of the chunkwise linear-recurrence layer, forward + backward.
+
+One step = the forward sub-sequence driver (sf_fwd_seq) and the backward one
+(sf_bwd_seq) over one batch of the workload, the gated delta rule with H=32,
+d=128, T=65536 cut into 16 sub-sequences of 4096 by default.  Prints one JSON
+line (rank 0).  ``--impl reference`` times the fp64 CPU oracle instead.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own independent
+copy of the workload (heads and batches are independent, so there is no
+exchange on the data path): weak scaling, value = all ranks' tokens / the
+slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from chunked_linear_recurrence_chunkwise_b200 import inputs  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+SM_COUNT = 148
+FP32_LANES_PER_SM = 128
+
+
+# ------------------------------------------------------------------ host logic
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="sf", choices=["sf", "reference"])
+    p.add_argument("--workload", default=inputs.BENCH_WORKLOAD, choices=list(inputs.WORKLOADS))
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-sample-tokens", type=int, default=16384)
+    return p.parse_args(argv)
+
+
+def dist_env():
+    """(rank, world, local_rank) from the torchrun environment."""
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def rank_workload(w, rank: int):
+    """Each rank gets an independent problem of the same shape (its own seed)."""
+    return w if rank == 0 else w.scaled(seed=w.seed + 7919 * rank)
+
+
+def reduce_max(value: float, group=None, device=None) -> float:
+    """Max of a float over the ranks of the default process group (identity if none)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(t.item())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except OSError:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_units(name: str, w) -> dict:
+    """Algorithmic bytes and flops of one chunk-head (64 tokens of one head) per kernel.
+
+    Bytes count each input and output the kernel must move once, at the
+    precision this implementation stores it (I/O in the workload dtype, g and
+    beta and every intermediate in fp32); flops count the chunk's arithmetic
+    once, triangle-aware (only the causal half of the 64 x 64 products).
+    """
+    C, d = 64, w.d
+    e = 2 if w.dtype == "bf16" else 4
+    f = 4
+    tri_s = C * (C - 1) // 2   # strictly lower entries
+    tri_i = C * (C + 1) // 2   # inclusive lower entries
+    tab = {
+        "intra_fwd": (2 * C * d * e + 2 * C * f + C * f + 2 * C * d * f,
+                      tri_s * 2 * d + tri_s * 2 * 2 * d),
+        "state_fwd": (2 * C * d * f + C * d * e + C * f + d * d * f + C * d * f,
+                      4 * C * d * d),
+        "output": (2 * C * d * e + C * f + d * d * f + C * d * f + C * d * e,
+                   tri_i * 2 * d * 2 + 2 * C * d * d),
+        "dd_pre": (3 * C * d * e + C * f + C * d * f, tri_i * 2 * d * 2),
+        "state_bwd": (3 * C * d * e + 2 * C * d * f + C * f + d * d * f + C * d * f,
+                      6 * C * d * d),
+        "grad_delta": (2 * C * d * e + 2 * C * f + 3 * C * d * f + d * d * f + C * d * e + C * f
+                       + C * d * f + C * f,
+                       tri_s * 2 * d * 6 + C * C * C // 3 * 2 + 2 * C * d * d),
+        "grad_attn": (3 * C * d * e + C * d * f + C * f + 2 * d * d * f + C * d * f + C * f
+                      + 2 * C * d * e + C * f,
+                      tri_i * 2 * d * 4 + 4 * C * d * d),
+    }
+    b, fl = tab.get(name, (0, 0))
+    return {"bytes": b, "flops": fl}
+
+
+def roofline(timing: dict, w, steps: int, peaks: dict, peaks_src: str, clocks: dict):
+    """Roofline object of the kernel with the largest total time in the timed region."""
+    if not timing:
+        return None
+    name, (launches, ms) = max(timing.items(), key=lambda kv: kv[1][1])
+    if launches == 0 or ms <= 0:
+        return None
+    chunk_heads = w.B * w.H * ((w.T + 63) // 64) * steps  # over the timed steps
+    u = kernel_units(name, w)
+    per_launch_s = ms / 1e3 / launches
+    bytes_pl = u["bytes"] * chunk_heads / launches
+    flops_pl = u["flops"] * chunk_heads / launches
+    gbs = bytes_pl / per_launch_s / 1e9
+    tfs = flops_pl / per_launch_s / 1e12
+    hbm = float(peaks["hbm_gbs"])
+    # the current kernels do their arithmetic on fp32 CUDA cores: ALU peak from unit counts
+    mhz = float(peaks.get("sm_max_mhz", 1965.0))
+    alu = SM_COUNT * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+    if gbs / hbm >= tfs / alu:
+        obj = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+               "frac": round(gbs / hbm, 4)}
+    else:
+        obj = {"bound": "alu", "achieved": round(tfs, 2), "peak": round(alu, 1), "unit": "TFLOP/s",
+               "frac": round(tfs / alu, 4)}
+    obj.update({"kernel": name, "traffic": None, "launches": launches,
+                "avg_launch_ms": round(ms / launches, 4), "peak_source": peaks_src,
+                "share_of_kernel_time": round(ms / sum(v[1] for v in timing.values()), 4)})
+    return obj
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        return summarize_clocks(self.lines)
+
+
+def summarize_clocks(lines) -> dict:
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    sm, mx, reasons = [], [], set()
+    for ln in lines:
+        parts = [x.strip() for x in ln.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            mx.append(float(parts[2]))
+        except ValueError:
+            continue
+        for nm, val in zip(names, parts[5:9]):
+            if val.lower().startswith("active"):
+                reasons.add(nm)
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+            "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle timing
+def time_oracle(w, heads: int, tokens: int):
+    """fp64 oracle fwd + bwd on a bounded sample of workload w; returns (tokens/s, info)."""
+    import oracle
+    cores = oracle.max_threads()
+    hs = list(range(min(heads, w.H)))
+    x = inputs.generate(w, 0, tokens, heads=hs, with_grad=True)
+    t0 = time.perf_counter()
+    o, S = oracle.fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], nthreads=cores)
+    oracle.bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["dO"], nthreads=cores)
+    dt = time.perf_counter() - t0
+    layer_tokens = w.B * tokens * len(hs) / w.H  # a layer token covers all H heads
+    return layer_tokens / dt, {
+        "cores": cores, "seconds": round(dt, 3),
+        "sample": f"B={w.B} x {tokens} tokens x {len(hs)} of {w.H} heads, fwd+bwd, fp64 token loop; "
+                  f"tokens/s counts a token as all {w.H} heads",
+    }
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return 0
+    import oracle
+    cores = oracle.max_threads()
+    heads = max(1, min(w.H, cores))
+    tokens = min(w.T, 4096)
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, info = time_oracle(w, heads, tokens)
+        if i >= args.warmup:
+            vals.append(v)
+    val = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": "fwd+bwd tokens/s per layer", "value": round(val, 3),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(w.B * w.T / val * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d": w.d,
+                   "n_sub": w.n_sub, "chunk": 64},
+        "cpu_baseline": {"value": round(val, 3), "unit": "tokens/s", "cores": info["cores"],
+                         "kind": "oracle", "sample": info["sample"] + "; each step one sample"},
+        "e2e": {"value": round(val, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_sf(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from chunked_linear_recurrence_chunkwise_b200 import layer, sf
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wr = rank_workload(w, rank)
+    lens = inputs.sub_lengths(wr)
+    host = inputs.to_torch(wr, pin=True)  # pinned host copies (end-to-end leg)
+    x = {k_: (None if t is None else t.to(dev, non_blocking=True)) for k_, t in host.items()}
+    torch.cuda.synchronize()
+    B, T, H, d = wr.B, wr.T, wr.H, wr.d
+    sh = sf.shape_of(x["q"], x["v"])
+    ws_f = torch.empty(sf.sf_seq_workspace_bytes(sh, lens, sf.SF_OP_FWD), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(sf.sf_seq_workspace_bytes(sh, lens, sf.SF_OP_BWD), dtype=torch.uint8, device=dev)
+    main = torch.cuda.Stream(device=dev)
+    aux = torch.cuda.Stream(device=dev)
+    o = torch.empty_like(x["v"])
+    S_out = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+    S_saved = torch.empty((len(lens), B, H, d, d), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"])
+    dg = None if x["g"] is None else torch.empty_like(x["g"])
+    db = None if x["beta"] is None else torch.empty_like(x["beta"])
+    dS_in = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+
+    def step(src):
+        sf.sf_fwd_seq(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], None, o, S_out,
+                      S_saved, ws_f, stream_main=main, stream_aux=aux)
+        sf.sf_bwd_seq(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], S_saved,
+                      src["dO"], None, dq, dk, dv, dg, db, dS_in, ws_b, stream_main=main,
+                      stream_aux=aux)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+
+    for _ in range(args.warmup):
+        step(x)
+    torch.cuda.synchronize()
+    sf.sf_check(ws_f, main)
+    sf.sf_check(ws_b, main)
+
+    # ---- device-timed region (inputs resident in HBM; they exceed L2, so no flush)
+    clk = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    sf.sf_timing_reset()
+    sf.sf_timing_enable(True)
+    clk.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    for _ in range(args.steps):
+        step(x)
+    e1.record(main)
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    sf.sf_timing_enable(False)
+    timing = sf.sf_timing_read()
+    barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms_max = reduce_max(ms, device=dev)
+    sf.sf_check(ws_f, main)
+    sf.sf_check(ws_b, main)
+    launches = sum(v[0] for v in timing.values()) // max(1, args.steps)
+
+    # ---- end to end: pinned host inputs -> device -> fwd+bwd -> results back to host
+    e2e = None
+    if not args.no_e2e:
+        outs_h = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                  for n, t in [("o", o), ("dq", dq), ("dk", dk), ("dv", dv), ("S_out", S_out),
+                               ("dS_in", dS_in)] + ([("dg", dg)] if dg is not None else [])
+                  + ([("dbeta", db)] if db is not None else [])}
+        outs_d = {"o": o, "dq": dq, "dk": dk, "dv": dv, "S_out": S_out, "dS_in": dS_in, "dg": dg,
+                  "dbeta": db}
+        h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+        d2h = sum(t.numel() * t.element_size() for t in outs_h.values())
+        e2e_steps = max(1, min(args.steps, 5))
+        barrier()
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(main)
+        with torch.cuda.stream(main):
+            for _ in range(e2e_steps):
+                for n_, t in host.items():
+                    if t is not None:
+                        x[n_].copy_(t, non_blocking=True)
+                step(x)
+                for n_, t in outs_h.items():
+                    t.copy_(outs_d[n_], non_blocking=True)
+        f1.record(main)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = reduce_max(f0.elapsed_time(f1) / e2e_steps, device=dev)
+        e2e = {"value": round(world * B * T / (e_ms / 1e3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 3),
+               "steps": e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, info = time_oracle(w, heads=w.H, tokens=min(w.T, args.cpu_sample_tokens))
+        cpu = {"value": round(val, 3), "unit": "tokens/s", "cores": info["cores"], "kind": "oracle",
+               "sample": info["sample"]}
+
+    if rank == 0:
+        peaks, src = load_peaks()
+        line = {
+            "metric": "fwd+bwd tokens/s per layer", "value": round(world * B * T / (ms_max / 1e3), 1),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "T": T, "H": H, "d": d, "n_sub": len(lens),
+                       "chunk": 64, "variant": w.variant, "l2": "inputs larger than L2, no flush",
+                       "parallelism": f"replicas{world}"},
+            "clocks": clocks,
+            "gpu_launches": launches,
+            "e2e": e2e,
+            "roofline": roofline(timing, w, args.steps, peaks, src, clocks),
+            "kernels": {k_: {"launches": v[0] // max(1, args.steps),
+                             "ms_per_step": round(v[1] / args.steps, 4)} for k_, v in timing.items()},
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local_rank = dist_env()
+    w = inputs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        return run_sf(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

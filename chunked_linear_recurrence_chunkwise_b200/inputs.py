@@ -200,3 +200,65 @@ def random_state(w: Workload, seed_tag: int, scale: float = 0.1, B=None, H=None)
 
 def n_chunks(T: int, chunk: int = 64) -> int:
     return math.ceil(T / chunk)
+
+
+def iter_blocks(w: Workload, heads=None, with_grad: bool | None = None, threads: int | None = None):
+    """Yields ``(t0, t1, arrays)`` for consecutive 4096-token blocks of workload ``w``.
+
+    Blocks are drawn in a thread pool (numpy releases the GIL while drawing)
+    and yielded in order; concatenating them gives ``generate(w)``.
+    """
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    nblk = (w.T + BLOCK - 1) // BLOCK
+    threads = threads or min(32, os.cpu_count() or 1)
+    with ThreadPoolExecutor(threads) as ex:
+        futs = {}
+        ahead = 2 * threads
+
+        def submit(i):
+            t0, t1 = i * BLOCK, min(w.T, (i + 1) * BLOCK)
+            futs[i] = ex.submit(generate, w, t0, t1, heads, with_grad)
+
+        for i in range(min(nblk, ahead)):
+            submit(i)
+        for i in range(nblk):
+            arrays = futs.pop(i).result()
+            if i + ahead < nblk:
+                submit(i + ahead)
+            yield i * BLOCK, min(w.T, (i + 1) * BLOCK), arrays
+
+
+def to_torch(w: Workload, device="cpu", heads=None, with_grad: bool | None = None, pin=False):
+    """Workload inputs as torch tensors (q, k, v, dO in the workload dtype; g, beta float32).
+
+    Filled block by block, so the host never holds more than a few blocks in
+    float32.  ``pin`` allocates page-locked host memory (``device='cpu'``).
+    """
+    import torch
+
+    H = w.H if heads is None else len(heads)
+    io = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    grad = w.backward if with_grad is None else with_grad
+    shapes = {"q": (w.B, w.T, H, w.d), "k": (w.B, w.T, H, w.d), "v": (w.B, w.T, H, w.d)}
+    if w.has_g:
+        shapes["g"] = (w.B, w.T, H)
+    if w.has_beta:
+        shapes["beta"] = (w.B, w.T, H)
+    if grad:
+        shapes["dO"] = (w.B, w.T, H, w.d)
+    out = {}
+    for key, shp in shapes.items():
+        dt = torch.float32 if key in ("g", "beta") else io
+        if pin:
+            out[key] = torch.empty(shp, dtype=dt, pin_memory=True)
+        else:
+            out[key] = torch.empty(shp, dtype=dt, device=device)
+    for t0, t1, arr in iter_blocks(w, heads, grad):
+        for key in shapes:
+            src = torch.from_numpy(arr[key])
+            out[key][:, t0:t1].copy_(src.to(out[key].dtype))
+    for key in ("g", "beta", "dO"):
+        out.setdefault(key, None)
+    return out

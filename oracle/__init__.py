@@ -27,11 +27,11 @@ _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile sf_oracle.c into libsf_oracle.so next to it (gcc, -O2, OpenMP)."""
+    """Compile sf_oracle.c into libsf_oracle.so next to it (gcc, -O3, OpenMP)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call(
-            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99", _SRC, "-o", tmp, "-lm"]
+            ["gcc", "-O3", "-fopenmp", "-fPIC", "-shared", "-std=c99", _SRC, "-o", tmp, "-lm"]
         )
         os.replace(tmp, _LIB)
     return _LIB

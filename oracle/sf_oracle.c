@@ -193,16 +193,14 @@ static void oracle_bwd_head(const dims_t* d, int b, int h, int seg, const double
             if (beta) {
                 const double bt = beta[ti];
                 double db = 0.0;
-                for (int j = 0; j < dv; ++j) {
-                    double acc = 0.0;
-                    for (int i = 0; i < dk; ++i) acc += P[i * dv + j] * kt[i];
-                    y[j] = acc;
-                }
-                for (int j = 0; j < dv; ++j) {
-                    double acc = 0.0;
-                    for (int i = 0; i < dk; ++i) acc += dS[i * dv + j] * kt[i];
-                    dvt[j] = bt * acc;
-                }
+                /* y = P^T k and dv_t = b dS^T k, accumulated row by row */
+                for (int j = 0; j < dv; ++j) y[j] = 0.0, dvt[j] = 0.0;
+                for (int i = 0; i < dk; ++i)
+                    for (int j = 0; j < dv; ++j) {
+                        y[j] += P[i * dv + j] * kt[i];
+                        dvt[j] += dS[i * dv + j] * kt[i];
+                    }
+                for (int j = 0; j < dv; ++j) dvt[j] *= bt;
                 for (int i = 0; i < dk; ++i) {
                     double acc = 0.0;
                     for (int j = 0; j < dv; ++j) acc += dS[i * dv + j] * vt[j];
@@ -215,11 +213,10 @@ static void oracle_bwd_head(const dims_t* d, int b, int h, int seg, const double
                         da += dS[i * dv + j] * X;
                         dX[i * dv + j] = a * dS[i * dv + j];
                     }
-                for (int j = 0; j < dv; ++j) {
-                    double acc = 0.0;
-                    for (int i = 0; i < dk; ++i) acc += dX[i * dv + j] * kt[i];
-                    z[j] = acc;
-                }
+                /* z = dX^T k */
+                for (int j = 0; j < dv; ++j) z[j] = 0.0;
+                for (int i = 0; i < dk; ++i)
+                    for (int j = 0; j < dv; ++j) z[j] += dX[i * dv + j] * kt[i];
                 for (int i = 0; i < dk; ++i) {
                     double acc = 0.0;
                     for (int j = 0; j < dv; ++j) acc += dX[i * dv + j] * y[j] + P[i * dv + j] * z[j];
@@ -230,11 +227,10 @@ static void oracle_bwd_head(const dims_t* d, int b, int h, int seg, const double
                     for (int j = 0; j < dv; ++j) dS[i * dv + j] = dX[i * dv + j] - bt * kt[i] * z[j];
                 dbeta[ti] = db;
             } else {
-                for (int j = 0; j < dv; ++j) {
-                    double acc = 0.0;
-                    for (int i = 0; i < dk; ++i) acc += dS[i * dv + j] * kt[i];
-                    dvt[j] = acc;
-                }
+                /* dv_t = dS^T k */
+                for (int j = 0; j < dv; ++j) dvt[j] = 0.0;
+                for (int i = 0; i < dk; ++i)
+                    for (int j = 0; j < dv; ++j) dvt[j] += dS[i * dv + j] * kt[i];
                 for (int i = 0; i < dk; ++i) {
                     double acc = 0.0;
                     for (int j = 0; j < dv; ++j) acc += dS[i * dv + j] * vt[j];
