@@ -25,11 +25,13 @@ namespace sf {
 
 static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-WsLayout ws_layout(int B, int T, int H, int dk, int dv, bool delta, bool bwd, int nslots) {
+WsLayout ws_layout(int B, int T, int H, int dk, int dv, int dtype, bool delta, bool bwd,
+                   int nslots) {
     WsLayout L{};
     const size_t BH = (size_t)B * H;
     const size_t NC = (size_t)(T + kChunk - 1) / kChunk;
     const size_t TP = NC * kChunk;
+    const size_t tw = dtype == SF_BF16 ? 2 : 4;  // intermediates follow the I/O precision
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t o = off;
@@ -37,12 +39,12 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv, bool delta, bool bwd, in
         return o;
     };
     L.G = take(BH * TP * 4);
-    L.W = take(delta ? BH * TP * dk * 4 : 0);
-    L.U = take(delta ? BH * TP * dv * 4 : 0);
-    L.Sc = take(BH * NC * dk * dv * 4);
-    L.D = take(BH * TP * dv * 4);
-    L.dD = take(bwd ? BH * TP * dv * 4 : 0);
-    L.dSc = take(bwd ? BH * NC * dk * dv * 4 : 0);
+    L.Wt = take(delta ? BH * TP * dk * tw : 0);
+    L.Ut = take(BH * TP * dv * tw);
+    L.Sc = take(BH * NC * dk * dv * tw);
+    L.Dt = take(BH * TP * dv * tw);
+    L.dDt = take(bwd ? BH * TP * dv * tw : 0);
+    L.dSc = take(bwd ? BH * NC * dk * dv * tw : 0);
     L.dKp = take(bwd && delta ? BH * TP * dk * 4 : 0);
     L.dGp = take(bwd && delta ? BH * TP * 4 : 0);
     L.slot_bytes = off;
@@ -53,12 +55,12 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv, bool delta, bool bwd, in
 void bind_slot(Args& a, void* ws, const WsLayout& L, int slot, bool bwd) {
     char* base = (char*)ws + kErrBytes + (size_t)slot * L.slot_bytes;
     a.G = (float*)(base + L.G);
-    a.W = (float*)(base + L.W);
-    a.U = (float*)(base + L.U);
-    a.Sc = (float*)(base + L.Sc);
-    a.D = (float*)(base + L.D);
-    a.dD = bwd ? (float*)(base + L.dD) : nullptr;
-    a.dSc = bwd ? (float*)(base + L.dSc) : nullptr;
+    a.Wt = base + L.Wt;
+    a.Ut = base + L.Ut;
+    a.Sc = base + L.Sc;
+    a.Dt = base + L.Dt;
+    a.dDt = bwd ? (void*)(base + L.dDt) : nullptr;
+    a.dSc = bwd ? (void*)(base + L.dSc) : nullptr;
     a.dKp = bwd ? (float*)(base + L.dKp) : nullptr;
     a.dGp = bwd ? (float*)(base + L.dGp) : nullptr;
     a.err = (int*)ws;
@@ -163,11 +165,17 @@ cudaError_t copy_state(float* dst, const float* src, size_t n, cudaStream_t st) 
     return cudaMemsetAsync(dst, 0, n * sizeof(float), st);
 }
 
+// Kernel choice: the tensor-core kernels cover bf16 with d_k = d_v = 128; the
+// SIMT kernels cover everything else (and are the fp32 path).
+cudaError_t state_fwd(const Args& a, cudaStream_t st) {
+    return tc_eligible(a) ? launch_state_fwd_tc(a, st) : launch_state_fwd(a, st);
+}
+
 // The forward pieces of one call: intra (may go on its own stream), then state + output.
 cudaError_t run_intra(const Args& a, cudaStream_t st) { return launch_intra_fwd(a, st); }
 
 cudaError_t run_state_output(const Args& a, cudaStream_t st, bool output) {
-    cudaError_t e = launch_state_fwd(a, st);
+    cudaError_t e = state_fwd(a, st);
     if (e == cudaSuccess && output) e = launch_output(a, st);
     return e;
 }
@@ -178,7 +186,7 @@ cudaError_t run_bwd_prep(Args a, cudaStream_t st) {
     cudaError_t e = launch_intra_fwd(a, st);
     if (e != cudaSuccess) return e;
     a.S_out = nullptr;
-    e = launch_state_fwd(a, st);
+    e = state_fwd(a, st);
     if (e != cudaSuccess) return e;
     return launch_dd_pre(a, st);
 }
@@ -247,7 +255,7 @@ extern "C" {
 size_t sf_workspace_bytes(const sf_shape* s, int op) {
     if (check_shape(s) != SF_OK || (op != SF_OP_FWD && op != SF_OP_BWD)) return 0;
     // Whether beta is given is not known here: size for the delta rule (the superset).
-    return ws_layout(s->B, s->T, s->H, s->dk, s->dv, true, op == SF_OP_BWD, 1).total;
+    return ws_layout(s->B, s->T, s->H, s->dk, s->dv, s->dtype, true, op == SF_OP_BWD, 1).total;
 }
 
 size_t sf_seq_workspace_bytes(const sf_shape* s, int n_sub, const int* lens, int op) {
@@ -261,7 +269,7 @@ size_t sf_seq_workspace_bytes(const sf_shape* s, int n_sub, const int* lens, int
     }
     if (sum != s->T) return 0;
     const size_t states = 2 * (size_t)s->B * s->H * s->dk * s->dv * sizeof(float);
-    return ws_layout(s->B, lmax, s->H, s->dk, s->dv, true, op == SF_OP_BWD, 2).total + states;
+    return ws_layout(s->B, lmax, s->H, s->dk, s->dv, s->dtype, true, op == SF_OP_BWD, 2).total + states;
 }
 
 sf_status sf_fwd(const sf_shape* s, const void* q, const void* k, const void* v, const float* g,
@@ -277,7 +285,7 @@ sf_status sf_fwd(const sf_shape* s, const void* q, const void* k, const void* v,
                     {q, k, v, o}, {g, beta, S_in, S_out});
     if (st != SF_OK) return st;
     if (!work) return cuda_status(copy_state(S_out, S_in, nstate, cs));
-    const WsLayout L = ws_layout(s->B, s->T, s->H, s->dk, s->dv, beta != nullptr, false, 1);
+    const WsLayout L = ws_layout(s->B, s->T, s->H, s->dk, s->dv, s->dtype, beta != nullptr, false, 1);
     if (!ws || ws_bytes < L.total || !aligned(ws, 256)) return SF_ERR_WORKSPACE;
     Args a = make_args(s);
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S_in = S_in; a.o = o; a.S_out = S_out;
@@ -303,7 +311,7 @@ sf_status sf_bwd(const sf_shape* s, const void* q, const void* k, const void* v,
                     {q, k, v, dO, dq, dk, dv}, {g, beta, S_in, dS_out, dg, dbeta, dS_in});
     if (st != SF_OK) return st;
     if (!work) return cuda_status(copy_state(dS_in, dS_out, nstate, cs));
-    const WsLayout L = ws_layout(s->B, s->T, s->H, s->dk, s->dv, beta != nullptr, true, 1);
+    const WsLayout L = ws_layout(s->B, s->T, s->H, s->dk, s->dv, s->dtype, beta != nullptr, true, 1);
     if (!ws || ws_bytes < L.total || !aligned(ws, 256)) return SF_ERR_WORKSPACE;
     Args a = make_args(s);
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S_in = S_in; a.dO = dO;
@@ -332,7 +340,7 @@ sf_status sf_fwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
     if (st != SF_OK) return st;
     if (!work) return SF_OK;
     const size_t nstate = (size_t)s->B * s->H * s->dk * s->dv;
-    const WsLayout L = ws_layout(s->B, p.lmax, s->H, s->dk, s->dv, beta != nullptr, false, 2);
+    const WsLayout L = ws_layout(s->B, p.lmax, s->H, s->dk, s->dv, s->dtype, beta != nullptr, false, 2);
     const size_t need = L.total + 2 * nstate * sizeof(float);
     if (!ws || ws_bytes < need || !aligned(ws, 256)) return SF_ERR_WORKSPACE;
     float* pingpong = (float*)((char*)ws + L.total);
@@ -415,7 +423,7 @@ sf_status sf_bwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
     if (st != SF_OK) return st;
     if (!work) return SF_OK;
     const size_t nstate = (size_t)s->B * s->H * s->dk * s->dv;
-    const WsLayout L = ws_layout(s->B, p.lmax, s->H, s->dk, s->dv, beta != nullptr, true, 2);
+    const WsLayout L = ws_layout(s->B, p.lmax, s->H, s->dk, s->dv, s->dtype, beta != nullptr, true, 2);
     const size_t need = L.total + 2 * nstate * sizeof(float);
     if (!ws || ws_bytes < need || !aligned(ws, 256)) return SF_ERR_WORKSPACE;
     float* pingpong = (float*)((char*)ws + L.total);

@@ -33,29 +33,32 @@ struct Args {
     float* dg;
     float* dbeta;
     float* dS_in;        // may be null
-    // workspace (fp32, per (b,h) contiguous, TP = NC * 64 padded tokens)
-    float* G;     // [BH][TP]          chunk-local inclusive cumsum of g
-    float* W;     // [BH][TP][dk]      T diag(beta*gamma) K            (delta rule)
-    float* U;     // [BH][TP][dv]      T diag(beta) V                  (delta rule)
-    float* Sc;    // [BH][NC][dk][dv]  state entering each chunk
-    float* D;     // [BH][TP][dv]      Delta = U - W S_c (V for linear attention)
-    float* dD;    // [BH][TP][dv]      dL/dDelta
-    float* dSc;   // [BH][NC][dk][dv]  dL/d(state leaving each chunk)
-    float* dKp;   // [BH][TP][dk]      delta-rule part of dk
-    float* dGp;   // [BH][TP]          delta-rule part of dG
+    // Workspace.  Intermediates have element type TW = float for fp32 I/O and
+    // bf16 for bf16 I/O; chunk-transposed tiles keep the 64 tokens of a chunk
+    // contiguous (TP = NC * 64 padded tokens).
+    float* G;     // [BH][TP]            fp32 chunk-local inclusive cumsum of g
+    void* Wt;     // [BH][NC][dk][64]    W^T per chunk, W = T diag(beta gamma) K   (delta rule)
+    void* Ut;     // [BH][NC][dv][64]    U^T per chunk, U = T diag(beta) V (V for linear attention)
+    void* Sc;     // [BH][NC][dv][dk]    S^T entering each chunk
+    void* Dt;     // [BH][NC][dv][64]    Delta^T per chunk (V^T for linear attention)
+    void* dDt;    // [BH][NC][dv][64]    dL/dDelta, transposed per chunk
+    void* dSc;    // [BH][NC][dv][dk]    (dL/dS leaving each chunk)^T
+    float* dKp;   // [BH][TP][dk]        fp32 delta-rule part of dk (SIMT gradient kernels)
+    float* dGp;   // [BH][TP]            fp32 delta-rule part of dG (SIMT gradient kernels)
     int* err;     // device error word
 };
 
 // Workspace carve-up for a piece of at most T tokens.
 struct WsLayout {
-    size_t G, W, U, Sc, D, dD, dSc, dKp, dGp;  // byte offsets inside one slot
+    size_t G, Wt, Ut, Sc, Dt, dDt, dSc, dKp, dGp;  // byte offsets inside one slot
     size_t slot_bytes;
     size_t total;  // err header + nslots * slot_bytes
 };
 
 constexpr size_t kErrBytes = 256;
 
-WsLayout ws_layout(int B, int T, int H, int dk, int dv, bool delta, bool bwd, int nslots);
+WsLayout ws_layout(int B, int T, int H, int dk, int dv, int dtype, bool delta, bool bwd,
+                   int nslots);
 void bind_slot(Args& a, void* ws, const WsLayout& L, int slot, bool bwd);
 
 // Kernel launchers (SIMT fp32 arithmetic; I/O in a.dtype).  Each returns the
@@ -67,6 +70,10 @@ cudaError_t launch_dd_pre(const Args& a, cudaStream_t s);
 cudaError_t launch_state_bwd(const Args& a, cudaStream_t s);
 cudaError_t launch_grad_delta(const Args& a, cudaStream_t s);
 cudaError_t launch_grad_attn(const Args& a, cudaStream_t s);
+
+// Tensor-core kernels (sm_100a tcgen05/TMEM/TMA; bf16, d_k = d_v = 128).
+bool tc_eligible(const Args& a);
+cudaError_t launch_state_fwd_tc(const Args& a, cudaStream_t s);
 
 // Per-kernel timing registry (sf_timing_*).
 enum KernelKind {

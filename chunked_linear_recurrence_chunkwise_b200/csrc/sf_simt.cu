@@ -40,6 +40,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "sf_internal.h"
 #include "../../include/sf.h"
 
@@ -48,6 +50,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kNT = 32;  // d_v columns per CTA in the state passes
+constexpr int kNTp = kNT + 1;
 
 __device__ __forceinline__ float ldf(const float* p) { return *p; }
 __device__ __forceinline__ float ldf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
@@ -56,6 +59,14 @@ __device__ __forceinline__ void stf(__nv_bfloat16* p, float x) { *p = __float2bf
 
 __device__ __forceinline__ size_t tok(const Args& a, int b, int t, int h) {
     return ((size_t)b * a.ld_t + t) * a.H + h;
+}
+// [BH][NC][d][64] chunk-transposed tile element (x, r)
+__device__ __forceinline__ size_t ct(const Args& a, int bh, int c, int d, int x, int r) {
+    return (((size_t)bh * a.NC + c) * d + x) * kChunk + r;
+}
+// [BH][NC][dv][dk] transposed chunk state element (j, i)
+__device__ __forceinline__ size_t st(const Args& a, int bh, int c, int j, int i) {
+    return (((size_t)bh * a.NC + c) * a.dv + j) * a.dk + i;
 }
 
 // Loads the chunk's g into Gs and turns it into the inclusive cumsum (or zeros).
@@ -78,31 +89,47 @@ __device__ void load_cumsum(const Args& a, int b, int h, int t0, int L, float* G
 // rows [0, 64) of a token-major [.., H, d] tensor into smem [64][ld], zero past L
 template <typename TIO>
 __device__ void load_rows(const Args& a, const TIO* base, int d, int b, int h, int t0, int L,
-                          float* dst, int ld, float scale_unused = 1.f) {
+                          float* dst, int ld) {
     for (int e = threadIdx.x; e < kChunk * d; e += blockDim.x) {
         const int r = e / d, i = e - r * d;
         dst[r * ld + i] = (r < L) ? ldf(base + tok(a, b, t0 + r, h) * d + i) : 0.f;
     }
 }
 
+// chunk-transposed tile [d][64] (global, TW) -> smem [64][ld] (row r, column x)
+template <typename TW>
+__device__ void load_ct(const TW* src, int d, float* dst, int ld) {
+    for (int e = threadIdx.x; e < d * kChunk; e += blockDim.x) {
+        const int x = e >> 6, r = e & 63;
+        dst[r * ld + x] = ldf(src + e);
+    }
+}
+
 // ---------------------------------------------------------------- intra fwd
-// Grid (NC, H, B).  Writes G; with beta also W and U.
-template <typename TIO>
+// Grid (NC, H, B).  Writes G and U^T; with beta also W^T.
+template <typename TIO, typename TW>
 __global__ void __launch_bounds__(kThreads) intra_fwd_kernel(Args a) {
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int bh = b * a.H + h, TP = a.NC * kChunk;
     const int t0 = c * kChunk, L = min(kChunk, a.T - t0);
-    const int dk = a.dk, dv = a.dv, nc = dk + dv;
+    const int dk = a.dk, dv = a.dv, nc = dk + dv, ldx = nc + 1;
     extern __shared__ float sm[];
     float* Gs = sm;
     float* bs = Gs + kChunk;
     float* Ks = bs + kChunk;            // [64][dk+1]
-    float* X = Ks + kChunk * (dk + 1);  // [64][dk+dv]
-    float* As = X + kChunk * nc;        // [64][64]
+    float* X = Ks + kChunk * (dk + 1);  // [64][dk+dv+1]
+    float* As = X + kChunk * ldx;       // [64][64]
 
     load_cumsum(a, b, h, t0, L, Gs);
     if (threadIdx.x < kChunk) a.G[(size_t)bh * TP + t0 + threadIdx.x] = Gs[threadIdx.x];
-    if (!a.beta) return;
+    if (!a.beta) {  // linear attention: U = V (stored transposed like the delta rule's U)
+        for (int e = threadIdx.x; e < dv * kChunk; e += blockDim.x) {
+            const int j = e >> 6, r = e & 63;
+            const float x = (r < L) ? ldf((const TIO*)a.v + tok(a, b, t0 + r, h) * dv + j) : 0.f;
+            stf((TW*)a.Ut + ct(a, bh, c, dv, j, r), x);
+        }
+        return;
+    }
     if (threadIdx.x < kChunk) {
         const int r = threadIdx.x;
         bs[r] = (r < L) ? a.beta[tok(a, b, t0 + r, h)] : 0.f;
@@ -110,7 +137,7 @@ __global__ void __launch_bounds__(kThreads) intra_fwd_kernel(Args a) {
     load_rows(a, (const TIO*)a.k, dk, b, h, t0, L, Ks, dk + 1);
     for (int e = threadIdx.x; e < kChunk * dv; e += blockDim.x) {
         const int r = e / dv, j = e - r * dv;
-        X[r * nc + dk + j] = (r < L) ? ldf((const TIO*)a.v + tok(a, b, t0 + r, h) * dv + j) : 0.f;
+        X[r * ldx + dk + j] = (r < L) ? ldf((const TIO*)a.v + tok(a, b, t0 + r, h) * dv + j) : 0.f;
     }
     __syncthreads();
     for (int e = threadIdx.x; e < kChunk * kChunk; e += blockDim.x) {
@@ -126,55 +153,59 @@ __global__ void __launch_bounds__(kThreads) intra_fwd_kernel(Args a) {
     for (int e = threadIdx.x; e < kChunk * nc; e += blockDim.x) {
         const int r = e / nc, col = e - r * nc;
         if (col < dk)
-            X[e] = bs[r] * __expf(Gs[r]) * Ks[r * (dk + 1) + col];
+            X[r * ldx + col] = bs[r] * __expf(Gs[r]) * Ks[r * (dk + 1) + col];
         else
-            X[e] *= bs[r];
+            X[r * ldx + col] *= bs[r];
     }
     __syncthreads();
     // (I + A) X = RHS by forward substitution; each thread owns whole columns.
     for (int col = threadIdx.x; col < nc; col += blockDim.x) {
         for (int r = 1; r < kChunk; ++r) {
-            float acc = X[r * nc + col];
-            for (int i = 0; i < r; ++i) acc -= As[r * kChunk + i] * X[i * nc + col];
-            X[r * nc + col] = acc;
+            float acc = X[r * ldx + col];
+            for (int i = 0; i < r; ++i) acc -= As[r * kChunk + i] * X[i * ldx + col];
+            X[r * ldx + col] = acc;
         }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < kChunk * dk; e += blockDim.x) {
-        const int r = e / dk, i = e - r * dk;
-        a.W[((size_t)bh * TP + t0 + r) * dk + i] = X[r * nc + i];
+    TW* Wt = (TW*)a.Wt;
+    TW* Ut = (TW*)a.Ut;
+    for (int e = threadIdx.x; e < dk * kChunk; e += blockDim.x) {
+        const int i = e >> 6, r = e & 63;
+        stf(Wt + ct(a, bh, c, dk, i, r), X[r * ldx + i]);
     }
-    for (int e = threadIdx.x; e < kChunk * dv; e += blockDim.x) {
-        const int r = e / dv, j = e - r * dv;
-        a.U[((size_t)bh * TP + t0 + r) * dv + j] = X[r * nc + dk + j];
+    for (int e = threadIdx.x; e < dv * kChunk; e += blockDim.x) {
+        const int j = e >> 6, r = e & 63;
+        stf(Ut + ct(a, bh, c, dv, j, r), X[r * ldx + dk + j]);
     }
 }
 
 // ---------------------------------------------------------------- state fwd
 // Grid (ceil(dv / 32), H, B).  Sequential over chunks; S tile [dk][32] in smem.
-template <typename TIO>
+template <typename TIO, typename TW>
 __global__ void __launch_bounds__(kThreads) state_fwd_kernel(Args a) {
     const int h = blockIdx.y, b = blockIdx.z;
     const int bh = b * a.H + h, TP = a.NC * kChunk;
     const int dk = a.dk, dv = a.dv;
     const int n0 = blockIdx.x * kNT, nt = min(kNT, dv - n0);
     extern __shared__ float sm[];
-    float* Ss = sm;                      // [dk][32]
-    float* Gs = Ss + kMaxD * kNT;        // [64]
-    float* Us = Gs + kChunk;             // [64][32]  U tile, then Delta
-    float* Kt = Us + kChunk * kNT;       // [64][dk+1]
+    float* Ss = sm;                      // [dk][33]
+    float* Gs = Ss + kMaxD * kNTp;       // [64]
+    float* Us = Gs + kChunk;             // [64][33]  U tile, then Delta
+    float* Kt = Us + kChunk * kNTp;      // [64][dk+1]
     float* Ws = Kt + kChunk * (dk + 1);  // [64][dk+1]
+    TW* Sc = (TW*)a.Sc;
+    TW* Dt = (TW*)a.Dt;
 
     for (int e = threadIdx.x; e < dk * kNT; e += blockDim.x) {
         const int i = e / kNT, n = e - i * kNT;
-        Ss[e] = (a.S_in && n < nt) ? a.S_in[((size_t)bh * dk + i) * dv + n0 + n] : 0.f;
+        Ss[i * kNTp + n] = (a.S_in && n < nt) ? a.S_in[((size_t)bh * dk + i) * dv + n0 + n] : 0.f;
     }
     for (int c = 0; c < a.NC; ++c) {
         const int t0 = c * kChunk, L = min(kChunk, a.T - t0);
         __syncthreads();
-        for (int e = threadIdx.x; e < dk * kNT; e += blockDim.x) {
-            const int i = e / kNT, n = e - i * kNT;
-            if (n < nt) a.Sc[(((size_t)bh * a.NC + c) * dk + i) * dv + n0 + n] = Ss[e];
+        for (int e = threadIdx.x; e < nt * dk; e += blockDim.x) {
+            const int n = e / dk, i = e - n * dk;
+            stf(Sc + st(a, bh, c, n0 + n, i), Ss[i * kNTp + n]);
         }
         if (threadIdx.x < kChunk) Gs[threadIdx.x] = a.G[(size_t)bh * TP + t0 + threadIdx.x];
         __syncthreads();
@@ -184,73 +215,74 @@ __global__ void __launch_bounds__(kThreads) state_fwd_kernel(Args a) {
             Kt[r * (dk + 1) + i] =
                 (r < L) ? ldf((const TIO*)a.k + tok(a, b, t0 + r, h) * dk + i) * __expf(gC - Gs[r])
                         : 0.f;
-            if (a.beta) Ws[r * (dk + 1) + i] = a.W[((size_t)bh * TP + t0 + r) * dk + i];
         }
-        for (int e = threadIdx.x; e < kChunk * kNT; e += blockDim.x) {
-            const int r = e / kNT, n = e - r * kNT;
+        if (a.beta) load_ct((const TW*)a.Wt + ct(a, bh, c, dk, 0, 0), dk, Ws, dk + 1);
+        for (int e = threadIdx.x; e < kNT * kChunk; e += blockDim.x) {
+            const int n = e >> 6, r = e & 63;
             float u = 0.f;
             if (n < nt) {
                 if (a.beta)
-                    u = a.U[((size_t)bh * TP + t0 + r) * dv + n0 + n];
+                    u = ldf((const TW*)a.Ut + ct(a, bh, c, dv, n0 + n, r));
                 else if (r < L)
                     u = ldf((const TIO*)a.v + tok(a, b, t0 + r, h) * dv + n0 + n);
             }
-            Us[e] = u;
+            Us[r * kNTp + n] = u;
         }
         __syncthreads();
         if (a.beta) {
             for (int e = threadIdx.x; e < kChunk * kNT; e += blockDim.x) {
                 const int r = e / kNT, n = e - r * kNT;
-                float acc = Us[e];
-                for (int i = 0; i < dk; ++i) acc -= Ws[r * (dk + 1) + i] * Ss[i * kNT + n];
-                Us[e] = acc;
+                float acc = Us[r * kNTp + n];
+                for (int i = 0; i < dk; ++i) acc -= Ws[r * (dk + 1) + i] * Ss[i * kNTp + n];
+                Us[r * kNTp + n] = acc;
             }
             __syncthreads();
         }
-        for (int e = threadIdx.x; e < kChunk * kNT; e += blockDim.x) {
-            const int r = e / kNT, n = e - r * kNT;
-            if (n < nt) a.D[((size_t)bh * TP + t0 + r) * dv + n0 + n] = Us[e];
+        for (int e = threadIdx.x; e < nt * kChunk; e += blockDim.x) {
+            const int n = e >> 6, r = e & 63;
+            stf(Dt + ct(a, bh, c, dv, n0 + n, r), Us[r * kNTp + n]);
         }
         const float gamC = __expf(gC);
         for (int e = threadIdx.x; e < dk * kNT; e += blockDim.x) {
             const int i = e / kNT, n = e - i * kNT;
-            float acc = gamC * Ss[e];
-            for (int r = 0; r < kChunk; ++r) acc += Kt[r * (dk + 1) + i] * Us[r * kNT + n];
-            Ss[e] = acc;
+            float acc = gamC * Ss[i * kNTp + n];
+            for (int r = 0; r < kChunk; ++r) acc += Kt[r * (dk + 1) + i] * Us[r * kNTp + n];
+            Ss[i * kNTp + n] = acc;
         }
     }
     __syncthreads();
     if (a.S_out) {
         for (int e = threadIdx.x; e < dk * kNT; e += blockDim.x) {
             const int i = e / kNT, n = e - i * kNT;
-            if (n < nt) a.S_out[((size_t)bh * dk + i) * dv + n0 + n] = Ss[e];
+            if (n < nt) a.S_out[((size_t)bh * dk + i) * dv + n0 + n] = Ss[i * kNTp + n];
         }
     }
 }
 
 // ---------------------------------------------------------------- output
 // Grid (NC, H, B).  O = diag(gamma) Q S_c + P Delta.
-template <typename TIO>
+template <typename TIO, typename TW>
 __global__ void __launch_bounds__(kThreads) output_kernel(Args a) {
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int bh = b * a.H + h, TP = a.NC * kChunk;
     const int t0 = c * kChunk, L = min(kChunk, a.T - t0);
-    const int dk = a.dk, dv = a.dv;
+    const int dk = a.dk, dv = a.dv, ldv = dv + 1;
     extern __shared__ float sm[];
     float* Gs = sm;
     float* Qs = Gs + kChunk;             // [64][dk+1]
     float* Ks = Qs + kChunk * (dk + 1);  // [64][dk+1]
     float* Ps = Ks + kChunk * (dk + 1);  // [64][64]
-    float* Ss = Ps + kChunk * kChunk;    // [dk][dv]
-    float* Ds = Ss + dk * dv;            // [64][dv]
+    float* Ss = Ps + kChunk * kChunk;    // [dk][dv+1]
+    float* Ds = Ss + dk * ldv;           // [64][dv+1]
 
     if (threadIdx.x < kChunk) Gs[threadIdx.x] = a.G[(size_t)bh * TP + t0 + threadIdx.x];
     load_rows(a, (const TIO*)a.q, dk, b, h, t0, L, Qs, dk + 1);
     load_rows(a, (const TIO*)a.k, dk, b, h, t0, L, Ks, dk + 1);
-    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x)
-        Ss[e] = a.Sc[((size_t)bh * a.NC + c) * dk * dv + e];
-    for (int e = threadIdx.x; e < kChunk * dv; e += blockDim.x)
-        Ds[e] = a.D[((size_t)bh * TP + t0) * dv + e];
+    for (int e = threadIdx.x; e < dv * dk; e += blockDim.x) {
+        const int j = e / dk, i = e - j * dk;
+        Ss[i * ldv + j] = ldf((const TW*)a.Sc + st(a, bh, c, 0, 0) + e);
+    }
+    load_ct((const TW*)a.Dt + ct(a, bh, c, dv, 0, 0), dv, Ds, ldv);
     __syncthreads();
     for (int e = threadIdx.x; e < kChunk * kChunk; e += blockDim.x) {
         const int r = e >> 6, i = e & 63;
@@ -268,16 +300,16 @@ __global__ void __launch_bounds__(kThreads) output_kernel(Args a) {
         const int r = e / dv, n = e - r * dv;
         if (r >= L) continue;
         float qs = 0.f;
-        for (int i = 0; i < dk; ++i) qs += Qs[r * (dk + 1) + i] * Ss[i * dv + n];
+        for (int i = 0; i < dk; ++i) qs += Qs[r * (dk + 1) + i] * Ss[i * ldv + n];
         float pd = 0.f;
-        for (int i = 0; i <= r; ++i) pd += Ps[r * kChunk + i] * Ds[i * dv + n];
+        for (int i = 0; i <= r; ++i) pd += Ps[r * kChunk + i] * Ds[i * ldv + n];
         stf(o + tok(a, b, t0 + r, h) * dv + n, __expf(Gs[r]) * qs + pd);
     }
 }
 
 // ---------------------------------------------------------------- dDelta pre
-// Grid (NC, H, B).  dD = P^T dO (the part of dDelta that does not need dS).
-template <typename TIO>
+// Grid (NC, H, B).  dDelta^T = (P^T dO)^T, the part of dDelta that does not need dS.
+template <typename TIO, typename TW>
 __global__ void __launch_bounds__(kThreads) dd_pre_kernel(Args a) {
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int bh = b * a.H + h, TP = a.NC * kChunk;
@@ -306,41 +338,45 @@ __global__ void __launch_bounds__(kThreads) dd_pre_kernel(Args a) {
         Ps[e] = val;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < kChunk * dv; e += blockDim.x) {
-        const int i = e / dv, n = e - i * dv;
+    TW* dDt = (TW*)a.dDt;
+    for (int e = threadIdx.x; e < dv * kChunk; e += blockDim.x) {
+        const int n = e >> 6, i = e & 63;
         float acc = 0.f;
         for (int r = i; r < kChunk; ++r) acc += Ps[r * kChunk + i] * dOs[r * dv + n];
-        a.dD[((size_t)bh * TP + t0 + i) * dv + n] = acc;
+        stf(dDt + ct(a, bh, c, dv, n, i), acc);
     }
 }
 
 // ---------------------------------------------------------------- state bwd
 // Grid (ceil(dv / 32), H, B).  Reverse pass over chunks carrying dS [dk][32].
-template <typename TIO>
+template <typename TIO, typename TW>
 __global__ void __launch_bounds__(kThreads) state_bwd_kernel(Args a) {
     const int h = blockIdx.y, b = blockIdx.z;
     const int bh = b * a.H + h, TP = a.NC * kChunk;
     const int dk = a.dk, dv = a.dv;
     const int n0 = blockIdx.x * kNT, nt = min(kNT, dv - n0);
     extern __shared__ float sm[];
-    float* dSs = sm;                     // [dk][32]
-    float* Gs = dSs + kMaxD * kNT;       // [64]
-    float* dOs = Gs + kChunk;            // [64][32]
-    float* dDs = dOs + kChunk * kNT;     // [64][32]
-    float* Kt = dDs + kChunk * kNT;      // [64][dk+1]
+    float* dSs = sm;                     // [dk][33]
+    float* Gs = dSs + kMaxD * kNTp;      // [64]
+    float* dOs = Gs + kChunk;            // [64][33]
+    float* dDs = dOs + kChunk * kNTp;    // [64][33]
+    float* Kt = dDs + kChunk * kNTp;     // [64][dk+1]
     float* Qg = Kt + kChunk * (dk + 1);  // [64][dk+1]
     float* Ws = Qg + kChunk * (dk + 1);  // [64][dk+1]
+    TW* dSc = (TW*)a.dSc;
+    TW* dDt = (TW*)a.dDt;
 
     for (int e = threadIdx.x; e < dk * kNT; e += blockDim.x) {
         const int i = e / kNT, n = e - i * kNT;
-        dSs[e] = (a.dS_out && n < nt) ? a.dS_out[((size_t)bh * dk + i) * dv + n0 + n] : 0.f;
+        dSs[i * kNTp + n] =
+            (a.dS_out && n < nt) ? a.dS_out[((size_t)bh * dk + i) * dv + n0 + n] : 0.f;
     }
     for (int c = a.NC - 1; c >= 0; --c) {
         const int t0 = c * kChunk, L = min(kChunk, a.T - t0);
         __syncthreads();
-        for (int e = threadIdx.x; e < dk * kNT; e += blockDim.x) {
-            const int i = e / kNT, n = e - i * kNT;
-            if (n < nt) a.dSc[(((size_t)bh * a.NC + c) * dk + i) * dv + n0 + n] = dSs[e];
+        for (int e = threadIdx.x; e < nt * dk; e += blockDim.x) {
+            const int n = e / dk, i = e - n * dk;
+            stf(dSc + st(a, bh, c, n0 + n, i), dSs[i * kNTp + n]);
         }
         if (threadIdx.x < kChunk) Gs[threadIdx.x] = a.G[(size_t)bh * TP + t0 + threadIdx.x];
         __syncthreads();
@@ -350,45 +386,47 @@ __global__ void __launch_bounds__(kThreads) state_bwd_kernel(Args a) {
             const size_t ti = tok(a, b, t0 + r, h) * dk + i;
             Kt[r * (dk + 1) + i] = (r < L) ? ldf((const TIO*)a.k + ti) * __expf(gC - Gs[r]) : 0.f;
             Qg[r * (dk + 1) + i] = (r < L) ? ldf((const TIO*)a.q + ti) * __expf(Gs[r]) : 0.f;
-            if (a.beta) Ws[r * (dk + 1) + i] = a.W[((size_t)bh * TP + t0 + r) * dk + i];
         }
-        for (int e = threadIdx.x; e < kChunk * kNT; e += blockDim.x) {
-            const int r = e / kNT, n = e - r * kNT;
+        if (a.beta) load_ct((const TW*)a.Wt + ct(a, bh, c, dk, 0, 0), dk, Ws, dk + 1);
+        for (int e = threadIdx.x; e < kNT * kChunk; e += blockDim.x) {
+            const int n = e >> 6, r = e & 63;
             float x = 0.f, y = 0.f;
             if (n < nt) {
                 if (r < L) x = ldf((const TIO*)a.dO + tok(a, b, t0 + r, h) * dv + n0 + n);
-                y = a.dD[((size_t)bh * TP + t0 + r) * dv + n0 + n];
+                y = ldf(dDt + ct(a, bh, c, dv, n0 + n, r));
             }
-            dOs[e] = x;
-            dDs[e] = y;
+            dOs[r * kNTp + n] = x;
+            dDs[r * kNTp + n] = y;
         }
         __syncthreads();
         for (int e = threadIdx.x; e < kChunk * kNT; e += blockDim.x) {
             const int r = e / kNT, n = e - r * kNT;
-            float acc = dDs[e];
-            for (int i = 0; i < dk; ++i) acc += Kt[r * (dk + 1) + i] * dSs[i * kNT + n];
-            dDs[e] = acc;
-            if (n < nt) {
-                a.dD[((size_t)bh * TP + t0 + r) * dv + n0 + n] = acc;
-                if (!a.beta && r < L) stf((TIO*)a.dv_ + tok(a, b, t0 + r, h) * dv + n0 + n, acc);
-            }
+            float acc = dDs[r * kNTp + n];
+            for (int i = 0; i < dk; ++i) acc += Kt[r * (dk + 1) + i] * dSs[i * kNTp + n];
+            dDs[r * kNTp + n] = acc;
+            if (!a.beta && n < nt && r < L)
+                stf((TIO*)a.dv_ + tok(a, b, t0 + r, h) * dv + n0 + n, acc);
         }
         __syncthreads();
+        for (int e = threadIdx.x; e < nt * kChunk; e += blockDim.x) {
+            const int n = e >> 6, r = e & 63;
+            stf(dDt + ct(a, bh, c, dv, n0 + n, r), dDs[r * kNTp + n]);
+        }
         const float gamC = __expf(gC);
         for (int e = threadIdx.x; e < dk * kNT; e += blockDim.x) {
             const int i = e / kNT, n = e - i * kNT;
-            float acc = gamC * dSs[e];
-            for (int r = 0; r < kChunk; ++r) acc += Qg[r * (dk + 1) + i] * dOs[r * kNT + n];
+            float acc = gamC * dSs[i * kNTp + n];
+            for (int r = 0; r < kChunk; ++r) acc += Qg[r * (dk + 1) + i] * dOs[r * kNTp + n];
             if (a.beta)
-                for (int r = 0; r < kChunk; ++r) acc -= Ws[r * (dk + 1) + i] * dDs[r * kNT + n];
-            dSs[e] = acc;
+                for (int r = 0; r < kChunk; ++r) acc -= Ws[r * (dk + 1) + i] * dDs[r * kNTp + n];
+            dSs[i * kNTp + n] = acc;
         }
     }
     __syncthreads();
     if (a.dS_in) {
         for (int e = threadIdx.x; e < dk * kNT; e += blockDim.x) {
             const int i = e / kNT, n = e - i * kNT;
-            if (n < nt) a.dS_in[((size_t)bh * dk + i) * dv + n0 + n] = dSs[e];
+            if (n < nt) a.dS_in[((size_t)bh * dk + i) * dv + n0 + n] = dSs[i * kNTp + n];
         }
     }
 }
@@ -396,7 +434,7 @@ __global__ void __launch_bounds__(kThreads) state_bwd_kernel(Args a) {
 // ---------------------------------------------------------------- grad delta
 // Grid (NC, H, B), delta rule only.  Writes dv, dbeta and the delta-rule parts
 // of dk (dKp) and dG (dGp).
-template <typename TIO>
+template <typename TIO, typename TW>
 __global__ void __launch_bounds__(kThreads) grad_delta_kernel(Args a) {
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int bh = b * a.H + h, TP = a.NC * kChunk;
@@ -425,10 +463,7 @@ __global__ void __launch_bounds__(kThreads) grad_delta_kernel(Args a) {
         red[r] = 0.f;
     }
     load_rows(a, (const TIO*)a.k, dk, b, h, t0, L, Ks, ldk);
-    for (int e = threadIdx.x; e < kChunk * dv; e += blockDim.x) {
-        const int r = e / dv, n = e - r * dv;
-        dDs[r * ldv + n] = a.dD[((size_t)bh * TP + t0 + r) * dv + n];
-    }
+    load_ct((const TW*)a.dDt + ct(a, bh, c, dv, 0, 0), dv, dDs, ldv);
     __syncthreads();
     for (int e = threadIdx.x; e < kChunk * kChunk; e += blockDim.x) {
         const int r = e >> 6, i = e & 63;
@@ -461,12 +496,12 @@ __global__ void __launch_bounds__(kThreads) grad_delta_kernel(Args a) {
     __syncthreads();
     float* dVh = R;                  // [64][dv+1]
     float* Us = R + kChunk * ldv;    // [64][dv+1]
+    load_ct((const TW*)a.Ut + ct(a, bh, c, dv, 0, 0), dv, Us, ldv);
     for (int e = threadIdx.x; e < kChunk * dv; e += blockDim.x) {
         const int r = e / dv, n = e - r * dv;
         float acc = 0.f;
         for (int i = r; i < kChunk; ++i) acc += Ts[i * kChunk + r] * dDs[i * ldv + n];
         dVh[r * ldv + n] = acc;
-        Us[r * ldv + n] = a.U[((size_t)bh * TP + t0 + r) * dv + n];
         if (r < L) {
             const size_t ti = tok(a, b, t0 + r, h) * dv + n;
             stf((TIO*)a.dv_ + ti, bs[r] * acc);
@@ -482,10 +517,10 @@ __global__ void __launch_bounds__(kThreads) grad_delta_kernel(Args a) {
         dAs[e] = acc;
     }
     __syncthreads();
-    float* Ss = R;  // [dk][dv+1]
-    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
-        const int i = e / dv, n = e - i * dv;
-        Ss[i * ldv + n] = a.Sc[((size_t)bh * a.NC + c) * dk * dv + e];
+    float* Ss = R;  // [dk][dv+1], S[i][n]
+    for (int e = threadIdx.x; e < dv * dk; e += blockDim.x) {
+        const int n = e / dk, i = e - n * dk;
+        Ss[i * ldv + n] = ldf((const TW*)a.Sc + st(a, bh, c, 0, 0) + e);
     }
     __syncthreads();
     for (int e = threadIdx.x; e < kChunk * dk; e += blockDim.x) {
@@ -505,10 +540,7 @@ __global__ void __launch_bounds__(kThreads) grad_delta_kernel(Args a) {
     }
     __syncthreads();
     float* Wsm = R;  // [64][dk+1]
-    for (int e = threadIdx.x; e < kChunk * dk; e += blockDim.x) {
-        const int r = e / dk, i = e - r * dk;
-        Wsm[r * ldk + i] = a.W[((size_t)bh * TP + t0 + r) * dk + i];
-    }
+    load_ct((const TW*)a.Wt + ct(a, bh, c, dk, 0, 0), dk, Wsm, ldk);
     __syncthreads();
     for (int e = threadIdx.x; e < kChunk * kChunk; e += blockDim.x) {
         const int r = e >> 6, i = e & 63;
@@ -552,7 +584,7 @@ __global__ void __launch_bounds__(kThreads) grad_delta_kernel(Args a) {
 
 // ---------------------------------------------------------------- grad attn
 // Grid (NC, H, B).  Writes dq, dk and dg.
-template <typename TIO>
+template <typename TIO, typename TW>
 __global__ void __launch_bounds__(kThreads) grad_attn_kernel(Args a) {
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int bh = b * a.H + h, TP = a.NC * kChunk;
@@ -571,6 +603,8 @@ __global__ void __launch_bounds__(kThreads) grad_attn_kernel(Args a) {
     float* R = Ds + kChunk * ldv;        // P, dP | S | dS'
     float* Ps = R;
     float* dPs = R + kChunk * kChunk;
+    const TW* Scg = (const TW*)a.Sc + st(a, bh, c, 0, 0);
+    const TW* dScg = (const TW*)a.dSc + st(a, bh, c, 0, 0);
 
     if (threadIdx.x < kChunk) {
         Gs[threadIdx.x] = a.G[(size_t)bh * TP + t0 + threadIdx.x];
@@ -580,10 +614,7 @@ __global__ void __launch_bounds__(kThreads) grad_attn_kernel(Args a) {
     load_rows(a, (const TIO*)a.q, dk, b, h, t0, L, Qs, ldk);
     load_rows(a, (const TIO*)a.k, dk, b, h, t0, L, Ks, ldk);
     load_rows(a, (const TIO*)a.dO, dv, b, h, t0, L, dOs, ldv);
-    for (int e = threadIdx.x; e < kChunk * dv; e += blockDim.x) {
-        const int r = e / dv, n = e - r * dv;
-        Ds[r * ldv + n] = a.D[((size_t)bh * TP + t0 + r) * dv + n];
-    }
+    load_ct((const TW*)a.Dt + ct(a, bh, c, dv, 0, 0), dv, Ds, ldv);
     __syncthreads();
     for (int e = threadIdx.x; e < kChunk * kChunk; e += blockDim.x) {
         const int r = e >> 6, i = e & 63;
@@ -629,10 +660,10 @@ __global__ void __launch_bounds__(kThreads) grad_attn_kernel(Args a) {
         }
     }
     __syncthreads();
-    float* Ss = R;  // [dk][dv+1]
-    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
-        const int i = e / dv, n = e - i * dv;
-        Ss[i * ldv + n] = a.Sc[((size_t)bh * a.NC + c) * dk * dv + e];
+    float* Ss = R;  // [dk][dv+1], S[i][n]
+    for (int e = threadIdx.x; e < dv * dk; e += blockDim.x) {
+        const int n = e / dk, i = e - n * dk;
+        Ss[i * ldv + n] = ldf(Scg + e);
     }
     __syncthreads();
 #pragma unroll
@@ -648,15 +679,13 @@ __global__ void __launch_bounds__(kThreads) grad_attn_kernel(Args a) {
         }
     }
     __syncthreads();
-    float* dSp = R;  // [dk][dv+1]
+    float* dSp = R;  // [dk][dv+1], dS'[i][n]
     float sdot = 0.f;
-    const float* Scg = a.Sc + ((size_t)bh * a.NC + c) * dk * dv;
-    const float* dScg = a.dSc + ((size_t)bh * a.NC + c) * dk * dv;
-    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
-        const int i = e / dv, n = e - i * dv;
-        const float x = dScg[e];
+    for (int e = threadIdx.x; e < dv * dk; e += blockDim.x) {
+        const int n = e / dk, i = e - n * dk;
+        const float x = ldf(dScg + e);
         dSp[i * ldv + n] = x;
-        sdot += x * Scg[e];
+        sdot += x * ldf(Scg + e);
     }
     atomicAdd(&scal[0], sdot);
     __syncthreads();
@@ -706,24 +735,27 @@ __global__ void __launch_bounds__(kThreads) grad_attn_kernel(Args a) {
 
 // ---------------------------------------------------------------- launchers
 size_t smem_intra(const Args& a) {
-    return sizeof(float) * (2 * kChunk + kChunk * (a.dk + 1) + kChunk * (a.dk + a.dv) + kChunk * kChunk);
+    return sizeof(float) *
+           (2 * kChunk + kChunk * (a.dk + 1) + kChunk * (a.dk + a.dv + 1) + kChunk * kChunk);
 }
 size_t smem_state_fwd(const Args& a) {
-    return sizeof(float) * (kMaxD * kNT + kChunk + kChunk * kNT + 2 * kChunk * (a.dk + 1));
+    return sizeof(float) * (kMaxD * kNTp + kChunk + kChunk * kNTp + 2 * kChunk * (a.dk + 1));
 }
 size_t smem_output(const Args& a) {
-    return sizeof(float) * (kChunk + 2 * kChunk * (a.dk + 1) + kChunk * kChunk + a.dk * a.dv + kChunk * a.dv);
+    return sizeof(float) * (kChunk + 2 * kChunk * (a.dk + 1) + kChunk * kChunk +
+                            a.dk * (a.dv + 1) + kChunk * (a.dv + 1));
 }
 size_t smem_dd_pre(const Args& a) {
     return sizeof(float) * (kChunk + 2 * kChunk * (a.dk + 1) + kChunk * kChunk + kChunk * a.dv);
 }
 size_t smem_state_bwd(const Args& a) {
-    return sizeof(float) * (kMaxD * kNT + kChunk + 2 * kChunk * kNT + 3 * kChunk * (a.dk + 1));
+    return sizeof(float) * (kMaxD * kNTp + kChunk + 2 * kChunk * kNTp + 3 * kChunk * (a.dk + 1));
 }
 size_t smem_grad_delta(const Args& a) {
     const int ldk = a.dk + 1, ldv = a.dv + 1;
     const int Rsize = std::max(2 * kChunk * ldv, std::max(a.dk * ldv, kChunk * ldk));
-    return sizeof(float) * (4 * kChunk + kChunk * ldk + 3 * kChunk * kChunk + kChunk * ldv + Rsize + kChunk * ldk);
+    return sizeof(float) *
+           (4 * kChunk + kChunk * ldk + 3 * kChunk * kChunk + kChunk * ldv + Rsize + kChunk * ldk);
 }
 size_t smem_grad_attn(const Args& a) {
     const int ldk = a.dk + 1, ldv = a.dv + 1;
@@ -748,9 +780,10 @@ dim3 tile_grid(const Args& a) { return dim3((a.dv + kNT - 1) / kNT, a.H, a.B); }
 
 }  // namespace
 
-#define SF_DISPATCH(KERNEL, KIND, GRID, SMEM)                                          \
-    (a.dtype == SF_BF16 ? launch(KERNEL<__nv_bfloat16>, KIND, GRID, SMEM, a, s)         \
-                        : launch(KERNEL<float>, KIND, GRID, SMEM, a, s))
+// bf16 I/O keeps bf16 intermediates; fp32 I/O keeps fp32 intermediates.
+#define SF_DISPATCH(KERNEL, KIND, GRID, SMEM)                                                   \
+    (a.dtype == SF_BF16 ? launch(KERNEL<__nv_bfloat16, __nv_bfloat16>, KIND, GRID, SMEM, a, s)   \
+                        : launch(KERNEL<float, float>, KIND, GRID, SMEM, a, s))
 
 cudaError_t launch_intra_fwd(const Args& a, cudaStream_t s) {
     return SF_DISPATCH(intra_fwd_kernel, KK_INTRA_FWD, chunk_grid(a), smem_intra(a));

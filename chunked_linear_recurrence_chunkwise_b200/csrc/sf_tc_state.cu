@@ -1,0 +1,340 @@
+// Tensor-core state-transition passes (sm_100a, bf16 operands, fp32 state).
+//
+// This is the low-latency state-transition kernel of the StateFlow summary
+// (gptget.net, section 方法详解: chunks joined by boundary states, a
+// low-latency state-transition kernel): sequential over the chunks of one
+// head, one CTA per (batch, head), the d_k x d_v state held on chip in fp32.
+//
+// The state is kept transposed, S^T (d_v rows = TMEM lanes, d_k columns), so
+// both per-chunk products are M = 128 UMMAs:
+//   X^T      = S^T W^T                    (128 x 64,  K = d_k)
+//   Delta^T  = U^T - X^T                   (threads, fp32)
+//   P^T      = (diag(e^{G_C - G}) Delta)^T K   (128 x 128, K = 64 tokens)
+//   S^T     <- gamma_C S^T + P^T            (threads, fp32 registers)
+// which is S' = gamma_C S + Ktil^T Delta with the decay moved from K onto
+// Delta (Ktil^T Delta = K^T diag(e^{G_C - G}) Delta), so K feeds the tensor
+// core straight from its TMA tile.  S^T is rounded to bf16 only as an MMA
+// operand (and for the stored chunk states); the carried state stays fp32.
+//
+// Per chunk c the kernel stores S^T entering c and Delta^T (both bf16) for
+// the output and gradient kernels.  W^T, U^T, K and the cumulative log-decay
+// of chunk c+1.. are prefetched by TMA into a 3-stage ring while chunk c runs.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "../../include/sf.h"
+#include "sf_internal.h"
+#include "tc_common.cuh"
+
+namespace sf {
+
+bool make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+               const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapDataType dtype,
+               CUtensorMapSwizzle swz) {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !p)
+            return false;
+        fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+    }
+    cuuint64_t d[5];
+    cuuint64_t st[4];
+    cuuint32_t bx[5], es[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        bx[i] = box[i];
+        es[i] = 1;
+        if (i + 1 < rank) st[i] = strides_bytes[i];
+    }
+    CUresult r = fn(map, dtype, (cuuint32_t)rank, const_cast<void*>(base), d, st, bx, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+namespace {
+
+using namespace tc;
+
+constexpr int kD = 128;                 // d_k = d_v on this path
+constexpr int kTile = 128 * 64 * 2;     // one 128-row x 128-byte bf16 tile (16 KB)
+constexpr int kStages = 3;
+
+// Shared-memory carve-up (byte offsets from a 1024-byte aligned base).
+struct FwdSmem {
+    static constexpr int Wt = 0;                          // [stage] W^T  [d_k][64 r]
+    static constexpr int Kt = Wt + kStages * kTile;       // [stage] K    [2][64 r][64 d_k]
+    static constexpr int Ut = Kt + kStages * kTile;       // [stage] U^T  [d_v][64 r]
+    static constexpr int St = Ut + kStages * kTile;       // S^T operand [2 kblk][d_v][64]
+    static constexpr int Dsc = St + 2 * kTile;            // (e^{G_C-G} Delta)^T operand
+    static constexpr int Dst = Dsc + kTile;               // Delta^T staging for the store
+    static constexpr int G = Dst + kTile;                 // [stage][64] fp32
+    static constexpr int Bar = G + kStages * 256;         // kStages load barriers + 1 MMA
+    static constexpr int Misc = Bar + (kStages + 1) * 8;  // TMEM base, abort flag
+    static constexpr int Size = Misc + 16;
+};
+
+template <bool kDelta>
+__global__ void __launch_bounds__(256, 1)
+    state_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_wt,
+                        const __grid_constant__ CUtensorMap tm_ut,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_sc,
+                        const __grid_constant__ CUtensorMap tm_dt, const Args a) {
+    using L = FwdSmem;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    float* Gs = (float*)(sm + L::G);
+    uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);
+    uint64_t* bar_mma = bar_ld + kStages;
+    uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
+    volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int j = quad * 32 + lane;  // d_v row = TMEM lane
+    const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+    const int NC = a.NC, TP = NC * kChunk;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&bar_ld[s], 1);
+        mbar_init(bar_mma, 1);
+        *s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc(s_tmem, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t tX = tmem, tP = tmem + 64;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+
+    auto issue_load = [&](int c) {  // thread 0
+        const int s = c % kStages;
+        const uint32_t bytes = (kDelta ? kTile : 0) + 2 * kTile + 256;
+        mbar_expect_tx(&bar_ld[s], bytes);
+        if (kDelta) tma_load_2d(sm + L::Wt + s * kTile, &tm_wt, 0, (bh * NC + c) * kD, &bar_ld[s]);
+        tma_load_2d(sm + L::Ut + s * kTile, &tm_ut, 0, (bh * NC + c) * kD, &bar_ld[s]);
+        tma_load_4d(sm + L::Kt + s * kTile, &tm_k, 0, h, c * kChunk, b, &bar_ld[s]);
+        tma_load_4d(sm + L::Kt + s * kTile + kTile / 2, &tm_k, 64, h, c * kChunk, b, &bar_ld[s]);
+        bulk_load(Gs + s * kChunk, a.G + (size_t)bh * TP + c * kChunk, 256, &bar_ld[s]);
+    };
+    int issued = 0;
+    if (tid == 0)
+        for (; issued < min(kStages, NC); ++issued) issue_load(issued);
+
+    // S^T row j, columns i in [64 half, 64 half + 64): S[q] = S_{i, j}
+    float S[64];
+#pragma unroll
+    for (int q = 0; q < 64; ++q)
+        S[q] = a.S_in ? a.S_in[((size_t)bh * kD + half * 64 + q) * kD + j] : 0.f;
+    uint8_t* St = sm + L::St + half * kTile;
+    auto write_state = [&]() {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            uint4 v;
+            v.x = pack_bf16(S[q * 8 + 0], S[q * 8 + 1]);
+            v.y = pack_bf16(S[q * 8 + 2], S[q * 8 + 3]);
+            v.z = pack_bf16(S[q * 8 + 4], S[q * 8 + 5]);
+            v.w = pack_bf16(S[q * 8 + 6], S[q * 8 + 7]);
+            *(uint4*)(St + sw128(j, q)) = v;
+        }
+    };
+    write_state();
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        tma_store_2d(&tm_sc, sm + L::St, 0, bh * NC * kD);
+        tma_store_2d(&tm_sc, sm + L::St + kTile, 64, bh * NC * kD);
+        bulk_commit();
+    }
+
+    uint32_t mma_phase = 0;
+    bool mma_pending = false;  // thread 0: an MMA commit whose wait timed out
+    int c = 0;
+    bool aborted = false;
+    for (; c < NC; ++c) {
+        const int s = c % kStages;
+        if (tid == 0) {
+            if (!mbar_wait(&bar_ld[s], (c / kStages) & 1)) {
+                *s_abort = 1;
+                atomicExch(a.err, kErrTimeoutTma);
+            } else if (kDelta) {
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(sm + L::St), b0 = smem_u32(sm + L::Wt + s * kTile);
+                constexpr uint32_t id = idesc_bf16(128, 64, false, true);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_bf16(tX, sdesc(a0 + (ks >> 2) * kTile + (ks & 3) * 32, 16, 1024),
+                             sdesc(b0 + ks * 2048, 8192, 1024), id, ks > 0);
+                mma_commit(bar_mma);
+                bulk_wait_read<1>();  // Delta^T staging of chunk c-1 has been read
+                if (!mbar_wait(bar_mma, mma_phase)) {
+                    *s_abort = 1;
+                    mma_pending = true;
+                    atomicExch(a.err, kErrTimeoutMma);
+                }
+            } else {
+                bulk_wait_read<1>();
+            }
+        }
+        if (kDelta) mma_phase ^= 1;
+        __syncthreads();
+        if (*s_abort) {
+            aborted = true;
+            break;
+        }
+        float X[32];
+        if (kDelta) {
+            tc_fence_after();
+            tmem_ld32(tX + lane_base + half * 32, X);
+            tmem_ld_wait();
+        } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) X[q] = 0.f;
+        }
+        const float* G = Gs + s * kChunk;
+        const float gC = G[kChunk - 1];
+        const uint8_t* Ut = sm + L::Ut + s * kTile;
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+            const int q = half * 4 + qq;  // tokens 8q .. 8q + 7
+            const uint4 u = *(const uint4*)(Ut + sw128(j, q));
+            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+            uint32_t dw[4], tw[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const float2 uf = unpack_bf16(uw[p]);
+                const int r0 = q * 8 + 2 * p;
+                const float d0 = uf.x - X[qq * 8 + 2 * p];
+                const float d1 = uf.y - X[qq * 8 + 2 * p + 1];
+                dw[p] = pack_bf16(d0, d1);
+                tw[p] = pack_bf16(d0 * __expf(gC - G[r0]), d1 * __expf(gC - G[r0 + 1]));
+            }
+            *(uint4*)(sm + L::Dst + sw128(j, q)) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+            *(uint4*)(sm + L::Dsc + sw128(j, q)) = make_uint4(tw[0], tw[1], tw[2], tw[3]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tma_store_2d(&tm_dt, sm + L::Dst, 0, (bh * NC + c) * kD);
+            bulk_commit();
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(sm + L::Dsc), b0 = smem_u32(sm + L::Kt + s * kTile);
+            constexpr uint32_t id = idesc_bf16(128, 128, false, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tP, sdesc(a0 + ks * 32, 16, 1024), sdesc(b0 + ks * 2048, 8192, 1024),
+                         id, ks > 0);
+            mma_commit(bar_mma);
+            bulk_wait_read<1>();  // the S^T store issued after chunk c-1 has been read
+            if (!mbar_wait(bar_mma, mma_phase)) {
+                *s_abort = 1;
+                mma_pending = true;
+                atomicExch(a.err, kErrTimeoutMma);
+            } else if (issued < NC) {
+                issue_load(issued);  // stage s is free again
+                ++issued;
+            }
+        }
+        mma_phase ^= 1;
+        __syncthreads();
+        if (*s_abort) {
+            aborted = true;
+            break;
+        }
+        tc_fence_after();
+        float P0[32], P1[32];
+        tmem_ld32(tP + lane_base + half * 64, P0);
+        tmem_ld32(tP + lane_base + half * 64 + 32, P1);
+        tmem_ld_wait();
+        const float gam = __expf(gC);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+            S[q] = gam * S[q] + P0[q];
+            S[32 + q] = gam * S[32 + q] + P1[q];
+        }
+        if (c + 1 < NC) {
+            write_state();
+            fence_async_smem();
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && c + 1 < NC) {
+            tma_store_2d(&tm_sc, sm + L::St, 0, (bh * NC + c + 1) * kD);
+            tma_store_2d(&tm_sc, sm + L::St + kTile, 64, (bh * NC + c + 1) * kD);
+            bulk_commit();
+        }
+    }
+    if (!aborted && a.S_out) {
+#pragma unroll
+        for (int q = 0; q < 64; ++q) a.S_out[((size_t)bh * kD + half * 64 + q) * kD + j] = S[q];
+    }
+    if (tid == 0) {
+        if (aborted) {
+            // let every copy and MMA this CTA started finish before it exits (bounded)
+            for (int cc = c; cc < issued; ++cc) mbar_wait(&bar_ld[cc % kStages], (cc / kStages) & 1);
+            if (mma_pending) mbar_wait(bar_mma, mma_phase ^ 1);
+        }
+        bulk_wait<0>();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+bool tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+    const uint64_t dims[2] = {inner, rows};
+    const uint64_t strides[1] = {inner * 2};
+    const uint32_t box[2] = {64, box_rows};
+    return make_tmap(m, base, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// [B, ld_t, H, d] token-major input, tiles of 64 tokens x 64 features of one head.
+bool tmap_tokens(CUtensorMap* m, const void* base, const Args& a, int d) {
+    const uint64_t dims[4] = {(uint64_t)d, (uint64_t)a.H, (uint64_t)a.T, (uint64_t)a.B};
+    const uint64_t strides[3] = {(uint64_t)d * 2, (uint64_t)a.H * d * 2,
+                                 (uint64_t)a.ld_t * a.H * d * 2};
+    const uint32_t box[4] = {64, 1, 64, 1};
+    return make_tmap(m, base, 4, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+}  // namespace
+
+bool tc_eligible(const Args& a) {
+    return a.dtype == SF_BF16 && a.dk == kD && a.dv == kD;
+}
+
+cudaError_t launch_state_fwd_tc(const Args& a, cudaStream_t s) {
+    const int BH = a.B * a.H;
+    if (BH == 0 || a.NC == 0) return cudaSuccess;
+    const uint64_t rows = (uint64_t)BH * a.NC * kD;
+    CUtensorMap tm_wt{}, tm_ut{}, tm_k{}, tm_sc{}, tm_dt{};
+    bool ok = tmap_2d(&tm_ut, a.Ut, 64, rows, 128) && tmap_tokens(&tm_k, a.k, a, kD) &&
+              tmap_2d(&tm_sc, a.Sc, kD, rows, 128) && tmap_2d(&tm_dt, a.Dt, 64, rows, 128);
+    if (a.beta) ok = ok && tmap_2d(&tm_wt, a.Wt, 64, rows, 128);
+    if (!ok) return cudaErrorInvalidValue;
+    const size_t smem = FwdSmem::Size + 1024;
+    auto kern = a.beta ? state_fwd_tc_kernel<true> : state_fwd_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    timing_begin(KK_STATE_FWD, s);
+    kern<<<BH, 256, smem, s>>>(tm_wt, tm_ut, tm_k, tm_sc, tm_dt, a);
+    e = cudaGetLastError();
+    timing_end(KK_STATE_FWD, s);
+    return e;
+}
+
+}  // namespace sf
