@@ -45,6 +45,7 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv, int dtype, bool delta, b
     L.Dt = take(BH * TP * dv * tw);
     L.dDt = take(bwd ? BH * TP * dv * tw : 0);
     L.dSc = take(bwd ? BH * NC * dk * dv * tw : 0);
+    L.Pm = take(bwd ? BH * NC * kChunk * kChunk * tw : 0);
     L.dKp = take(bwd && delta ? BH * TP * dk * 4 : 0);
     L.dGp = take(bwd && delta ? BH * TP * 4 : 0);
     L.slot_bytes = off;
@@ -61,6 +62,7 @@ void bind_slot(Args& a, void* ws, const WsLayout& L, int slot, bool bwd) {
     a.Dt = base + L.Dt;
     a.dDt = bwd ? (void*)(base + L.dDt) : nullptr;
     a.dSc = bwd ? (void*)(base + L.dSc) : nullptr;
+    a.Pm = bwd ? (void*)(base + L.Pm) : nullptr;
     a.dKp = bwd ? (float*)(base + L.dKp) : nullptr;
     a.dGp = bwd ? (float*)(base + L.dGp) : nullptr;
     a.err = (int*)ws;
@@ -171,19 +173,26 @@ cudaError_t state_fwd(const Args& a, cudaStream_t st) {
     return tc_eligible(a) ? launch_state_fwd_tc(a, st) : launch_state_fwd(a, st);
 }
 
-// The forward pieces of one call: intra (may go on its own stream), then state + output.
-cudaError_t run_intra(const Args& a, cudaStream_t st) { return launch_intra_fwd(a, st); }
+cudaError_t intra(const Args& a, bool with_p, cudaStream_t st) {
+    return tc_eligible(a) ? launch_intra_tc(a, with_p, st) : launch_intra_fwd(a, st);
+}
+cudaError_t output(const Args& a, cudaStream_t st) {
+    return tc_eligible(a) ? launch_output_tc(a, st) : launch_output(a, st);
+}
 
-cudaError_t run_state_output(const Args& a, cudaStream_t st, bool output) {
+// The forward pieces of one call: intra (may go on its own stream), then state + output.
+cudaError_t run_intra(const Args& a, cudaStream_t st) { return intra(a, false, st); }
+
+cudaError_t run_state_output(const Args& a, cudaStream_t st, bool with_output) {
     cudaError_t e = state_fwd(a, st);
-    if (e == cudaSuccess && output) e = launch_output(a, st);
+    if (e == cudaSuccess && with_output) e = output(a, st);
     return e;
 }
 
 // Everything of the backward of one piece that does not need dS: recompute of
 // the intra-chunk terms and the chunk states, and dDelta's P^T dO part.
 cudaError_t run_bwd_prep(Args a, cudaStream_t st) {
-    cudaError_t e = launch_intra_fwd(a, st);
+    cudaError_t e = intra(a, true, st);
     if (e != cudaSuccess) return e;
     a.S_out = nullptr;
     e = state_fwd(a, st);

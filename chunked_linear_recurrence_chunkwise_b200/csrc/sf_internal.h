@@ -43,6 +43,7 @@ struct Args {
     void* Dt;     // [BH][NC][dv][64]    Delta^T per chunk (V^T for linear attention)
     void* dDt;    // [BH][NC][dv][64]    dL/dDelta, transposed per chunk
     void* dSc;    // [BH][NC][dv][dk]    (dL/dS leaving each chunk)^T
+    void* Pm;     // [BH][NC][64][64]    P = (Q K^T) .* Gamma, lower incl. (backward)
     float* dKp;   // [BH][TP][dk]        fp32 delta-rule part of dk (SIMT gradient kernels)
     float* dGp;   // [BH][TP]            fp32 delta-rule part of dG (SIMT gradient kernels)
     int* err;     // device error word
@@ -50,7 +51,7 @@ struct Args {
 
 // Workspace carve-up for a piece of at most T tokens.
 struct WsLayout {
-    size_t G, Wt, Ut, Sc, Dt, dDt, dSc, dKp, dGp;  // byte offsets inside one slot
+    size_t G, Wt, Ut, Sc, Dt, dDt, dSc, Pm, dKp, dGp;  // byte offsets inside one slot
     size_t slot_bytes;
     size_t total;  // err header + nslots * slot_bytes
 };
@@ -74,6 +75,9 @@ cudaError_t launch_grad_attn(const Args& a, cudaStream_t s);
 // Tensor-core kernels (sm_100a tcgen05/TMEM/TMA; bf16, d_k = d_v = 128).
 bool tc_eligible(const Args& a);
 cudaError_t launch_state_fwd_tc(const Args& a, cudaStream_t s);
+// with_p: also store P (backward recompute)
+cudaError_t launch_intra_tc(const Args& a, bool with_p, cudaStream_t s);
+cudaError_t launch_output_tc(const Args& a, cudaStream_t s);
 
 // Per-kernel timing registry (sf_timing_*).
 enum KernelKind {

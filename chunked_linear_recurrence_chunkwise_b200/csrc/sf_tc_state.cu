@@ -293,6 +293,8 @@ __global__ void __launch_bounds__(256, 1)
     }
 }
 
+}  // namespace
+
 bool tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
     const uint64_t dims[2] = {inner, rows};
     const uint64_t strides[1] = {inner * 2};
@@ -310,8 +312,6 @@ bool tmap_tokens(CUtensorMap* m, const void* base, const Args& a, int d) {
     return make_tmap(m, base, 4, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                      CU_TENSOR_MAP_SWIZZLE_128B);
 }
-
-}  // namespace
 
 bool tc_eligible(const Args& a) {
     return a.dtype == SF_BF16 && a.dk == kD && a.dv == kD;

@@ -235,4 +235,10 @@ bool make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dim
                const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapDataType dtype,
                CUtensorMapSwizzle swz);
 
+struct Args;
+// 2-D bf16 map over rows of `inner` elements, tiles of 64 x box_rows, 128-byte swizzle.
+bool tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows);
+// [B, ld_t, H, d] token-major bf16 input of one call: tiles of 64 tokens x 64 features.
+bool tmap_tokens(CUtensorMap* m, const void* base, const Args& a, int d);
+
 }  // namespace sf
