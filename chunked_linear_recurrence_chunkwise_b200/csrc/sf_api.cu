@@ -197,12 +197,13 @@ cudaError_t run_bwd_prep(Args a, cudaStream_t st) {
     a.S_out = nullptr;
     e = state_fwd(a, st);
     if (e != cudaSuccess) return e;
-    return launch_dd_pre(a, st);
+    // the tensor-core reverse pass forms P^T dO itself from the stored P
+    return tc_eligible(a) ? cudaSuccess : launch_dd_pre(a, st);
 }
 
 // The dS-dependent part: reverse state pass, then the per-chunk gradients.
 cudaError_t run_bwd_grads(const Args& a, cudaStream_t st) {
-    cudaError_t e = launch_state_bwd(a, st);
+    cudaError_t e = tc_eligible(a) ? launch_state_bwd_tc(a, st) : launch_state_bwd(a, st);
     if (e == cudaSuccess && a.beta) e = launch_grad_delta(a, st);
     if (e == cudaSuccess) e = launch_grad_attn(a, st);
     return e;

@@ -293,6 +293,281 @@ __global__ void __launch_bounds__(256, 1)
     }
 }
 
+
+// Shared-memory carve-up of the reverse pass (byte offsets from a 1024-aligned base).
+constexpr int kBStages = 2;
+struct BwdSmem {
+    static constexpr int Kt = 0;                          // [stage] K   [2][64 r][64 d_k]
+    static constexpr int dO = Kt + kBStages * kTile;      // [stage] dO  [2][64 r][64 d_v]
+    static constexpr int Q = dO + kBStages * kTile;       // [stage] Q   [2][64 r][64 d_k]
+    static constexpr int Wt = Q + kBStages * kTile;       // [stage] W^T [d_k][64 r]
+    static constexpr int P = Wt + kBStages * kTile;       // [stage] P   [64 i][64 r]
+    static constexpr int St = P + kBStages * 8192;        // dS^T operand [2 kblk][d_v][64]
+    static constexpr int Dop = St + 2 * kTile;            // dDelta^T [d_v][64 r] (operand + store)
+    static constexpr int Dv = Dop + kTile;                // dv staging [2][64 r][64 d_v] (no beta)
+    static constexpr int G = Dv + kTile;                  // [stage][64] fp32
+    static constexpr int Bar = G + kBStages * 256;
+    static constexpr int Misc = Bar + (kBStages + 1) * 8;
+    static constexpr int Size = Misc + 16;
+};
+
+// Reverse pass over the chunks of one head, carrying dS^T in fp32 registers:
+//   dDelta^T = diag-scaled (dS'^T K^T) + dO^T P           (UMMAs, then threads)
+//   dS^T    <- gamma_C dS'^T + dO^T (diag(gamma) Q) - dDelta^T W
+// (the transpose of dS = gamma_C dS' + (diag(gamma) Q)^T dO - W^T dDelta with
+// dDelta = P^T dO + Ktil dS').  Stores dS'^T of every chunk and dDelta^T (or
+// dv = dDelta directly for linear attention).
+template <bool kDelta>
+__global__ void __launch_bounds__(256, 1)
+    state_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_do,
+                        const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_wt,
+                        const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_dsc,
+                        const __grid_constant__ CUtensorMap tm_ddt, const __grid_constant__ CUtensorMap tm_dv,
+                        const Args a) {
+    using L = BwdSmem;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    float* Gs = (float*)(sm + L::G);
+    uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);
+    uint64_t* bar_mma = bar_ld + kBStages;
+    uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
+    volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int j = quad * 32 + lane;  // d_v row = TMEM lane
+    const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+    const int NC = a.NC, TP = NC * kChunk;
+
+    if (tid == 0) {
+        for (int s = 0; s < kBStages; ++s) mbar_init(&bar_ld[s], 1);
+        mbar_init(bar_mma, 1);
+        *s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc(s_tmem, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t tY1 = tmem, tY2 = tmem + 64, tZ = tmem + 128;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+
+    // n-th load (n = 0, 1, ...) is chunk NC - 1 - n, stage n % 2
+    auto issue_load = [&](int n) {
+        const int c = NC - 1 - n, s = n % kBStages;
+        const uint32_t bytes = 3 * kTile + 8192 + (kDelta ? kTile : 0) + 256;
+        mbar_expect_tx(&bar_ld[s], bytes);
+        tma_load_4d(sm + L::Kt + s * kTile, &tm_k, 0, h, c * kChunk, b, &bar_ld[s]);
+        tma_load_4d(sm + L::Kt + s * kTile + 8192, &tm_k, 64, h, c * kChunk, b, &bar_ld[s]);
+        tma_load_4d(sm + L::dO + s * kTile, &tm_do, 0, h, c * kChunk, b, &bar_ld[s]);
+        tma_load_4d(sm + L::dO + s * kTile + 8192, &tm_do, 64, h, c * kChunk, b, &bar_ld[s]);
+        tma_load_4d(sm + L::Q + s * kTile, &tm_q, 0, h, c * kChunk, b, &bar_ld[s]);
+        tma_load_4d(sm + L::Q + s * kTile + 8192, &tm_q, 64, h, c * kChunk, b, &bar_ld[s]);
+        if (kDelta) tma_load_2d(sm + L::Wt + s * kTile, &tm_wt, 0, (bh * NC + c) * kD, &bar_ld[s]);
+        tma_load_2d(sm + L::P + s * 8192, &tm_p, 0, (bh * NC + c) * kChunk, &bar_ld[s]);
+        bulk_load(Gs + s * kChunk, a.G + (size_t)bh * TP + c * kChunk, 256, &bar_ld[s]);
+    };
+    int issued = 0;
+    if (tid == 0)
+        for (; issued < min(kBStages, NC); ++issued) issue_load(issued);
+
+    // dS^T row j, columns i in [64 half, 64 half + 64): S[q] = dS_{i, j}
+    float S[64];
+#pragma unroll
+    for (int q = 0; q < 64; ++q)
+        S[q] = a.dS_out ? a.dS_out[((size_t)bh * kD + half * 64 + q) * kD + j] : 0.f;
+    uint8_t* St = sm + L::St + half * kTile;
+    auto write_state = [&]() {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            uint4 v;
+            v.x = pack_bf16(S[q * 8 + 0], S[q * 8 + 1]);
+            v.y = pack_bf16(S[q * 8 + 2], S[q * 8 + 3]);
+            v.z = pack_bf16(S[q * 8 + 4], S[q * 8 + 5]);
+            v.w = pack_bf16(S[q * 8 + 6], S[q * 8 + 7]);
+            *(uint4*)(St + sw128(j, q)) = v;
+        }
+    };
+    write_state();
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        tma_store_2d(&tm_dsc, sm + L::St, 0, (bh * NC + NC - 1) * kD);
+        tma_store_2d(&tm_dsc, sm + L::St + kTile, 64, (bh * NC + NC - 1) * kD);
+        bulk_commit();
+    }
+
+    uint32_t mma_phase = 0;
+    bool mma_pending = false;
+    bool aborted = false;
+    int n = 0;
+    for (; n < NC; ++n) {
+        const int c = NC - 1 - n, s = n % kBStages;
+        if (tid == 0) {
+            if (!mbar_wait(&bar_ld[s], (n / kBStages) & 1)) {
+                *s_abort = 1;
+                atomicExch(a.err, kErrTimeoutTma);
+            } else {
+                tc_fence_after();
+                const uint32_t st = smem_u32(sm + L::St), kt = smem_u32(sm + L::Kt + s * kTile);
+                const uint32_t dob = smem_u32(sm + L::dO + s * kTile), pb = smem_u32(sm + L::P + s * 8192);
+                constexpr uint32_t id1 = idesc_bf16(128, 64, false, false);
+                constexpr uint32_t id2 = idesc_bf16(128, 64, true, true);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_bf16(tY1, sdesc(st + (ks >> 2) * kTile + (ks & 3) * 32, 16, 1024),
+                             sdesc(kt + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id1, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tY2, sdesc(dob + ks * 2048, 8192, 1024), sdesc(pb + ks * 2048, 8192, 1024),
+                             id2, ks > 0);
+                mma_commit(bar_mma);
+                bulk_wait_read<1>();  // the dDelta^T / dv store of chunk c+1 has been read
+                if (!mbar_wait(bar_mma, mma_phase)) {
+                    *s_abort = 1;
+                    mma_pending = true;
+                    atomicExch(a.err, kErrTimeoutMma);
+                }
+            }
+        }
+        mma_phase ^= 1;
+        __syncthreads();
+        if (*s_abort) {
+            aborted = true;
+            break;
+        }
+        tc_fence_after();
+        const float* G = Gs + s * kChunk;
+        const float gC = G[kChunk - 1];
+        {
+            float y1[32], y2[32];
+            tmem_ld32(tY1 + lane_base + half * 32, y1);
+            tmem_ld32(tY2 + lane_base + half * 32, y2);
+            tmem_ld_wait();
+            float d[32];
+#pragma unroll
+            for (int q = 0; q < 32; ++q) d[q] = __expf(gC - G[half * 32 + q]) * y1[q] + y2[q];
+            if (kDelta) {
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    uint4 u;
+                    u.x = pack_bf16(d[qq * 8 + 0], d[qq * 8 + 1]);
+                    u.y = pack_bf16(d[qq * 8 + 2], d[qq * 8 + 3]);
+                    u.z = pack_bf16(d[qq * 8 + 4], d[qq * 8 + 5]);
+                    u.w = pack_bf16(d[qq * 8 + 6], d[qq * 8 + 7]);
+                    *(uint4*)(sm + L::Dop + sw128(j, half * 4 + qq)) = u;
+                }
+            } else {
+                // linear attention: dv = dDelta, staged token-major for a TMA store
+                const uint32_t jb = (uint32_t)(j >> 6) * 8192, jq = (j & 63) >> 3, je = (j & 7) * 2;
+#pragma unroll
+                for (int q = 0; q < 32; ++q)
+                    *(__nv_bfloat16*)(sm + L::Dv + jb + sw128(half * 32 + q, jq) + je) =
+                        __float2bfloat16_rn(d[q]);
+            }
+        }
+        if (tid < 128) {  // diag(gamma) Q in place, one 128-byte line per thread
+            const int r = tid & 63, blk = tid >> 6;
+            uint8_t* line = sm + L::Q + s * kTile + blk * 8192 + r * 128;
+            const float f = __expf(G[r]);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                uint4 u = *(uint4*)(line + q * 16);
+                uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const float2 x = unpack_bf16(w[p]);
+                    w[p] = pack_bf16(x.x * f, x.y * f);
+                }
+                *(uint4*)(line + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            if (kDelta) {
+                tma_store_2d(&tm_ddt, sm + L::Dop, 0, (bh * NC + c) * kD);
+            } else {
+                tma_store_4d(&tm_dv, sm + L::Dv, 0, h, c * kChunk, b);
+                tma_store_4d(&tm_dv, sm + L::Dv + 8192, 64, h, c * kChunk, b);
+            }
+            bulk_commit();
+            tc_fence_after();
+            const uint32_t dob = smem_u32(sm + L::dO + s * kTile), qb = smem_u32(sm + L::Q + s * kTile);
+            constexpr uint32_t idA = idesc_bf16(128, 128, true, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tZ, sdesc(dob + ks * 2048, 8192, 1024), sdesc(qb + ks * 2048, 8192, 1024), idA,
+                         ks > 0);
+            if (kDelta) {
+                const uint32_t dop = smem_u32(sm + L::Dop), wt = smem_u32(sm + L::Wt + s * kTile);
+                constexpr uint32_t idB = idesc_bf16(128, 128, false, false, true);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tZ, sdesc(dop + ks * 32, 16, 1024), sdesc(wt + ks * 32, 16, 1024), idB, 1);
+            }
+            mma_commit(bar_mma);
+            bulk_wait_read<1>();  // the dS'^T store issued after chunk c+1 has been read
+            if (!mbar_wait(bar_mma, mma_phase)) {
+                *s_abort = 1;
+                mma_pending = true;
+                atomicExch(a.err, kErrTimeoutMma);
+            } else if (issued < NC) {
+                issue_load(issued);  // stage s is free again
+                ++issued;
+            }
+        }
+        mma_phase ^= 1;
+        __syncthreads();
+        if (*s_abort) {
+            aborted = true;
+            break;
+        }
+        tc_fence_after();
+        {
+            float z0[32], z1[32];
+            tmem_ld32(tZ + lane_base + half * 64, z0);
+            tmem_ld32(tZ + lane_base + half * 64 + 32, z1);
+            tmem_ld_wait();
+            const float gam = __expf(gC);
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                S[q] = gam * S[q] + z0[q];
+                S[32 + q] = gam * S[32 + q] + z1[q];
+            }
+        }
+        if (c > 0) {
+            write_state();
+            fence_async_smem();
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && c > 0) {
+            tma_store_2d(&tm_dsc, sm + L::St, 0, (bh * NC + c - 1) * kD);
+            tma_store_2d(&tm_dsc, sm + L::St + kTile, 64, (bh * NC + c - 1) * kD);
+            bulk_commit();
+        }
+    }
+    if (!aborted && a.dS_in) {
+#pragma unroll
+        for (int q = 0; q < 64; ++q) a.dS_in[((size_t)bh * kD + half * 64 + q) * kD + j] = S[q];
+    }
+    if (tid == 0) {
+        if (aborted) {
+            for (int m = n; m < issued; ++m) mbar_wait(&bar_ld[m % kBStages], (m / kBStages) & 1);
+            if (mma_pending) mbar_wait(bar_mma, mma_phase ^ 1);
+        }
+        bulk_wait<0>();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
 }  // namespace
 
 bool tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
@@ -334,6 +609,31 @@ cudaError_t launch_state_fwd_tc(const Args& a, cudaStream_t s) {
     kern<<<BH, 256, smem, s>>>(tm_wt, tm_ut, tm_k, tm_sc, tm_dt, a);
     e = cudaGetLastError();
     timing_end(KK_STATE_FWD, s);
+    return e;
+}
+
+cudaError_t launch_state_bwd_tc(const Args& a, cudaStream_t s) {
+    const int BH = a.B * a.H;
+    if (BH == 0 || a.NC == 0) return cudaSuccess;
+    const uint64_t rows = (uint64_t)BH * a.NC * kD;
+    CUtensorMap tm_k{}, tm_do{}, tm_q{}, tm_wt{}, tm_p{}, tm_dsc{}, tm_ddt{}, tm_dv{};
+    bool ok = tmap_tokens(&tm_k, a.k, a, kD) && tmap_tokens(&tm_do, a.dO, a, kD) &&
+              tmap_tokens(&tm_q, a.q, a, kD) &&
+              tmap_2d(&tm_p, a.Pm, 64, (uint64_t)BH * a.NC * kChunk, 64) &&
+              tmap_2d(&tm_dsc, a.dSc, kD, rows, 128);
+    if (a.beta)
+        ok = ok && tmap_2d(&tm_wt, a.Wt, 64, rows, 128) && tmap_2d(&tm_ddt, a.dDt, 64, rows, 128);
+    else
+        ok = ok && tmap_tokens(&tm_dv, a.dv_, a, kD);
+    if (!ok) return cudaErrorInvalidValue;
+    const size_t smem = BwdSmem::Size + 1024;
+    auto kern = a.beta ? state_bwd_tc_kernel<true> : state_bwd_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    timing_begin(KK_STATE_BWD, s);
+    kern<<<BH, 256, smem, s>>>(tm_k, tm_do, tm_q, tm_wt, tm_p, tm_dsc, tm_ddt, tm_dv, a);
+    e = cudaGetLastError();
+    timing_end(KK_STATE_BWD, s);
     return e;
 }
 

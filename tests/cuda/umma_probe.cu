@@ -8,7 +8,7 @@ using namespace sf::tc;
 
 __global__ void __launch_bounds__(128, 1)
     umma_probe_kernel(const __nv_bfloat16* A, const __nv_bfloat16* B, float* C, int M, int N,
-                      int K, int a_mn, int b_mn, int* err) {
+                      int K, int a_mn, int b_mn, int neg_a, int* err) {
     extern __shared__ uint8_t raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)raw + 1023) & ~(uintptr_t)1023);
     uint8_t* As = sm;                 // up to 128 x 128 bf16 = 32 KB
@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(128, 1)
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
     if (tid == 0) {
-        const uint32_t id = idesc_bf16(M, N, a_mn, b_mn);
+        const uint32_t id = idesc_bf16(M, N, a_mn, b_mn, neg_a != 0);
         const uint32_t a0 = smem_u32(As), b0 = smem_u32(Bs);
         for (int ks = 0; ks < K / 16; ++ks) {
             const uint64_t ad = a_mn ? sdesc(a0 + ks * 2048, K * 128, 1024)
@@ -77,12 +77,12 @@ __global__ void __launch_bounds__(128, 1)
 }
 
 extern "C" int umma_probe(const void* A, const void* B, void* C, int M, int N, int K, int a_mn,
-                          int b_mn, void* err, void* stream) {
+                          int b_mn, int neg_a, void* err, void* stream) {
     if (!(M == 64 || M == 128) || N % 32 || N > 128 || K % 64 || K > 128) return 1;
     const int smem = 65536 + 64 + 1024;
     cudaFuncSetAttribute(umma_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     umma_probe_kernel<<<1, 128, smem, (cudaStream_t)stream>>>(
         (const __nv_bfloat16*)A, (const __nv_bfloat16*)B, (float*)C, M, N, K, a_mn, b_mn,
-        (int*)err);
+        neg_a, (int*)err);
     return (int)cudaGetLastError();
 }

@@ -21,7 +21,7 @@ def probe(tmp_path_factory):
                            os.path.join(HERE, "cuda", "umma_probe.cu"), "-o", out])
     lib = ctypes.CDLL(out)
     lib.umma_probe.restype = ctypes.c_int
-    lib.umma_probe.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 5 + [ctypes.c_void_p] * 2
+    lib.umma_probe.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 6 + [ctypes.c_void_p] * 2
     return lib
 
 
@@ -30,15 +30,16 @@ def probe(tmp_path_factory):
 @pytest.mark.parametrize("K", [64, 128])
 @pytest.mark.parametrize("a_mn", [0, 1])
 @pytest.mark.parametrize("b_mn", [0, 1])
-def test_umma_tile(probe, M, N, K, a_mn, b_mn):
+@pytest.mark.parametrize("neg_a", [0, 1])
+def test_umma_tile(probe, M, N, K, a_mn, b_mn, neg_a):
     g = torch.Generator(device="cuda").manual_seed(M * 7 + N * 3 + K + 2 * a_mn + b_mn)
     A = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
     B = torch.randn(K, N, device="cuda", generator=g).to(torch.bfloat16)
     C = torch.full((M, N), float("nan"), device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    rc = probe.umma_probe(A.data_ptr(), B.data_ptr(), C.data_ptr(), M, N, K, a_mn, b_mn,
+    rc = probe.umma_probe(A.data_ptr(), B.data_ptr(), C.data_ptr(), M, N, K, a_mn, b_mn, neg_a,
                           err.data_ptr(), torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
     assert rc == 0 and int(err.item()) == 0
-    ref = A.float() @ B.float()
+    ref = (A.float() @ B.float()) * (-1.0 if neg_a else 1.0)
     assert torch.allclose(C, ref, rtol=1e-3, atol=1e-3), (C - ref).abs().max().item()
