@@ -80,6 +80,8 @@ cudaError_t launch_intra_tc(const Args& a, bool with_p, cudaStream_t s);
 cudaError_t launch_output_tc(const Args& a, cudaStream_t s);
 // reverse dS pass; consumes P from the backward intra kernel (no dDelta pre-pass)
 cudaError_t launch_state_bwd_tc(const Args& a, cudaStream_t s);
+// dq, dk, dg (adds dKp / dGp of the delta-rule gradient kernel when beta is given)
+cudaError_t launch_grad_attn_tc(const Args& a, cudaStream_t s);
 
 // Per-kernel timing registry (sf_timing_*).
 enum KernelKind {

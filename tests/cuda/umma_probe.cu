@@ -8,7 +8,7 @@ using namespace sf::tc;
 
 __global__ void __launch_bounds__(128, 1)
     umma_probe_kernel(const __nv_bfloat16* A, const __nv_bfloat16* B, float* C, int M, int N,
-                      int K, int a_mn, int b_mn, int neg_a, int* err) {
+                      int K, int a_mn, int b_mn, int neg_a, int lane16, int restore, int* err) {
     extern __shared__ uint8_t raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)raw + 1023) & ~(uintptr_t)1023);
     uint8_t* As = sm;                 // up to 128 x 128 bf16 = 32 KB
@@ -42,29 +42,56 @@ __global__ void __launch_bounds__(128, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    if (tid == 0) {
-        const uint32_t id = idesc_bf16(M, N, a_mn, b_mn, neg_a != 0);
-        const uint32_t a0 = smem_u32(As), b0 = smem_u32(Bs);
+    // lane16: an M = 64 accumulator placed at TMEM lane offset 16 (lanes 16-31 of each quadrant)
+    const uint32_t tD = tmem + ((lane16 ? 16u : 0u) << 16);
+    const uint32_t id = idesc_bf16(M, N, a_mn, b_mn, neg_a != 0);
+    const uint32_t a0 = smem_u32(As), b0 = smem_u32(Bs);
+    auto issue = [&](uint32_t acc0) {
         for (int ks = 0; ks < K / 16; ++ks) {
             const uint64_t ad = a_mn ? sdesc(a0 + ks * 2048, K * 128, 1024)
                                      : sdesc(a0 + (ks / 4) * (M * 128) + (ks % 4) * 32, 16, 1024);
             const uint64_t bd = b_mn ? sdesc(b0 + ks * 2048, K * 128, 1024)
                                      : sdesc(b0 + (ks / 4) * (N * 128) + (ks % 4) * 32, 16, 1024);
-            mma_bf16(tmem, ad, bd, id, ks > 0);
+            mma_bf16(tD, ad, bd, id, (ks > 0) || acc0);
         }
+    };
+    if (tid == 0) {
+        issue(0);
         mma_commit(bar);
         if (!mbar_wait(bar, 0)) atomicExch(err, 1);
     }
     __syncthreads();
     tc_fence_after();
     const int lane = tid & 31;
+    // restore: read the accumulator, double it, store it back, accumulate A*B once more (3 A*B)
+    if (restore) {
+        for (int n0 = 0; n0 < N; n0 += 32) {
+            float v[32];
+            tmem_ld32(taddr(tmem, warp * 32, n0), v);
+            tmem_ld_wait();
+            for (int q = 0; q < 32; ++q) v[q] *= 2.f;
+            tmem_st32(taddr(tmem, warp * 32, n0), v);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            issue(1);
+            mma_commit(bar);
+            if (!mbar_wait(bar, 1)) atomicExch(err, 1);
+        }
+        __syncthreads();
+        tc_fence_after();
+    }
     for (int n0 = 0; n0 < N; n0 += 32) {
         float v[32];
         tmem_ld32(taddr(tmem, warp * 32, n0), v);
         tmem_ld_wait();
         int row = -1;
         if (M == 128) row = warp * 32 + lane;
-        else if (lane < 16) row = warp * 16 + lane;
+        else if (!lane16 && lane < 16) row = warp * 16 + lane;
+        else if (lane16 && lane >= 16) row = warp * 16 + lane - 16;
         if (row >= 0)
             for (int q = 0; q < 32; ++q) C[row * N + n0 + q] = v[q];
     }
@@ -77,12 +104,12 @@ __global__ void __launch_bounds__(128, 1)
 }
 
 extern "C" int umma_probe(const void* A, const void* B, void* C, int M, int N, int K, int a_mn,
-                          int b_mn, int neg_a, void* err, void* stream) {
-    if (!(M == 64 || M == 128) || N % 32 || N > 128 || K % 64 || K > 128) return 1;
+                          int b_mn, int neg_a, int lane16, int restore, void* err, void* stream) {
+    if (!(M == 64 || M == 128) || N % 32 || N > 128 || K % 64 || K > 128 || (lane16 && M != 64)) return 1;
     const int smem = 65536 + 64 + 1024;
     cudaFuncSetAttribute(umma_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     umma_probe_kernel<<<1, 128, smem, (cudaStream_t)stream>>>(
         (const __nv_bfloat16*)A, (const __nv_bfloat16*)B, (float*)C, M, N, K, a_mn, b_mn,
-        neg_a, (int*)err);
+        neg_a, lane16, restore, (int*)err);
     return (int)cudaGetLastError();
 }

@@ -21,7 +21,7 @@ def probe(tmp_path_factory):
                            os.path.join(HERE, "cuda", "umma_probe.cu"), "-o", out])
     lib = ctypes.CDLL(out)
     lib.umma_probe.restype = ctypes.c_int
-    lib.umma_probe.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 6 + [ctypes.c_void_p] * 2
+    lib.umma_probe.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 8 + [ctypes.c_void_p] * 2
     return lib
 
 
@@ -32,14 +32,27 @@ def probe(tmp_path_factory):
 @pytest.mark.parametrize("b_mn", [0, 1])
 @pytest.mark.parametrize("neg_a", [0, 1])
 def test_umma_tile(probe, M, N, K, a_mn, b_mn, neg_a):
+    run_probe(probe, M, N, K, a_mn, b_mn, neg_a, 0, 0)
+
+
+@pytest.mark.parametrize("lane16", [0, 1])
+@pytest.mark.parametrize("restore", [0, 1])
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (1, 1)])
+def test_m64_lane_offset_and_tmem_store(probe, lane16, restore, a_mn, b_mn):
+    """M = 64 accumulators at TMEM lane offset 16, and tcgen05.st of a rescaled
+    accumulator followed by accumulating UMMAs (result 3 A B when restored)."""
+    run_probe(probe, 64, 128, 128, a_mn, b_mn, 0, lane16, restore)
+
+
+def run_probe(probe, M, N, K, a_mn, b_mn, neg_a, lane16, restore):
     g = torch.Generator(device="cuda").manual_seed(M * 7 + N * 3 + K + 2 * a_mn + b_mn)
     A = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
     B = torch.randn(K, N, device="cuda", generator=g).to(torch.bfloat16)
     C = torch.full((M, N), float("nan"), device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     rc = probe.umma_probe(A.data_ptr(), B.data_ptr(), C.data_ptr(), M, N, K, a_mn, b_mn, neg_a,
-                          err.data_ptr(), torch.cuda.current_stream().cuda_stream)
+                          lane16, restore, err.data_ptr(), torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
     assert rc == 0 and int(err.item()) == 0
-    ref = (A.float() @ B.float()) * (-1.0 if neg_a else 1.0)
+    ref = (A.float() @ B.float()) * (-1.0 if neg_a else 1.0) * (3.0 if restore else 1.0)
     assert torch.allclose(C, ref, rtol=1e-3, atol=1e-3), (C - ref).abs().max().item()
