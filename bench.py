@@ -44,6 +44,9 @@ def parse_args(argv=None):
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=16384)
+    p.add_argument("--tokens", type=int, default=None,
+                   help="override T (a smaller case of the same workload, e.g. for ncu captures)")
+    p.add_argument("--heads", type=int, default=None, help="override H")
     return p.parse_args(argv)
 
 
@@ -279,12 +282,13 @@ def run_sf(args, w, rank, world, local_rank):
     db = None if x["beta"] is None else torch.empty_like(x["beta"])
     dS_in = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
 
-    def step(src):
+    def step(src, serial=False):
+        sa = main if serial else aux
         sf.sf_fwd_seq(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], None, o, S_out,
-                      S_saved, ws_f, stream_main=main, stream_aux=aux)
+                      S_saved, ws_f, stream_main=main, stream_aux=sa)
         sf.sf_bwd_seq(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], S_saved,
                       src["dO"], None, dq, dk, dv, dg, db, dS_in, ws_b, stream_main=main,
-                      stream_aux=aux)
+                      stream_aux=sa)
 
     def barrier():
         if world > 1:
@@ -300,8 +304,6 @@ def run_sf(args, w, rank, world, local_rank):
     clk = ClockSampler(local_rank)
     barrier()
     torch.cuda.synchronize()
-    sf.sf_timing_reset()
-    sf.sf_timing_enable(True)
     clk.start()
     time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -311,13 +313,22 @@ def run_sf(args, w, rank, world, local_rank):
     e1.record(main)
     torch.cuda.synchronize()
     clocks = clk.stop()
-    sf.sf_timing_enable(False)
-    timing = sf.sf_timing_read()
     barrier()
     ms = e0.elapsed_time(e1) / args.steps
     ms_max = reduce_max(ms, device=dev)
     sf.sf_check(ws_f, main)
     sf.sf_check(ws_b, main)
+
+    # ---- per-kernel durations: the same steps with both driver streams on one
+    # stream, every launch bracketed by CUDA events on its stream (with two
+    # streams an event pair also counts time spent queued behind the other one)
+    sf.sf_timing_reset()
+    sf.sf_timing_enable(True)
+    for _ in range(args.steps):
+        step(x, serial=True)
+    torch.cuda.synchronize()
+    sf.sf_timing_enable(False)
+    timing = sf.sf_timing_read()
     launches = sum(v[0] for v in timing.values()) // max(1, args.steps)
 
     # ---- end to end: pinned host inputs -> device -> fwd+bwd -> results back to host
@@ -374,7 +385,9 @@ def run_sf(args, w, rank, world, local_rank):
             "e2e": e2e,
             "roofline": roofline(timing, w, args.steps, peaks, src, clocks),
             "kernels": {k_: {"launches": v[0] // max(1, args.steps),
-                             "ms_per_step": round(v[1] / args.steps, 4)} for k_, v in timing.items()},
+                             "ms_per_step": round(v[1] / args.steps, 4)} for k_, v in timing.items()
+                        if v[0] > 0},
+            "kernel_timing": "serialized pass (driver streams merged), CUDA events per launch",
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
@@ -385,6 +398,9 @@ def main(argv=None):
     args = parse_args(argv)
     rank, world, local_rank = dist_env()
     w = inputs.WORKLOADS[args.workload]
+    if args.tokens or args.heads:
+        T = args.tokens or w.T
+        w = w.scaled(T=T, H=args.heads or w.H, n_sub=max(1, min(w.n_sub, T // 4096)))
     if args.impl == "reference":
         return run_reference(args, w, rank, world)
     if world > 1:

@@ -204,7 +204,7 @@ cudaError_t run_bwd_prep(Args a, cudaStream_t st) {
 // The dS-dependent part: reverse state pass, then the per-chunk gradients.
 cudaError_t run_bwd_grads(const Args& a, cudaStream_t st) {
     cudaError_t e = tc_eligible(a) ? launch_state_bwd_tc(a, st) : launch_state_bwd(a, st);
-    if (e == cudaSuccess && a.beta) e = launch_grad_delta(a, st);
+    if (e == cudaSuccess && a.beta) e = tc_eligible(a) ? launch_grad_delta_tc(a, st) : launch_grad_delta(a, st);
     if (e == cudaSuccess) e = tc_eligible(a) ? launch_grad_attn_tc(a, st) : launch_grad_attn(a, st);
     return e;
 }

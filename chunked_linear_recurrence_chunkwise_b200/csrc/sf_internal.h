@@ -82,6 +82,8 @@ cudaError_t launch_output_tc(const Args& a, cudaStream_t s);
 cudaError_t launch_state_bwd_tc(const Args& a, cudaStream_t s);
 // dq, dk, dg (adds dKp / dGp of the delta-rule gradient kernel when beta is given)
 cudaError_t launch_grad_attn_tc(const Args& a, cudaStream_t s);
+// dv, dbeta and the delta-rule parts dKp, dGp
+cudaError_t launch_grad_delta_tc(const Args& a, cudaStream_t s);
 
 // Per-kernel timing registry (sf_timing_*).
 enum KernelKind {
