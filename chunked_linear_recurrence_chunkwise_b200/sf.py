@@ -41,6 +41,7 @@ _SIGS = {
     "sf_bwd": (_I, [_SP] + [_P] * 14 + [_P, _S, _P]),
     "sf_fwd_seq": (_I, [_SP, _I, _IP] + [_P] * 9 + [_P, _S, _P, _P]),
     "sf_bwd_seq": (_I, [_SP, _I, _IP] + [_P] * 14 + [_P, _S, _P, _P]),
+    "sf_fwd_noalloc": (_I, [_SP] + [_P] * 8 + [_P]),
     "sf_check": (_I, [_P, _P]),
     "sf_status_string": (ctypes.c_char_p, [_I]),
     "sf_timing_enable": (None, [_I]),
@@ -146,6 +147,12 @@ def sf_bwd_seq(sh, lens, q, k, v, g, beta, S_saved, dO, dS_out, dq, dk, dv, dg, 
                            _ptr(g), _ptr(beta), _ptr(S_saved), _ptr(dO), _ptr(dS_out), _ptr(dq),
                            _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(dS_in), _ptr(ws),
                            ws_bytes, sm, sa), "sf_bwd_seq")
+
+
+def sf_fwd_noalloc(sh, q, k, v, g, beta, S_in, o, S_out, stream=None):
+    """sf_fwd with the library's built-in scratch instead of a caller workspace."""
+    _check(_lib.sf_fwd_noalloc(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                               _ptr(S_in), _ptr(o), _ptr(S_out), _stream(stream)), "sf_fwd_noalloc")
 
 
 def sf_check(ws, stream=None):

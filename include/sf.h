@@ -117,6 +117,31 @@ sf_status sf_bwd_seq(const sf_shape* shape, int n_sub, const int* lens, const vo
                      void* dk, void* dv, float* dg, float* dbeta, float* dS_in, void* ws,
                      size_t ws_bytes, void* stream_main, void* stream_aux);
 
+/* Forward without a caller workspace, for callers that cannot allocate device
+ * memory (a plugin that is handed only its input and output buffers by a
+ * framework that plans all memory up front, code running inside an
+ * allocator's callbacks, or loops that must not call cudaMalloc because it can
+ * synchronise the device).  The pages have no counterpart: this is an
+ * interface convenience, not part of the method.
+ *
+ * Same arguments, semantics and errors as sf_fwd minus (ws, ws_bytes).  The
+ * scratch is a fixed 32 MiB array compiled into the library, held in device
+ * memory by every GPU that loads the library until the process exits.  A shape
+ * whose sf_workspace_bytes(shape, SF_OP_FWD) exceeds 32 MiB is rejected with
+ * SF_ERR_WORKSPACE before anything is launched (bf16, d_k = d_v = 128 needs
+ * about 1.3 KB per token and head).  The first call on a device looks up the
+ * array's device address (once per device, with that device current); make
+ * that first call before any stream capture.  All calls share the one array:
+ * calls whose work may overlap on the GPU (other streams, other host threads)
+ * race on it, calls ordered on one stream do not.  The array keeps the previous
+ * call's contents; each call first clears the error word that bounded device
+ * waits set (it lives in the array, so sf_check cannot read it for this entry
+ * point).  Allocates nothing: no cudaMalloc, cudaFree or allocating library
+ * routine is called. */
+sf_status sf_fwd_noalloc(const sf_shape* shape, const void* q, const void* k, const void* v,
+                         const float* g, const float* beta, const float* S_in, void* o,
+                         float* S_out, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error word kept at
  * the head of workspace `ws`.  Returns SF_ERR_TIMEOUT if a kernel gave up a
  * bounded wait since the last check, SF_ERR_CUDA on a CUDA error, else SF_OK. */
