@@ -72,6 +72,11 @@ def reduce_max(value: float, group=None, device=None) -> float:
     return float(t.item())
 
 
+def job_tokens_per_s(world: int, B: int, T: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank processed B*T tokens; the slowest rank sets the time."""
+    return world * B * T / (ms_max / 1e3)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -82,67 +87,102 @@ def load_peaks():
         return dict(PEAKS_FALLBACK), "fallback"
 
 
+def tc_path(w) -> bool:
+    """The tensor-core kernels serve bf16 with d_k = d_v = 128; everything else is SIMT."""
+    return w.dtype == "bf16" and w.d == 128
+
+
 def kernel_units(name: str, w) -> dict:
     """Algorithmic bytes and flops of one chunk-head (64 tokens of one head) per kernel.
 
-    Bytes count each input and output the kernel must move once, at the
-    precision this implementation stores it (I/O in the workload dtype, g and
-    beta and every intermediate in fp32); flops count the chunk's arithmetic
-    once, triangle-aware (only the causal half of the 64 x 64 products).
+    Bytes count each tensor the kernel must read or write once, at the
+    precision the path stores it: on the tensor-core path q, k, v, o and the
+    gradients are bf16, intermediates (W^T, U^T, chunk states, Delta, P) bf16,
+    g, beta, the cumulative decay and the delta-rule partial dk fp32.  Flops
+    are 2 x the multiply-adds of the chunk's dense products as the kernel
+    issues them on 64 x 64 / 64 x 128 / 128 x 128 tiles.
     """
     C, d = 64, w.d
-    e = 2 if w.dtype == "bf16" else 4
     f = 4
-    tri_s = C * (C - 1) // 2   # strictly lower entries
-    tri_i = C * (C + 1) // 2   # inclusive lower entries
-    tab = {
-        "intra_fwd": (2 * C * d * e + 2 * C * f + C * f + 2 * C * d * f,
-                      tri_s * 2 * d + tri_s * 2 * 2 * d),
-        "state_fwd": (2 * C * d * f + C * d * e + C * f + d * d * f + C * d * f,
-                      4 * C * d * d),
-        "output": (2 * C * d * e + C * f + d * d * f + C * d * f + C * d * e,
-                   tri_i * 2 * d * 2 + 2 * C * d * d),
-        "dd_pre": (3 * C * d * e + C * f + C * d * f, tri_i * 2 * d * 2),
-        "state_bwd": (3 * C * d * e + 2 * C * d * f + C * f + d * d * f + C * d * f,
-                      6 * C * d * d),
-        "grad_delta": (2 * C * d * e + 2 * C * f + 3 * C * d * f + d * d * f + C * d * e + C * f
-                       + C * d * f + C * f,
-                       tri_s * 2 * d * 6 + C * C * C // 3 * 2 + 2 * C * d * d),
-        "grad_attn": (3 * C * d * e + C * d * f + C * f + 2 * d * d * f + C * d * f + C * f
-                      + 2 * C * d * e + C * f,
-                      tri_i * 2 * d * 4 + 4 * C * d * d),
-    }
+    if tc_path(w):
+        e = 2                       # bf16 I/O and intermediates
+        tile = C * d * e            # one 64 x 128 bf16 tile: 16 KB
+        st = d * d * e              # one chunk state, bf16: 32 KB
+        mm = lambda m, n, k: 2 * m * n * k
+        tab = {
+            # read k, v (+ q), g, beta; write G, W^T, U^T (+ P)
+            "intra_fwd": (2 * tile + 2 * C * f + C * f + 2 * tile,
+                          mm(C, C, d) + 2 * mm(d, C, C)),
+            "intra_bwd": (3 * tile + 2 * C * f + C * f + 2 * tile + C * C * e,
+                          mm(2 * C, C, d) + 2 * mm(d, C, C)),
+            # read W^T, U^T, k, G; write S^T, Delta^T
+            "state_fwd": (3 * tile + C * f + st + tile, mm(d, C, d) + mm(d, d, C)),
+            # read q, k, S^T, Delta^T, G; write o
+            "output": (2 * tile + st + tile + C * f + tile,
+                       mm(C, C, d) + mm(d, C, d) + mm(d, C, C)),
+            # read k, dO, q, W^T, P, G; write dS'^T, dDelta^T
+            "state_bwd": (4 * tile + C * C * e + C * f + st + tile,
+                          mm(d, C, d) + mm(d, C, C) + 2 * mm(d, d, C)),
+            # read k, v, dDelta^T, S^T, W^T, U^T, beta, G; write dv, dbeta, dKp (fp32), dGp
+            "grad_delta": (5 * tile + st + 2 * C * f + tile + C * d * f + 2 * C * f,
+                           mm(C, C, d) + mm(C, d, d) + 2 * mm(C, d, C) + 2 * mm(C, C, d)
+                           + mm(C, d, C)),
+            # read q, k, dO, Delta^T, S^T, dS'^T, G, dKp, dGp; write dq, dk, dg
+            "grad_attn": (4 * tile + 2 * st + C * f + C * d * f + C * f + 2 * tile + C * f,
+                          2 * mm(C, C, d) + 2 * mm(C, d, d) + 2 * mm(C, d, C)),
+        }
+    else:
+        e = 2 if w.dtype == "bf16" else 4
+        tri_s = C * (C - 1) // 2
+        tri_i = C * (C + 1) // 2
+        tab = {
+            "intra_fwd": (2 * C * d * e + 3 * C * f + 2 * C * d * e, tri_s * 2 * d * 3),
+            "state_fwd": (3 * C * d * e + C * f + d * d * e + C * d * e, 4 * C * d * d),
+            "output": (3 * C * d * e + C * f + d * d * e + C * d * e, tri_i * 4 * d + 2 * C * d * d),
+            "dd_pre": (3 * C * d * e + C * f + C * d * e, tri_i * 4 * d),
+            "state_bwd": (5 * C * d * e + C * f + d * d * e + C * d * e, 6 * C * d * d),
+            "grad_delta": (6 * C * d * e + d * d * e + C * d * f + 3 * C * f,
+                           tri_s * 12 * d + 2 * C * d * d),
+            "grad_attn": (5 * C * d * e + 2 * d * d * e + C * d * f + 2 * C * f,
+                          tri_i * 8 * d + 4 * C * d * d),
+        }
     b, fl = tab.get(name, (0, 0))
     return {"bytes": b, "flops": fl}
 
 
 def roofline(timing: dict, w, steps: int, peaks: dict, peaks_src: str, clocks: dict):
-    """Roofline object of the kernel with the largest total time in the timed region."""
+    """Roofline object of the kernel with the largest total time (serialized pass).
+
+    Every kernel of this layer moves more bytes than its arithmetic can hide
+    (about 20-60 flop/byte against a ridge near 240 flop/byte), so the bound
+    is HBM bandwidth; the tensor-pipe fraction of the same kernel is reported
+    beside it.
+    """
     if not timing:
         return None
     name, (launches, ms) = max(timing.items(), key=lambda kv: kv[1][1])
     if launches == 0 or ms <= 0:
         return None
-    chunk_heads = w.B * w.H * ((w.T + 63) // 64) * steps  # over the timed steps
+    per_step = launches / steps
+    chunk_heads = w.B * w.H * ((w.T + 63) // 64)  # per step, over all pieces
+    # launches of one kind per step each process one piece; their chunk-heads add up to
+    # the whole sequence once per pass (intra and the forward state pass run twice: forward
+    # and backward recompute, and are timed as separate kinds or as two launches per piece)
+    passes = 2 if (name == "state_fwd") else 1
+    units_per_launch = chunk_heads * passes / per_step
     u = kernel_units(name, w)
     per_launch_s = ms / 1e3 / launches
-    bytes_pl = u["bytes"] * chunk_heads / launches
-    flops_pl = u["flops"] * chunk_heads / launches
-    gbs = bytes_pl / per_launch_s / 1e9
-    tfs = flops_pl / per_launch_s / 1e12
+    gbs = u["bytes"] * units_per_launch / per_launch_s / 1e9
+    tfs = u["flops"] * units_per_launch / per_launch_s / 1e12
     hbm = float(peaks["hbm_gbs"])
-    # the current kernels do their arithmetic on fp32 CUDA cores: ALU peak from unit counts
-    mhz = float(peaks.get("sm_max_mhz", 1965.0))
-    alu = SM_COUNT * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
-    if gbs / hbm >= tfs / alu:
-        obj = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
-               "frac": round(gbs / hbm, 4)}
-    else:
-        obj = {"bound": "alu", "achieved": round(tfs, 2), "peak": round(alu, 1), "unit": "TFLOP/s",
-               "frac": round(tfs / alu, 4)}
-    obj.update({"kernel": name, "traffic": None, "launches": launches,
-                "avg_launch_ms": round(ms / launches, 4), "peak_source": peaks_src,
-                "share_of_kernel_time": round(ms / sum(v[1] for v in timing.values()), 4)})
+    bf16 = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1590.0)))
+    obj = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+           "frac": round(gbs / hbm, 4), "traffic": None,
+           "kernel": name, "launches": launches, "avg_launch_ms": round(ms / launches, 4),
+           "bytes_per_launch": int(u["bytes"] * units_per_launch),
+           "tensor_tflops": round(tfs, 2), "tensor_frac": round(tfs / bf16, 4),
+           "peak_source": peaks_src + " (hbm_gbs; bf16_tflops_sustained for tensor_frac)",
+           "share_of_kernel_time": round(ms / sum(v[1] for v in timing.values()), 4)}
     return obj
 
 
@@ -359,7 +399,7 @@ def run_sf(args, w, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         e_ms = reduce_max(f0.elapsed_time(f1) / e2e_steps, device=dev)
-        e2e = {"value": round(world * B * T / (e_ms / 1e3), 1), "unit": "tokens/s",
+        e2e = {"value": round(job_tokens_per_s(world, B, T, e_ms), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 3),
                "steps": e2e_steps}
 
@@ -372,7 +412,7 @@ def run_sf(args, w, rank, world, local_rank):
     if rank == 0:
         peaks, src = load_peaks()
         line = {
-            "metric": "fwd+bwd tokens/s per layer", "value": round(world * B * T / (ms_max / 1e3), 1),
+            "metric": "fwd+bwd tokens/s per layer", "value": round(job_tokens_per_s(world, B, T, ms_max), 1),
             "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",

@@ -93,8 +93,8 @@ cudaEvent_t pool_get() {
 }  // namespace
 
 const char* kernel_name(int kind) {
-    static const char* names[KK_COUNT] = {"intra_fwd", "state_fwd",  "output",   "dd_pre",
-                                          "state_bwd", "grad_delta", "grad_attn"};
+    static const char* names[KK_COUNT] = {"intra_fwd", "state_fwd",  "output",    "dd_pre",
+                                          "state_bwd", "grad_delta", "grad_attn", "intra_bwd"};
     return (kind >= 0 && kind < KK_COUNT) ? names[kind] : "?";
 }
 

@@ -94,6 +94,7 @@ enum KernelKind {
     KK_STATE_BWD,
     KK_GRAD_DELTA,
     KK_GRAD_ATTN,
+    KK_INTRA_BWD,
     KK_COUNT
 };
 const char* kernel_name(int kind);

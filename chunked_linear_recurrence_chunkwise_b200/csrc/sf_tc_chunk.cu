@@ -539,7 +539,8 @@ cudaError_t launch_intra_tc(const Args& a, bool with_p, cudaStream_t s) {
     if (!ok) return cudaErrorInvalidValue;
     const dim3 grid(a.NC, BH);
     cudaError_t e;
-    timing_begin(KK_INTRA_FWD, s);
+    const int kind = with_p ? KK_INTRA_BWD : KK_INTRA_FWD;
+    timing_begin(kind, s);
     if (with_p) {
         const size_t smem = IntraSmem<true>::Size + 1024;
         auto kern = a.beta ? intra_tc_kernel<true, true> : intra_tc_kernel<false, true>;
@@ -552,7 +553,7 @@ cudaError_t launch_intra_tc(const Args& a, bool with_p, cudaStream_t s) {
         if (e == cudaSuccess) kern<<<grid, 128, smem, s>>>(tm_q, tm_k, tm_v, tm_wt, tm_ut, tm_p, a);
     }
     if (e == cudaSuccess) e = cudaGetLastError();
-    timing_end(KK_INTRA_FWD, s);
+    timing_end(kind, s);
     return e;
 }
 

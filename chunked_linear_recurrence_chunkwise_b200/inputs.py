@@ -230,11 +230,15 @@ def iter_blocks(w: Workload, heads=None, with_grad: bool | None = None, threads:
             yield i * BLOCK, min(w.T, (i + 1) * BLOCK), arrays
 
 
-def to_torch(w: Workload, device="cpu", heads=None, with_grad: bool | None = None, pin=False):
+def to_torch(w: Workload, device="cpu", heads=None, with_grad: bool | None = None, pin=False,
+             keep_heads=None):
     """Workload inputs as torch tensors (q, k, v, dO in the workload dtype; g, beta float32).
 
     Filled block by block, so the host never holds more than a few blocks in
     float32.  ``pin`` allocates page-locked host memory (``device='cpu'``).
+    ``keep_heads`` (list of (b, h)) also returns, under key "kept", a list of
+    float32 numpy dicts with the full sequence of those (batch, head) pairs,
+    taken from the same draw (single-head arrays shaped [1, T, 1, ...]).
     """
     import torch
 
@@ -255,10 +259,21 @@ def to_torch(w: Workload, device="cpu", heads=None, with_grad: bool | None = Non
             out[key] = torch.empty(shp, dtype=dt, pin_memory=True)
         else:
             out[key] = torch.empty(shp, dtype=dt, device=device)
+    kept = None if keep_heads is None else [{key: [] for key in shapes} for _ in keep_heads]
     for t0, t1, arr in iter_blocks(w, heads, grad):
         for key in shapes:
             src = torch.from_numpy(arr[key])
             out[key][:, t0:t1].copy_(src.to(out[key].dtype))
+            if kept is not None:
+                for i, (b, h) in enumerate(keep_heads):
+                    kept[i][key].append(arr[key][b:b + 1, :, h:h + 1].copy())
     for key in ("g", "beta", "dO"):
         out.setdefault(key, None)
+    if kept is not None:
+        out["kept"] = []
+        for d in kept:
+            full = {key: np.concatenate(parts, axis=1) for key, parts in d.items()}
+            for key in ("g", "beta", "dO"):
+                full.setdefault(key, None)
+            out["kept"].append(full)
     return out

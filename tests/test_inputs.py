@@ -43,3 +43,11 @@ def test_sub_lengths(name):
     if w.cut == "dirichlet":
         assert len(set(lens)) > 1
         assert lens == inputs.sub_lengths(w)  # seeded
+
+
+def test_kept_heads_match_the_device_copy():
+    w = inputs.WORKLOADS["gated_deltanet_bf16_h32_t64k"].scaled(T=5000, H=3)
+    x = inputs.to_torch(w, device="cpu", keep_heads=[(0, 2), (0, 0)])
+    for (b, h), kept in zip([(0, 2), (0, 0)], x["kept"]):
+        for key in ("q", "k", "v", "g", "beta", "dO"):
+            np.testing.assert_array_equal(kept[key][0, :, 0], x[key][b, :, h].float().numpy())
