@@ -25,6 +25,10 @@ namespace sf {
 
 static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Workspace slots of the sub-sequence drivers: up to three pieces are in flight at once
+// (piece i uses slot i % 3; fewer pieces need fewer slots).
+constexpr int kSeqSlots = 3;
+
 WsLayout ws_layout(int B, int T, int H, int dk, int dv, int dtype, bool delta, bool bwd,
                    int nslots) {
     WsLayout L{};
@@ -46,6 +50,7 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv, int dtype, bool delta, b
     L.dDt = take(bwd ? BH * TP * dv * tw : 0);
     L.dSc = take(bwd ? BH * NC * dk * dv * tw : 0);
     L.Pm = take(bwd ? BH * NC * kChunk * kChunk * tw : 0);
+    L.Tm = take(bwd && delta ? BH * NC * kChunk * kChunk * tw : 0);
     L.dKp = take(bwd && delta ? BH * TP * dk * 4 : 0);
     L.dGp = take(bwd && delta ? BH * TP * 4 : 0);
     L.slot_bytes = off;
@@ -63,6 +68,7 @@ void bind_slot(Args& a, void* ws, const WsLayout& L, int slot, bool bwd) {
     a.dDt = bwd ? (void*)(base + L.dDt) : nullptr;
     a.dSc = bwd ? (void*)(base + L.dSc) : nullptr;
     a.Pm = bwd ? (void*)(base + L.Pm) : nullptr;
+    a.Tm = bwd ? (void*)(base + L.Tm) : nullptr;
     a.dKp = bwd ? (float*)(base + L.dKp) : nullptr;
     a.dGp = bwd ? (float*)(base + L.dGp) : nullptr;
     a.err = (int*)ws;
@@ -201,6 +207,25 @@ cudaError_t run_bwd_prep(Args a, cudaStream_t st) {
     return tc_eligible(a) ? cudaSuccess : launch_dd_pre(a, st);
 }
 
+// The sequential part of one piece's backward: recompute of the chunk states
+// (and, on the SIMT path, the P^T dO pre-pass), then the reverse dS pass.
+cudaError_t run_bwd_state(Args a, cudaStream_t st) {
+    Args f = a;
+    f.S_out = nullptr;
+    cudaError_t e = state_fwd(f, st);
+    if (e == cudaSuccess && !tc_eligible(a)) e = launch_dd_pre(a, st);
+    if (e == cudaSuccess) e = tc_eligible(a) ? launch_state_bwd_tc(a, st) : launch_state_bwd(a, st);
+    return e;
+}
+
+// The per-chunk gradients of one piece (after its reverse pass).
+cudaError_t run_bwd_chunk_grads(const Args& a, cudaStream_t st) {
+    cudaError_t e = cudaSuccess;
+    if (a.beta) e = tc_eligible(a) ? launch_grad_delta_tc(a, st) : launch_grad_delta(a, st);
+    if (e == cudaSuccess) e = tc_eligible(a) ? launch_grad_attn_tc(a, st) : launch_grad_attn(a, st);
+    return e;
+}
+
 // The dS-dependent part: reverse state pass, then the per-chunk gradients.
 cudaError_t run_bwd_grads(const Args& a, cudaStream_t st) {
     cudaError_t e = tc_eligible(a) ? launch_state_bwd_tc(a, st) : launch_state_bwd(a, st);
@@ -279,7 +304,8 @@ size_t sf_seq_workspace_bytes(const sf_shape* s, int n_sub, const int* lens, int
     }
     if (sum != s->T) return 0;
     const size_t states = 2 * (size_t)s->B * s->H * s->dk * s->dv * sizeof(float);
-    return ws_layout(s->B, lmax, s->H, s->dk, s->dv, s->dtype, true, op == SF_OP_BWD, 2).total + states;
+    return ws_layout(s->B, lmax, s->H, s->dk, s->dv, s->dtype, true, op == SF_OP_BWD,
+                     std::min(kSeqSlots, n_sub)).total + states;
 }
 
 sf_status sf_fwd(const sf_shape* s, const void* q, const void* k, const void* v, const float* g,
@@ -350,7 +376,8 @@ sf_status sf_fwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
     if (st != SF_OK) return st;
     if (!work) return SF_OK;
     const size_t nstate = (size_t)s->B * s->H * s->dk * s->dv;
-    const WsLayout L = ws_layout(s->B, p.lmax, s->H, s->dk, s->dv, s->dtype, beta != nullptr, false, 2);
+    const WsLayout L = ws_layout(s->B, p.lmax, s->H, s->dk, s->dv, s->dtype, beta != nullptr, false,
+                                 std::min(kSeqSlots, n_sub));
     const size_t need = L.total + 2 * nstate * sizeof(float);
     if (!ws || ws_bytes < need || !aligned(ws, 256)) return SF_ERR_WORKSPACE;
     float* pingpong = (float*)((char*)ws + L.total);
@@ -359,11 +386,17 @@ sf_status sf_fwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
     const size_t es = esize(s);
     const int ld_t = s->ld_t ? s->ld_t : s->T;
 
+    // Schedule: the main stream carries only the sequential state passes; the
+    // aux stream runs the parallel work around them (intra of pieces i+1, i+2
+    // ahead, output of piece i behind), three workspace slots in flight.
+    constexpr int NS = kSeqSlots;
     EventSet evs;
-    // 0,1: intra of slot ready; 2,3: slot free again; 4: aux start; 5: aux done
-    SF_TRY(evs.make(6));
-    SF_TRY(cudaEventRecord(evs.ev[4], sm));
-    SF_TRY(cudaStreamWaitEvent(sa, evs.ev[4], 0));
+    SF_TRY(evs.make(2 * NS + 2));
+    cudaEvent_t* ev_intra = &evs.ev[0];   // intra of the slot's piece done (aux)
+    cudaEvent_t* ev_state = &evs.ev[NS];  // state pass of the slot's piece done (main)
+    cudaEvent_t ev_start = evs.ev[2 * NS], ev_aux_done = evs.ev[2 * NS + 1];
+    SF_TRY(cudaEventRecord(ev_start, sm));
+    SF_TRY(cudaStreamWaitEvent(sa, ev_start, 0));
 
     auto piece = [&](int i) {
         Args a = make_args(s);
@@ -385,32 +418,29 @@ sf_status sf_fwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
                                                   : pingpong + (size_t)(i & 1) * nstate);
         a.S_in = sin;
         a.S_out = sout;
-        bind_slot(a, ws, L, i & 1, false);
+        bind_slot(a, ws, L, i % kSeqSlots, false);
         return a;
     };
 
     if (S_saved) SF_TRY(copy_state(S_saved, S_in, nstate, sm));
-    {
-        Args a0 = piece(0);
-        SF_TRY(run_intra(a0, sa));
-        SF_TRY(cudaEventRecord(evs.ev[0], sa));
+    for (int j = 0; j < std::min(2, n_sub); ++j) {
+        SF_TRY(run_intra(piece(j), sa));
+        SF_TRY(cudaEventRecord(ev_intra[j % NS], sa));
     }
     for (int i = 0; i < n_sub; ++i) {
-        if (i + 1 < n_sub) {
-            const int sl = (i + 1) & 1;
-            if (i + 1 >= 2) SF_TRY(cudaStreamWaitEvent(sa, evs.ev[2 + sl], 0));
-            Args an = piece(i + 1);
-            SF_TRY(run_intra(an, sa));
-            SF_TRY(cudaEventRecord(evs.ev[sl], sa));
+        const Args a = piece(i);
+        SF_TRY(cudaStreamWaitEvent(sm, ev_intra[i % NS], 0));
+        SF_TRY(run_state_output(a, sm, false));
+        SF_TRY(cudaEventRecord(ev_state[i % NS], sm));
+        if (i + 2 < n_sub) {  // its slot's previous piece (i-1) finished its output on this stream
+            SF_TRY(run_intra(piece(i + 2), sa));
+            SF_TRY(cudaEventRecord(ev_intra[(i + 2) % NS], sa));
         }
-        Args a = piece(i);
-        // S_out of the last piece may be NULL: the state pass then writes nothing.
-        SF_TRY(cudaStreamWaitEvent(sm, evs.ev[i & 1], 0));
-        SF_TRY(run_state_output(a, sm, true));
-        SF_TRY(cudaEventRecord(evs.ev[2 + (i & 1)], sm));
+        SF_TRY(cudaStreamWaitEvent(sa, ev_state[i % NS], 0));
+        SF_TRY(output(a, sa));
     }
-    SF_TRY(cudaEventRecord(evs.ev[5], sa));
-    SF_TRY(cudaStreamWaitEvent(sm, evs.ev[5], 0));
+    SF_TRY(cudaEventRecord(ev_aux_done, sa));
+    SF_TRY(cudaStreamWaitEvent(sm, ev_aux_done, 0));
     return SF_OK;
 }
 
@@ -433,7 +463,8 @@ sf_status sf_bwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
     if (st != SF_OK) return st;
     if (!work) return SF_OK;
     const size_t nstate = (size_t)s->B * s->H * s->dk * s->dv;
-    const WsLayout L = ws_layout(s->B, p.lmax, s->H, s->dk, s->dv, s->dtype, beta != nullptr, true, 2);
+    const WsLayout L = ws_layout(s->B, p.lmax, s->H, s->dk, s->dv, s->dtype, beta != nullptr, true,
+                                 std::min(kSeqSlots, n_sub));
     const size_t need = L.total + 2 * nstate * sizeof(float);
     if (!ws || ws_bytes < need || !aligned(ws, 256)) return SF_ERR_WORKSPACE;
     float* pingpong = (float*)((char*)ws + L.total);
@@ -442,11 +473,18 @@ sf_status sf_bwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
     const size_t es = esize(s);
     const int ld_t = s->ld_t ? s->ld_t : s->T;
 
+    // Schedule (pieces in reverse): the main stream carries the sequential
+    // passes of each piece (forward-state recompute, then the reverse dS pass);
+    // the aux stream runs the parallel work (intra recompute two pieces ahead,
+    // per-chunk gradients one piece behind), three workspace slots in flight.
+    constexpr int NS = kSeqSlots;
     EventSet evs;
-    // 0,1: prep of slot ready; 2,3: slot free again; 4: aux start; 5: aux done
-    SF_TRY(evs.make(6));
-    SF_TRY(cudaEventRecord(evs.ev[4], sm));
-    SF_TRY(cudaStreamWaitEvent(sa, evs.ev[4], 0));
+    SF_TRY(evs.make(2 * NS + 2));
+    cudaEvent_t* ev_prep = &evs.ev[0];    // intra recompute of the slot's piece done (aux)
+    cudaEvent_t* ev_state = &evs.ev[NS];  // reverse pass of the slot's piece done (main)
+    cudaEvent_t ev_start = evs.ev[2 * NS], ev_aux_done = evs.ev[2 * NS + 1];
+    SF_TRY(cudaEventRecord(ev_start, sm));
+    SF_TRY(cudaStreamWaitEvent(sa, ev_start, 0));
 
     auto piece = [&](int i) {
         Args a = make_args(s);
@@ -470,30 +508,28 @@ sf_status sf_bwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
         // dS leaving piece i (from piece i+1) and dS entering it (to piece i-1)
         a.dS_out = (i == n_sub - 1) ? dS_out : pingpong + (size_t)((n_sub - 2 - i) & 1) * nstate;
         a.dS_in = (i == 0) ? dS_in : pingpong + (size_t)((n_sub - 1 - i) & 1) * nstate;
-        bind_slot(a, ws, L, i & 1, true);
+        bind_slot(a, ws, L, i % kSeqSlots, true);
         return a;
     };
 
-    {
-        Args a0 = piece(n_sub - 1);
-        SF_TRY(run_bwd_prep(a0, sa));
-        SF_TRY(cudaEventRecord(evs.ev[(n_sub - 1) & 1], sa));
+    for (int j = n_sub - 1; j >= std::max(0, n_sub - 2); --j) {
+        SF_TRY(intra(piece(j), true, sa));
+        SF_TRY(cudaEventRecord(ev_prep[j % NS], sa));
     }
     for (int i = n_sub - 1; i >= 0; --i) {
-        if (i - 1 >= 0) {
-            const int sl = (i - 1) & 1;
-            if (i - 1 <= n_sub - 3) SF_TRY(cudaStreamWaitEvent(sa, evs.ev[2 + sl], 0));
-            Args an = piece(i - 1);
-            SF_TRY(run_bwd_prep(an, sa));
-            SF_TRY(cudaEventRecord(evs.ev[sl], sa));
+        const Args a = piece(i);
+        SF_TRY(cudaStreamWaitEvent(sm, ev_prep[i % NS], 0));
+        SF_TRY(run_bwd_state(a, sm));
+        SF_TRY(cudaEventRecord(ev_state[i % NS], sm));
+        if (i - 2 >= 0) {  // its slot's previous piece (i+1) finished its gradients on this stream
+            SF_TRY(intra(piece(i - 2), true, sa));
+            SF_TRY(cudaEventRecord(ev_prep[(i - 2) % NS], sa));
         }
-        Args a = piece(i);
-        SF_TRY(cudaStreamWaitEvent(sm, evs.ev[i & 1], 0));
-        SF_TRY(run_bwd_grads(a, sm));
-        SF_TRY(cudaEventRecord(evs.ev[2 + (i & 1)], sm));
+        SF_TRY(cudaStreamWaitEvent(sa, ev_state[i % NS], 0));
+        SF_TRY(run_bwd_chunk_grads(a, sa));
     }
-    SF_TRY(cudaEventRecord(evs.ev[5], sa));
-    SF_TRY(cudaStreamWaitEvent(sm, evs.ev[5], 0));
+    SF_TRY(cudaEventRecord(ev_aux_done, sa));
+    SF_TRY(cudaStreamWaitEvent(sm, ev_aux_done, 0));
     return SF_OK;
 }
 

@@ -44,6 +44,7 @@ struct Args {
     void* dDt;    // [BH][NC][dv][64]    dL/dDelta, transposed per chunk
     void* dSc;    // [BH][NC][dv][dk]    (dL/dS leaving each chunk)^T
     void* Pm;     // [BH][NC][64][64]    P = (Q K^T) .* Gamma, lower incl. (backward)
+    void* Tm;     // [BH][NC][64][64]    T = (I + A)^-1, bf16 (backward, tensor-core path)
     float* dKp;   // [BH][TP][dk]        fp32 delta-rule part of dk (SIMT gradient kernels)
     float* dGp;   // [BH][TP]            fp32 delta-rule part of dG (SIMT gradient kernels)
     int* err;     // device error word
@@ -51,7 +52,7 @@ struct Args {
 
 // Workspace carve-up for a piece of at most T tokens.
 struct WsLayout {
-    size_t G, Wt, Ut, Sc, Dt, dDt, dSc, Pm, dKp, dGp;  // byte offsets inside one slot
+    size_t G, Wt, Ut, Sc, Dt, dDt, dSc, Pm, Tm, dKp, dGp;  // byte offsets inside one slot
     size_t slot_bytes;
     size_t total;  // err header + nslots * slot_bytes
 };

@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(128)
     intra_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_wt,
                     const __grid_constant__ CUtensorMap tm_ut, const __grid_constant__ CUtensorMap tm_p,
-                    const Args a) {
+                    const __grid_constant__ CUtensorMap tm_t, const Args a) {
     using L = IntraSmem<kP>;
     constexpr bool kKK = kDelta || kP;  // a K K^T (or [Q;K] K^T) product is needed
     extern __shared__ uint8_t smem_raw[];
@@ -302,6 +302,7 @@ __global__ void __launch_bounds__(128)
     if (tid == 0) {
         if (kP) {
             tma_store_2d(&tm_p, sm + L::Pst, 0, (bh * NC + c) * kChunk);
+            if (kDelta) tma_store_2d(&tm_t, sm + L::Tb, 0, (bh * NC + c) * kChunk);  // for the gradients
             bulk_commit();
         }
         tc_fence_after();
@@ -530,12 +531,13 @@ cudaError_t launch_intra_tc(const Args& a, bool with_p, cudaStream_t s) {
     const int BH = a.B * a.H;
     if (BH == 0 || a.NC == 0) return cudaSuccess;
     const uint64_t rows = (uint64_t)BH * a.NC * kD;
-    CUtensorMap tm_q{}, tm_k{}, tm_v{}, tm_wt{}, tm_ut{}, tm_p{};
+    CUtensorMap tm_q{}, tm_k{}, tm_v{}, tm_wt{}, tm_ut{}, tm_p{}, tm_t{};
     bool ok = tmap_tokens(&tm_k, a.k, a, kD) && tmap_tokens(&tm_v, a.v, a, kD) &&
               tmap_2d(&tm_ut, a.Ut, 64, rows, 128) && tmap_2d(&tm_wt, a.Wt, 64, rows, 128);
     if (with_p)
         ok = ok && tmap_tokens(&tm_q, a.q, a, kD) &&
              tmap_2d(&tm_p, a.Pm, 64, (uint64_t)BH * a.NC * kChunk, 64);
+    if (with_p && a.beta) ok = ok && tmap_2d(&tm_t, a.Tm, 64, (uint64_t)BH * a.NC * kChunk, 64);
     if (!ok) return cudaErrorInvalidValue;
     const dim3 grid(a.NC, BH);
     cudaError_t e;
@@ -545,12 +547,12 @@ cudaError_t launch_intra_tc(const Args& a, bool with_p, cudaStream_t s) {
         const size_t smem = IntraSmem<true>::Size + 1024;
         auto kern = a.beta ? intra_tc_kernel<true, true> : intra_tc_kernel<false, true>;
         e = set_smem(kern, smem);
-        if (e == cudaSuccess) kern<<<grid, 128, smem, s>>>(tm_q, tm_k, tm_v, tm_wt, tm_ut, tm_p, a);
+        if (e == cudaSuccess) kern<<<grid, 128, smem, s>>>(tm_q, tm_k, tm_v, tm_wt, tm_ut, tm_p, tm_t, a);
     } else {
         const size_t smem = IntraSmem<false>::Size + 1024;
         auto kern = a.beta ? intra_tc_kernel<true, false> : intra_tc_kernel<false, false>;
         e = set_smem(kern, smem);
-        if (e == cudaSuccess) kern<<<grid, 128, smem, s>>>(tm_q, tm_k, tm_v, tm_wt, tm_ut, tm_p, a);
+        if (e == cudaSuccess) kern<<<grid, 128, smem, s>>>(tm_q, tm_k, tm_v, tm_wt, tm_ut, tm_p, tm_t, a);
     }
     if (e == cudaSuccess) e = cudaGetLastError();
     timing_end(kind, s);

@@ -349,7 +349,7 @@ teardown:
 
 // ---------------------------------------------------------------------------
 // Delta-rule part of the per-chunk gradients (beta given):
-//   B = (K K^T) .* Gamma (strictly lower),  T = (I + diag(beta) B)^-1
+//   B = (K K^T) .* Gamma (strictly lower),  T = (I + diag(beta) B)^-1 (stored by the intra kernel)
 //   dVhat = T^T dDelta,  dW = -dDelta S^T,  dKhat = T^T dW
 //   dA = -(dKhat W^T + dVhat U^T) .* strictly lower,  dB = diag(beta) dA,  E = dB .* Gamma
 //   dv = diag(beta) dVhat
@@ -364,60 +364,19 @@ struct DeltaSmem {
     static constexpr int St = dDt + kTile;         // S^T [2 kblk][128 j][64 i]
     static constexpr int Wt = St + 2 * kTile;      // W^T [128 i][64 r]
     static constexpr int Ut = Wt + kTile;          // U^T [128 j][64 r]
-    static constexpr int Tb = Ut + kTile;          // T, bf16 [r'][64 r]
+    static constexpr int Tb = Ut + kTile;          // T, bf16 [r'][64 r] (from the intra kernel)
     static constexpr int dWb = Tb + kHalf;         // dW, then dKhat: bf16 [iblk][64 r][64]
     static constexpr int dVb = dWb + kTile;        // dVhat: bf16 [jblk][64 r][64]
     static constexpr int Bf = dVb + kTile;         // fp32 [64][65] B
-    static constexpr int Af = Bf + 64 * 65 * 4;    // fp32 [64][65] A, later E
-    static constexpr int Tf = Af + 64 * 65 * 4;    // fp32 [64][65] T, later Esym tile (bf16)
-    static constexpr int Mb = Tf + 64 * 65 * 4;    // fp32 [3][16][17]
-    static constexpr int Gs = Mb + 3 * 272 * 4;
+    static constexpr int Af = Bf + 64 * 65 * 4;    // fp32 [64][65] E = dB .* Gamma
+    static constexpr int Tf = Af + 64 * 65 * 4;    // fp32 [64][65] dB .* B
+    static constexpr int Gs = Tf + 64 * 65 * 4;
     static constexpr int Bs = Gs + 256;
     static constexpr int part = Bs + 256;          // fp32 [10][64] partial row sums
     static constexpr int Bar = part + 10 * 256;
     static constexpr int Misc = Bar + 16;
     static constexpr int Size = Misc + 16;
 };
-
-__device__ void tri_inverse64_256(const float* Af, float* Tf, float* Mb, int tid) {
-    for (int e = tid; e < 64 * 65; e += 256) Tf[e] = 0.f;
-    __syncthreads();
-    if (tid < 64) {
-        const int o = (tid >> 4) * 16, col = tid & 15;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float v = (r == col) ? 1.f : 0.f;
-#pragma unroll
-            for (int i = 0; i < r; ++i) v -= Af[(o + r) * 65 + o + i] * x[i];
-            x[r] = (r < col) ? 0.f : v;
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) Tf[(o + r) * 65 + o + col] = x[r];
-    }
-    __syncthreads();
-    for (int d = 1; d < 4; ++d) {
-        const int nb = 4 - d;
-        for (int e = tid; e < nb * 256; e += 256) {
-            const int m = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-            const int bi = m + d, bj = m;
-            float acc = 0.f;
-            for (int k = 16 * bj; k < 16 * bi; ++k)
-                acc += Af[(16 * bi + rr) * 65 + k] * Tf[k * 65 + 16 * bj + cc];
-            Mb[m * 272 + rr * 17 + cc] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < nb * 256; e += 256) {
-            const int m = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-            const int bi = m + d, bj = m;
-            float acc = 0.f;
-            for (int k = 0; k <= rr; ++k)
-                acc += Tf[(16 * bi + rr) * 65 + 16 * bi + k] * Mb[m * 272 + k * 17 + cc];
-            Tf[(16 * bi + rr) * 65 + 16 * bj + cc] = -acc;
-        }
-        __syncthreads();
-    }
-}
 
 __device__ __forceinline__ void store_row_half(uint8_t* tile, int row, int q0, const float* v, int n) {
     // n/8 16-byte chunks starting at chunk q0 of `row` in a 128-byte-swizzled tile
@@ -434,7 +393,8 @@ __device__ __forceinline__ void store_row_half(uint8_t* tile, int row, int q0, c
 __global__ void __launch_bounds__(256, 1)
     grad_delta_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_ddt,
                          const __grid_constant__ CUtensorMap tm_sc, const __grid_constant__ CUtensorMap tm_wt,
-                         const __grid_constant__ CUtensorMap tm_ut, const Args a) {
+                         const __grid_constant__ CUtensorMap tm_ut, const __grid_constant__ CUtensorMap tm_t,
+                         const Args a) {
     using L = DeltaSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -443,9 +403,8 @@ __global__ void __launch_bounds__(256, 1)
     float* Bf = (float*)(sm + L::Bf);
     float* Af = (float*)(sm + L::Af);
     float* Tf = (float*)(sm + L::Tf);
-    float* Mb = (float*)(sm + L::Mb);
     float* part = (float*)(sm + L::part);
-    float* Ef = Af;  // E = dB .* Gamma, fp32 [64][65] (after the inverse)
+    float* Ef = Af;  // E = dB .* Gamma, fp32 [64][65]
     uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);
     uint64_t* bar_mma = bar_ld + 1;
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
@@ -464,7 +423,8 @@ __global__ void __launch_bounds__(256, 1)
         mbar_init(bar_mma, 1);
         *s_abort = 0;
         fence_barrier_init();
-        mbar_expect_tx(bar_ld, 6 * kTile + 256);
+        mbar_expect_tx(bar_ld, 6 * kTile + kHalf + 256);
+        tma_load_2d(sm + L::Tb, &tm_t, 0, (bh * NC + c) * kChunk, bar_ld);  // T from the intra kernel
         tma_load_4d(sm + L::K, &tm_k, 0, h, t0, b, bar_ld);
         tma_load_4d(sm + L::K + kHalf, &tm_k, 64, h, t0, b, bar_ld);
         tma_load_2d(sm + L::dDt, &tm_ddt, 0, (bh * NC + c) * kD, bar_ld);
@@ -526,13 +486,11 @@ __global__ void __launch_bounds__(256, 1)
         tmem_ld32(tKK + lane_base + ch * 32, v);  // warp-collective; lanes 0-15 hold K K^T
         tmem_ld_wait();
         if (!hi) {
-            // B and A = diag(beta) B on columns [32 ch, 32 ch + 32) of row r
+            // B on columns [32 ch, 32 ch + 32) of row r
 #pragma unroll
             for (int q = 0; q < 32; ++q) {
                 const int t = ch * 32 + q;
-                const float bv = (t < r) ? __expf(Gr - Gs[t]) * v[q] : 0.f;
-                Bf[r * 65 + t] = bv;
-                Af[r * 65 + t] = Bs[r] * bv;
+                Bf[r * 65 + t] = (t < r) ? __expf(Gr - Gs[t]) * v[q] : 0.f;
             }
         }
         // dW = -(dDelta S^T), row r, columns [64 ch, 64 ch + 64) -> bf16 MN-major B tile
@@ -545,16 +503,6 @@ __global__ void __launch_bounds__(256, 1)
             for (int q = 0; q < 64; ++q) x[q] = -x[q];
             store_row_half(sm + L::dWb + ch * kHalf, r, 0, x, 64);
         }
-    }
-    __syncthreads();
-    tri_inverse64_256(Af, Tf, Mb, tid);
-    {
-        // T as bf16 [r'][64 r] (row-major; read as the MN-major A operand T^T)
-        const int rr = tid >> 2, q0 = (tid & 3) * 2;
-        float t[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) t[e] = Tf[rr * 65 + q0 * 8 + e];
-        store_row_half(sm + L::Tb, rr, q0, t, 16);
     }
     fence_async_smem();
     tc_fence_before();
@@ -755,17 +703,18 @@ cudaError_t launch_grad_delta_tc(const Args& a, cudaStream_t s) {
     const int BH = a.B * a.H;
     if (BH == 0 || a.NC == 0) return cudaSuccess;
     const uint64_t rows = (uint64_t)BH * a.NC * kD;
-    CUtensorMap tm_k{}, tm_ddt{}, tm_sc{}, tm_wt{}, tm_ut{};
+    CUtensorMap tm_k{}, tm_ddt{}, tm_sc{}, tm_wt{}, tm_ut{}, tm_t{};
     const bool ok = tmap_tokens(&tm_k, a.k, a, kD) && tmap_2d(&tm_ddt, a.dDt, 64, rows, 128) &&
                     tmap_2d(&tm_sc, a.Sc, kD, rows, 128) && tmap_2d(&tm_wt, a.Wt, 64, rows, 128) &&
-                    tmap_2d(&tm_ut, a.Ut, 64, rows, 128);
+                    tmap_2d(&tm_ut, a.Ut, 64, rows, 128) &&
+                    tmap_2d(&tm_t, a.Tm, 64, (uint64_t)BH * a.NC * kChunk, 64);
     if (!ok) return cudaErrorInvalidValue;
     const size_t smem = DeltaSmem::Size + 1024;
     cudaError_t e = cudaFuncSetAttribute(grad_delta_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     timing_begin(KK_GRAD_DELTA, s);
-    grad_delta_tc_kernel<<<dim3(a.NC, BH), 256, smem, s>>>(tm_k, tm_ddt, tm_sc, tm_wt, tm_ut, a);
+    grad_delta_tc_kernel<<<dim3(a.NC, BH), 256, smem, s>>>(tm_k, tm_ddt, tm_sc, tm_wt, tm_ut, tm_t, a);
     e = cudaGetLastError();
     timing_end(KK_GRAD_DELTA, s);
     return e;
