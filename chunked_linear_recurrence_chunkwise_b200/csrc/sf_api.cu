@@ -43,6 +43,7 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv, int dtype, bool delta, b
         return o;
     };
     L.G = take(BH * TP * 4);
+    L.Ed = take(BH * NC * 128 * 4);
     L.Wt = take(delta ? BH * TP * dk * tw : 0);
     L.Ut = take(BH * TP * dv * tw);
     L.Sc = take(BH * NC * dk * dv * tw);
@@ -61,6 +62,7 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv, int dtype, bool delta, b
 void bind_slot(Args& a, void* ws, const WsLayout& L, int slot, bool bwd) {
     char* base = (char*)ws + kErrBytes + (size_t)slot * L.slot_bytes;
     a.G = (float*)(base + L.G);
+    a.Ed = (float*)(base + L.Ed);
     a.Wt = base + L.Wt;
     a.Ut = base + L.Ut;
     a.Sc = base + L.Sc;

@@ -37,6 +37,7 @@ struct Args {
     // bf16 for bf16 I/O; chunk-transposed tiles keep the 64 tokens of a chunk
     // contiguous (TP = NC * 64 padded tokens).
     float* G;     // [BH][TP]            fp32 chunk-local inclusive cumsum of g
+    float* Ed;    // [BH][NC][128]       fp32 per chunk: e^{G_C - G_r} (r < 64), then e^{G_r}
     void* Wt;     // [BH][NC][dk][64]    W^T per chunk, W = T diag(beta gamma) K   (delta rule)
     void* Ut;     // [BH][NC][dv][64]    U^T per chunk, U = T diag(beta) V (V for linear attention)
     void* Sc;     // [BH][NC][dv][dk]    S^T entering each chunk
@@ -52,7 +53,7 @@ struct Args {
 
 // Workspace carve-up for a piece of at most T tokens.
 struct WsLayout {
-    size_t G, Wt, Ut, Sc, Dt, dDt, dSc, Pm, Tm, dKp, dGp;  // byte offsets inside one slot
+    size_t G, Ed, Wt, Ut, Sc, Dt, dDt, dSc, Pm, Tm, dKp, dGp;  // byte offsets inside one slot
     size_t slot_bytes;
     size_t total;  // err header + nslots * slot_bytes
 };

@@ -37,51 +37,78 @@ __device__ __forceinline__ size_t tok_index(const Args& a, int b, int t, int h) 
 // T = (I + A)^-1 for a 64 x 64 strictly lower A (fp32, row stride 65), by
 // inverting the four 16 x 16 diagonal blocks with substitution and filling the
 // off-diagonal blocks by distance: T_ij = -T_ii sum_{i>k>=j} A_ik T_kj.
-// Called by all 128 threads of the CTA; ends with a barrier.
+// T is written with row stride 68 (16-byte aligned rows).  Each thread of the
+// off-diagonal phases computes a strip of 4 adjacent columns of one row, so
+// its four multiply-add chains are independent.  Called by all 128 threads of
+// the CTA; ends with a barrier.
+constexpr int kTS = 68;  // row stride of T in floats (16-byte aligned rows)
+constexpr int kMS = 20;  // row stride of the 16 x 16 scratch blocks (16-byte aligned)
+constexpr int kMB = 16 * kMS;
 __device__ void tri_inverse64(const float* Af, float* Tf, float* Mb, int tid) {
-    for (int e = tid; e < 64 * 65; e += 128) Tf[e] = 0.f;
+    for (int e = tid; e < 64 * kTS; e += 128) Tf[e] = 0.f;
     __syncthreads();
     if (tid < 64) {
+        // column `col` of the inverse of diagonal block `o`: right-looking substitution
         const int o = (tid >> 4) * 16, col = tid & 15;
-        float x[16];
+        float v[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) v[r] = (r == col) ? 1.f : 0.f;
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-            float v = (r == col) ? 1.f : 0.f;
+            const float x = (r < col) ? 0.f : v[r];
+            v[r] = x;
 #pragma unroll
-            for (int i = 0; i < r; ++i) v -= Af[(o + r) * 65 + o + i] * x[i];
-            x[r] = (r < col) ? 0.f : v;
+            for (int r2 = r + 1; r2 < 16; ++r2) v[r2] -= Af[(o + r2) * 65 + o + r] * x;
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Tf[(o + r) * 65 + o + col] = x[r];
+        for (int r = 0; r < 16; ++r) Tf[(o + r) * kTS + o + col] = v[r];
     }
     __syncthreads();
     for (int d = 1; d < 4; ++d) {
-        const int nb = 4 - d;
-        for (int e = tid; e < nb * 256; e += 128) {
-            const int m = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+        const int nstrip = (4 - d) * 64;  // blocks (bi, bj) = (m + d, m), 16 rows x 4 strips
+        for (int e = tid; e < nstrip; e += 128) {
+            const int m = e >> 6, rr = (e >> 2) & 15, c4 = (e & 3) * 4;
             const int bi = m + d, bj = m;
-            float acc = 0.f;
-            for (int k = 16 * bj; k < 16 * bi; ++k)
-                acc += Af[(16 * bi + rr) * 65 + k] * Tf[k * 65 + 16 * bj + cc];
-            Mb[m * 272 + rr * 17 + cc] = acc;
+            const float* arow = Af + (16 * bi + rr) * 65;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int k = 16 * bj; k < 16 * bi; ++k) {
+                const float a = arow[k];
+                const float4 t = *(const float4*)(Tf + k * kTS + 16 * bj + c4);
+                acc.x += a * t.x;
+                acc.y += a * t.y;
+                acc.z += a * t.z;
+                acc.w += a * t.w;
+            }
+            *(float4*)(Mb + m * kMB + rr * kMS + c4) = acc;
         }
         __syncthreads();
-        for (int e = tid; e < nb * 256; e += 128) {
-            const int m = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+        for (int e = tid; e < nstrip; e += 128) {
+            const int m = e >> 6, rr = (e >> 2) & 15, c4 = (e & 3) * 4;
             const int bi = m + d, bj = m;
-            float acc = 0.f;
-            for (int k = 0; k <= rr; ++k)
-                acc += Tf[(16 * bi + rr) * 65 + 16 * bi + k] * Mb[m * 272 + k * 17 + cc];
-            Tf[(16 * bi + rr) * 65 + 16 * bj + cc] = -acc;
+            const float* trow = Tf + (16 * bi + rr) * kTS + 16 * bi;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int k = 0; k <= rr; ++k) {
+                const float t = trow[k];
+                const float4 mv = *(const float4*)(Mb + m * kMB + k * kMS + c4);
+                acc.x += t * mv.x;
+                acc.y += t * mv.y;
+                acc.z += t * mv.z;
+                acc.w += t * mv.w;
+            }
+            *(float4*)(Tf + (16 * bi + rr) * kTS + 16 * bj + c4) =
+                make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
         }
         __syncthreads();
     }
 }
 
-// Scales the 128-byte lines (64 bf16) of one row of a tile by f, in place.
-__device__ __forceinline__ void scale_line(uint8_t* line, float f) {
+// Scales the 128-byte line (64 bf16) of row `row` of a tile by f, in place.
+// Lanes of a warp handle different rows; starting each row at a different
+// 16-byte chunk keeps the warp's accesses on distinct banks.
+__device__ __forceinline__ void scale_line(uint8_t* line, int row, float f) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
+    for (int qq = 0; qq < 8; ++qq) {
+        const int q = (qq + row) & 7;
         uint4 u = *(uint4*)(line + q * 16);
         uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -116,9 +143,9 @@ struct IntraSmem {
     static constexpr int Tb = V + kTile;                      // T, bf16 K-major [r][64 i]
     static constexpr int Pst = Tb + kHalf;                    // P staging (kP)
     static constexpr int Af = Pst + (kP ? kHalf : 0);         // fp32 [64][65]
-    static constexpr int Tf = Af + 64 * 65 * 4;               // fp32 [64][65]
-    static constexpr int Mb = Tf + 64 * 65 * 4;               // fp32 [3][16][17]
-    static constexpr int Gs = Mb + 3 * 272 * 4;
+    static constexpr int Tf = Af + 64 * 65 * 4;               // fp32 [64][68]
+    static constexpr int Mb = Tf + 64 * 68 * 4;               // fp32 [3][16][20]
+    static constexpr int Gs = Mb + 3 * 320 * 4;
     static constexpr int Bs = Gs + 256;
     static constexpr int Bar = Bs + 256;
     static constexpr int Misc = Bar + 16;
@@ -181,8 +208,16 @@ __global__ void __launch_bounds__(128)
             if (lane >= off) incl += y;
         }
         const float excl = incl - g0 - g1;
-        Gs[r0] = excl + g0;
-        Gs[r1] = excl + g0 + g1;
+        const float G0 = excl + g0, G1 = excl + g0 + g1;
+        Gs[r0] = G0;
+        Gs[r1] = G1;
+        // decay table of the chunk for the state passes: e^{G_C - G_r}, then e^{G_r}
+        const float gC = __shfl_sync(0xffffffffu, G1, 31);
+        float* ed = a.Ed + ((size_t)bh * NC + c) * 128;
+        ed[r0] = __expf(gC - G0);
+        ed[r1] = __expf(gC - G1);
+        ed[64 + r0] = __expf(G0);
+        ed[64 + r1] = __expf(G1);
     } else if (warp == 1) {
         const int r0 = 2 * lane, r1 = r0 + 1;
         if (kDelta) {
@@ -281,7 +316,7 @@ __global__ void __launch_bounds__(128)
             float t[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-                t[e] = kDelta ? Tf[r * 65 + q * 8 + e] : ((q * 8 + e == r) ? 1.f : 0.f);
+                t[e] = kDelta ? Tf[r * kTS + q * 8 + e] : ((q * 8 + e == r) ? 1.f : 0.f);
             uint4 u;
             u.x = pack_bf16(t[0], t[1]);
             u.y = pack_bf16(t[2], t[3]);
@@ -292,8 +327,8 @@ __global__ void __launch_bounds__(128)
         // K_hat = diag(beta gamma) K and V_hat = diag(beta) V, in place
         const int blk = tid & 1;
         if (kDelta) {
-            scale_line(sm + L::Kb + blk * L::Kblk + r * 128, Bs[r] * __expf(Gs[r]));
-            scale_line(sm + L::V + blk * kHalf + r * 128, Bs[r]);
+            scale_line(sm + L::Kb + blk * L::Kblk + r * 128, r, Bs[r] * __expf(Gs[r]));
+            scale_line(sm + L::V + blk * kHalf + r * 128, r, Bs[r]);
         }
     }
     fence_async_smem();

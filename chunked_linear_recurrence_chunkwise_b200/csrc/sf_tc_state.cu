@@ -65,6 +65,12 @@ constexpr int kD = 128;                 // d_k = d_v on this path
 constexpr int kTile = 128 * 64 * 2;     // one 128-row x 128-byte bf16 tile (16 KB)
 constexpr int kStages = 3;
 
+// Thread layout of both passes: 512 threads = 16 warps; warp w reads TMEM lane
+// quadrant (w & 3), i.e. d_v rows j = 32 (w & 3) + lane, and owns the column
+// quarter p = w >> 2 of every per-row tile (16 of 64 token columns, 32 of 128
+// state columns), so each step's elementwise work is split four ways per row.
+constexpr int kThreads = 512;
+
 // Shared-memory carve-up (byte offsets from a 1024-byte aligned base).
 struct FwdSmem {
     static constexpr int Wt = 0;                          // [stage] W^T  [d_k][64 r]
@@ -73,14 +79,27 @@ struct FwdSmem {
     static constexpr int St = Ut + kStages * kTile;       // S^T operand [2 kblk][d_v][64]
     static constexpr int Dsc = St + 2 * kTile;            // (e^{G_C-G} Delta)^T operand
     static constexpr int Dst = Dsc + kTile;               // Delta^T staging for the store
-    static constexpr int G = Dst + kTile;                 // [stage][64] fp32
-    static constexpr int Bar = G + kStages * 256;         // kStages load barriers + 1 MMA
+    static constexpr int Ed = Dst + kTile;                // [stage][128] fp32 decay table
+    static constexpr int Bar = Ed + kStages * 512;        // kStages load barriers + 1 MMA
     static constexpr int Misc = Bar + (kStages + 1) * 8;  // TMEM base, abort flag
     static constexpr int Size = Misc + 16;
 };
 
+// 32 fp32 values as four bf16 16-byte chunks q0 .. q0+3 of row `row` of a swizzled tile.
+__device__ __forceinline__ void put_row32(uint8_t* tile, int row, int q0, const float* v) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 u;
+        u.x = pack_bf16(v[q * 8 + 0], v[q * 8 + 1]);
+        u.y = pack_bf16(v[q * 8 + 2], v[q * 8 + 3]);
+        u.z = pack_bf16(v[q * 8 + 4], v[q * 8 + 5]);
+        u.w = pack_bf16(v[q * 8 + 6], v[q * 8 + 7]);
+        *(uint4*)(tile + sw128(row, q0 + q)) = u;
+    }
+}
+
 template <bool kDelta>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     state_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_wt,
                         const __grid_constant__ CUtensorMap tm_ut,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -89,17 +108,17 @@ __global__ void __launch_bounds__(256, 1)
     using L = FwdSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    float* Gs = (float*)(sm + L::G);
+    float* Eds = (float*)(sm + L::Ed);
     uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);
     uint64_t* bar_mma = bar_ld + kStages;
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
     volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
+    const int quad = warp & 3, part = warp >> 2;
     const int j = quad * 32 + lane;  // d_v row = TMEM lane
     const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
-    const int NC = a.NC, TP = NC * kChunk;
+    const int NC = a.NC;
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&bar_ld[s], 1);
@@ -117,36 +136,26 @@ __global__ void __launch_bounds__(256, 1)
 
     auto issue_load = [&](int c) {  // thread 0
         const int s = c % kStages;
-        const uint32_t bytes = (kDelta ? kTile : 0) + 2 * kTile + 256;
+        const uint32_t bytes = (kDelta ? kTile : 0) + 2 * kTile + 512;
         mbar_expect_tx(&bar_ld[s], bytes);
         if (kDelta) tma_load_2d(sm + L::Wt + s * kTile, &tm_wt, 0, (bh * NC + c) * kD, &bar_ld[s]);
         tma_load_2d(sm + L::Ut + s * kTile, &tm_ut, 0, (bh * NC + c) * kD, &bar_ld[s]);
         tma_load_4d(sm + L::Kt + s * kTile, &tm_k, 0, h, c * kChunk, b, &bar_ld[s]);
         tma_load_4d(sm + L::Kt + s * kTile + kTile / 2, &tm_k, 64, h, c * kChunk, b, &bar_ld[s]);
-        bulk_load(Gs + s * kChunk, a.G + (size_t)bh * TP + c * kChunk, 256, &bar_ld[s]);
+        bulk_load(Eds + s * 128, a.Ed + ((size_t)bh * NC + c) * 128, 512, &bar_ld[s]);
     };
     int issued = 0;
     if (tid == 0)
         for (; issued < min(kStages, NC); ++issued) issue_load(issued);
 
-    // S^T row j, columns i in [64 half, 64 half + 64): S[q] = S_{i, j}
-    float S[64];
+    // S^T row j, state columns i in [32 part, 32 part + 32): S[q] = S_{i, j}
+    float S[32];
 #pragma unroll
-    for (int q = 0; q < 64; ++q)
-        S[q] = a.S_in ? a.S_in[((size_t)bh * kD + half * 64 + q) * kD + j] : 0.f;
-    uint8_t* St = sm + L::St + half * kTile;
-    auto write_state = [&]() {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            uint4 v;
-            v.x = pack_bf16(S[q * 8 + 0], S[q * 8 + 1]);
-            v.y = pack_bf16(S[q * 8 + 2], S[q * 8 + 3]);
-            v.z = pack_bf16(S[q * 8 + 4], S[q * 8 + 5]);
-            v.w = pack_bf16(S[q * 8 + 6], S[q * 8 + 7]);
-            *(uint4*)(St + sw128(j, q)) = v;
-        }
-    };
-    write_state();
+    for (int q = 0; q < 32; ++q)
+        S[q] = a.S_in ? a.S_in[((size_t)bh * kD + part * 32 + q) * kD + j] : 0.f;
+    uint8_t* St = sm + L::St + (part >> 1) * kTile;
+    const int sq0 = (part & 1) * 4;  // first 16-byte chunk of this thread's 32 state columns
+    put_row32(St, j, sq0, S);
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {
@@ -190,32 +199,33 @@ __global__ void __launch_bounds__(256, 1)
             aborted = true;
             break;
         }
-        float X[32];
+        // Delta^T[j][r] = U^T[j][r] - X^T[j][r] for tokens r in [16 part, 16 part + 16)
+        float X[16];
         if (kDelta) {
             tc_fence_after();
-            tmem_ld32(tX + lane_base + half * 32, X);
+            tmem_ld16(tX + lane_base + part * 16, X);
             tmem_ld_wait();
         } else {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) X[q] = 0.f;
+            for (int q = 0; q < 16; ++q) X[q] = 0.f;
         }
-        const float* G = Gs + s * kChunk;
-        const float gC = G[kChunk - 1];
+        const float* E = Eds + s * 128;
         const uint8_t* Ut = sm + L::Ut + s * kTile;
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-            const int q = half * 4 + qq;  // tokens 8q .. 8q + 7
+        for (int qq = 0; qq < 2; ++qq) {
+            const int q = part * 2 + qq;  // tokens 8q .. 8q + 7
             const uint4 u = *(const uint4*)(Ut + sw128(j, q));
+            const float4 e0 = *(const float4*)(E + q * 8), e1 = *(const float4*)(E + q * 8 + 4);
+            const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
             const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
             uint32_t dw[4], tw[4];
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
                 const float2 uf = unpack_bf16(uw[p]);
-                const int r0 = q * 8 + 2 * p;
                 const float d0 = uf.x - X[qq * 8 + 2 * p];
                 const float d1 = uf.y - X[qq * 8 + 2 * p + 1];
                 dw[p] = pack_bf16(d0, d1);
-                tw[p] = pack_bf16(d0 * __expf(gC - G[r0]), d1 * __expf(gC - G[r0 + 1]));
+                tw[p] = pack_bf16(d0 * ev[2 * p], d1 * ev[2 * p + 1]);
             }
             *(uint4*)(sm + L::Dst + sw128(j, q)) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
             *(uint4*)(sm + L::Dsc + sw128(j, q)) = make_uint4(tw[0], tw[1], tw[2], tw[3]);
@@ -251,18 +261,16 @@ __global__ void __launch_bounds__(256, 1)
             break;
         }
         tc_fence_after();
-        float P0[32], P1[32];
-        tmem_ld32(tP + lane_base + half * 64, P0);
-        tmem_ld32(tP + lane_base + half * 64 + 32, P1);
-        tmem_ld_wait();
-        const float gam = __expf(gC);
+        {
+            float P[32];
+            tmem_ld32(tP + lane_base + part * 32, P);
+            tmem_ld_wait();
+            const float gam = E[64 + kChunk - 1];  // gamma_C
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-            S[q] = gam * S[q] + P0[q];
-            S[32 + q] = gam * S[32 + q] + P1[q];
+            for (int q = 0; q < 32; ++q) S[q] = gam * S[q] + P[q];
         }
         if (c + 1 < NC) {
-            write_state();
+            put_row32(St, j, sq0, S);
             fence_async_smem();
         }
         tc_fence_before();
@@ -275,7 +283,7 @@ __global__ void __launch_bounds__(256, 1)
     }
     if (!aborted && a.S_out) {
 #pragma unroll
-        for (int q = 0; q < 64; ++q) a.S_out[((size_t)bh * kD + half * 64 + q) * kD + j] = S[q];
+        for (int q = 0; q < 32; ++q) a.S_out[((size_t)bh * kD + part * 32 + q) * kD + j] = S[q];
     }
     if (tid == 0) {
         if (aborted) {
@@ -293,7 +301,6 @@ __global__ void __launch_bounds__(256, 1)
     }
 }
 
-
 // Shared-memory carve-up of the reverse pass (byte offsets from a 1024-aligned base).
 constexpr int kBStages = 2;
 struct BwdSmem {
@@ -305,8 +312,8 @@ struct BwdSmem {
     static constexpr int St = P + kBStages * 8192;        // dS^T operand [2 kblk][d_v][64]
     static constexpr int Dop = St + 2 * kTile;            // dDelta^T [d_v][64 r] (operand + store)
     static constexpr int Dv = Dop + kTile;                // dv staging [2][64 r][64 d_v] (no beta)
-    static constexpr int G = Dv + kTile;                  // [stage][64] fp32
-    static constexpr int Bar = G + kBStages * 256;
+    static constexpr int Ed = Dv + kTile;                 // [stage][128] fp32 decay table
+    static constexpr int Bar = Ed + kBStages * 512;
     static constexpr int Misc = Bar + (kBStages + 1) * 8;
     static constexpr int Size = Misc + 16;
 };
@@ -318,7 +325,7 @@ struct BwdSmem {
 // dDelta = P^T dO + Ktil dS').  Stores dS'^T of every chunk and dDelta^T (or
 // dv = dDelta directly for linear attention).
 template <bool kDelta>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     state_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_do,
                         const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_wt,
                         const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_dsc,
@@ -327,17 +334,17 @@ __global__ void __launch_bounds__(256, 1)
     using L = BwdSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    float* Gs = (float*)(sm + L::G);
+    float* Eds = (float*)(sm + L::Ed);
     uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);
     uint64_t* bar_mma = bar_ld + kBStages;
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
     volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
+    const int quad = warp & 3, part = warp >> 2;
     const int j = quad * 32 + lane;  // d_v row = TMEM lane
     const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
-    const int NC = a.NC, TP = NC * kChunk;
+    const int NC = a.NC;
 
     if (tid == 0) {
         for (int s = 0; s < kBStages; ++s) mbar_init(&bar_ld[s], 1);
@@ -356,7 +363,7 @@ __global__ void __launch_bounds__(256, 1)
     // n-th load (n = 0, 1, ...) is chunk NC - 1 - n, stage n % 2
     auto issue_load = [&](int n) {
         const int c = NC - 1 - n, s = n % kBStages;
-        const uint32_t bytes = 3 * kTile + 8192 + (kDelta ? kTile : 0) + 256;
+        const uint32_t bytes = 3 * kTile + 8192 + (kDelta ? kTile : 0) + 512;
         mbar_expect_tx(&bar_ld[s], bytes);
         tma_load_4d(sm + L::Kt + s * kTile, &tm_k, 0, h, c * kChunk, b, &bar_ld[s]);
         tma_load_4d(sm + L::Kt + s * kTile + 8192, &tm_k, 64, h, c * kChunk, b, &bar_ld[s]);
@@ -366,30 +373,20 @@ __global__ void __launch_bounds__(256, 1)
         tma_load_4d(sm + L::Q + s * kTile + 8192, &tm_q, 64, h, c * kChunk, b, &bar_ld[s]);
         if (kDelta) tma_load_2d(sm + L::Wt + s * kTile, &tm_wt, 0, (bh * NC + c) * kD, &bar_ld[s]);
         tma_load_2d(sm + L::P + s * 8192, &tm_p, 0, (bh * NC + c) * kChunk, &bar_ld[s]);
-        bulk_load(Gs + s * kChunk, a.G + (size_t)bh * TP + c * kChunk, 256, &bar_ld[s]);
+        bulk_load(Eds + s * 128, a.Ed + ((size_t)bh * NC + c) * 128, 512, &bar_ld[s]);
     };
     int issued = 0;
     if (tid == 0)
         for (; issued < min(kBStages, NC); ++issued) issue_load(issued);
 
-    // dS^T row j, columns i in [64 half, 64 half + 64): S[q] = dS_{i, j}
-    float S[64];
+    // dS^T row j, state columns i in [32 part, 32 part + 32): S[q] = dS_{i, j}
+    float S[32];
 #pragma unroll
-    for (int q = 0; q < 64; ++q)
-        S[q] = a.dS_out ? a.dS_out[((size_t)bh * kD + half * 64 + q) * kD + j] : 0.f;
-    uint8_t* St = sm + L::St + half * kTile;
-    auto write_state = [&]() {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            uint4 v;
-            v.x = pack_bf16(S[q * 8 + 0], S[q * 8 + 1]);
-            v.y = pack_bf16(S[q * 8 + 2], S[q * 8 + 3]);
-            v.z = pack_bf16(S[q * 8 + 4], S[q * 8 + 5]);
-            v.w = pack_bf16(S[q * 8 + 6], S[q * 8 + 7]);
-            *(uint4*)(St + sw128(j, q)) = v;
-        }
-    };
-    write_state();
+    for (int q = 0; q < 32; ++q)
+        S[q] = a.dS_out ? a.dS_out[((size_t)bh * kD + part * 32 + q) * kD + j] : 0.f;
+    uint8_t* St = sm + L::St + (part >> 1) * kTile;
+    const int sq0 = (part & 1) * 4;
+    put_row32(St, j, sq0, S);
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {
@@ -438,49 +435,49 @@ __global__ void __launch_bounds__(256, 1)
             break;
         }
         tc_fence_after();
-        const float* G = Gs + s * kChunk;
-        const float gC = G[kChunk - 1];
+        const float* E = Eds + s * 128;
         {
-            float y1[32], y2[32];
-            tmem_ld32(tY1 + lane_base + half * 32, y1);
-            tmem_ld32(tY2 + lane_base + half * 32, y2);
+            float y1[16], y2[16];
+            tmem_ld16(tY1 + lane_base + part * 16, y1);
+            tmem_ld16(tY2 + lane_base + part * 16, y2);
             tmem_ld_wait();
-            float d[32];
+            float d[16];
 #pragma unroll
-            for (int q = 0; q < 32; ++q) d[q] = __expf(gC - G[half * 32 + q]) * y1[q] + y2[q];
+            for (int q = 0; q < 16; ++q) d[q] = E[part * 16 + q] * y1[q] + y2[q];
             if (kDelta) {
 #pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
+                for (int qq = 0; qq < 2; ++qq) {
                     uint4 u;
                     u.x = pack_bf16(d[qq * 8 + 0], d[qq * 8 + 1]);
                     u.y = pack_bf16(d[qq * 8 + 2], d[qq * 8 + 3]);
                     u.z = pack_bf16(d[qq * 8 + 4], d[qq * 8 + 5]);
                     u.w = pack_bf16(d[qq * 8 + 6], d[qq * 8 + 7]);
-                    *(uint4*)(sm + L::Dop + sw128(j, half * 4 + qq)) = u;
+                    *(uint4*)(sm + L::Dop + sw128(j, part * 2 + qq)) = u;
                 }
             } else {
                 // linear attention: dv = dDelta, staged token-major for a TMA store
                 const uint32_t jb = (uint32_t)(j >> 6) * 8192, jq = (j & 63) >> 3, je = (j & 7) * 2;
 #pragma unroll
-                for (int q = 0; q < 32; ++q)
-                    *(__nv_bfloat16*)(sm + L::Dv + jb + sw128(half * 32 + q, jq) + je) =
+                for (int q = 0; q < 16; ++q)
+                    *(__nv_bfloat16*)(sm + L::Dv + jb + sw128(part * 16 + q, jq) + je) =
                         __float2bfloat16_rn(d[q]);
             }
         }
-        if (tid < 128) {  // diag(gamma) Q in place, one 128-byte line per thread
-            const int r = tid & 63, blk = tid >> 6;
-            uint8_t* line = sm + L::Q + s * kTile + blk * 8192 + r * 128;
-            const float f = __expf(G[r]);
+        if (tid < 256) {  // diag(gamma) Q in place, half a 128-byte line per thread
+            const int line = tid >> 1, r = line & 63, blk = line >> 6;
+            uint8_t* ln = sm + L::Q + s * kTile + blk * 8192 + r * 128 + (tid & 1) * 64;
+            const float f = E[64 + r];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                uint4 u = *(uint4*)(line + q * 16);
+            for (int qq = 0; qq < 4; ++qq) {
+                const int q = (qq + (line >> 1)) & 3;  // lanes on distinct banks
+                uint4 u = *(uint4*)(ln + q * 16);
                 uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
                     const float2 x = unpack_bf16(w[p]);
                     w[p] = pack_bf16(x.x * f, x.y * f);
                 }
-                *(uint4*)(line + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+                *(uint4*)(ln + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
             }
         }
         fence_async_smem();
@@ -527,19 +524,15 @@ __global__ void __launch_bounds__(256, 1)
         }
         tc_fence_after();
         {
-            float z0[32], z1[32];
-            tmem_ld32(tZ + lane_base + half * 64, z0);
-            tmem_ld32(tZ + lane_base + half * 64 + 32, z1);
+            float z[32];
+            tmem_ld32(tZ + lane_base + part * 32, z);
             tmem_ld_wait();
-            const float gam = __expf(gC);
+            const float gam = E[64 + kChunk - 1];
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                S[q] = gam * S[q] + z0[q];
-                S[32 + q] = gam * S[32 + q] + z1[q];
-            }
+            for (int q = 0; q < 32; ++q) S[q] = gam * S[q] + z[q];
         }
         if (c > 0) {
-            write_state();
+            put_row32(St, j, sq0, S);
             fence_async_smem();
         }
         tc_fence_before();
@@ -552,7 +545,7 @@ __global__ void __launch_bounds__(256, 1)
     }
     if (!aborted && a.dS_in) {
 #pragma unroll
-        for (int q = 0; q < 64; ++q) a.dS_in[((size_t)bh * kD + half * 64 + q) * kD + j] = S[q];
+        for (int q = 0; q < 32; ++q) a.dS_in[((size_t)bh * kD + part * 32 + q) * kD + j] = S[q];
     }
     if (tid == 0) {
         if (aborted) {
@@ -606,7 +599,7 @@ cudaError_t launch_state_fwd_tc(const Args& a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     timing_begin(KK_STATE_FWD, s);
-    kern<<<BH, 256, smem, s>>>(tm_wt, tm_ut, tm_k, tm_sc, tm_dt, a);
+    kern<<<BH, kThreads, smem, s>>>(tm_wt, tm_ut, tm_k, tm_sc, tm_dt, a);
     e = cudaGetLastError();
     timing_end(KK_STATE_FWD, s);
     return e;
@@ -631,7 +624,7 @@ cudaError_t launch_state_bwd_tc(const Args& a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     timing_begin(KK_STATE_BWD, s);
-    kern<<<BH, 256, smem, s>>>(tm_k, tm_do, tm_q, tm_wt, tm_p, tm_dsc, tm_ddt, tm_dv, a);
+    kern<<<BH, kThreads, smem, s>>>(tm_k, tm_do, tm_q, tm_wt, tm_p, tm_dsc, tm_ddt, tm_dv, a);
     e = cudaGetLastError();
     timing_end(KK_STATE_BWD, s);
     return e;
