@@ -130,6 +130,10 @@ def kernel_units(name: str, w) -> dict:
             # read q, k, dO, Delta^T, S^T, dS'^T, G, dKp, dGp; write dq, dk, dg
             "grad_attn": (4 * tile + 2 * st + C * f + C * d * f + C * f + 2 * tile + C * f,
                           2 * mm(C, C, d) + 2 * mm(C, d, d) + 2 * mm(C, d, C)),
+            # read q, k, v, dO, W^T, U^T, T, Delta^T, dDelta^T, S^T, dS'^T, G, beta;
+            # write dq, dk, dv, dg, dbeta
+            "grad_fused": (8 * tile + C * C * e + 2 * st + 2 * C * f + 3 * tile + 2 * C * f,
+                           5 * mm(C, C, d) + 3 * mm(C, d, d) + 5 * mm(C, d, C)),
         }
     else:
         e = 2 if w.dtype == "bf16" else 4

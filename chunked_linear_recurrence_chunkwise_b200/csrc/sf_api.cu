@@ -16,6 +16,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "../../include/sf.h"
@@ -36,6 +37,8 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv, int dtype, bool delta, b
     const size_t NC = (size_t)(T + kChunk - 1) / kChunk;
     const size_t TP = NC * kChunk;
     const size_t tw = dtype == SF_BF16 ? 2 : 4;  // intermediates follow the I/O precision
+    // the tensor-core path computes every delta-rule gradient in one kernel: no dKp / dGp
+    const bool split_grads = !(dtype == SF_BF16 && dk == 128 && dv == 128);
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t o = off;
@@ -52,8 +55,8 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv, int dtype, bool delta, b
     L.dSc = take(bwd ? BH * NC * dk * dv * tw : 0);
     L.Pm = take(bwd ? BH * NC * kChunk * kChunk * tw : 0);
     L.Tm = take(bwd && delta ? BH * NC * kChunk * kChunk * tw : 0);
-    L.dKp = take(bwd && delta ? BH * TP * dk * 4 : 0);
-    L.dGp = take(bwd && delta ? BH * TP * 4 : 0);
+    L.dKp = take(bwd && delta && split_grads ? BH * TP * dk * 4 : 0);
+    L.dGp = take(bwd && delta && split_grads ? BH * TP * 4 : 0);
     L.slot_bytes = off;
     L.total = kErrBytes + (size_t)nslots * L.slot_bytes;
     return L;
@@ -80,6 +83,7 @@ void bind_slot(Args& a, void* ws, const WsLayout& L, int slot, bool bwd) {
 namespace {
 struct TimingRec {
     int kind;
+    cudaStream_t stream;
     cudaEvent_t e0, e1;
 };
 bool g_timing_on = false;
@@ -101,14 +105,14 @@ cudaEvent_t pool_get() {
 }  // namespace
 
 const char* kernel_name(int kind) {
-    static const char* names[KK_COUNT] = {"intra_fwd", "state_fwd",  "output",    "dd_pre",
-                                          "state_bwd", "grad_delta", "grad_attn", "intra_bwd"};
+    static const char* names[KK_COUNT] = {"intra_fwd", "state_fwd", "output",    "dd_pre",    "state_bwd",
+                                          "grad_delta", "grad_attn", "intra_bwd", "grad_fused"};
     return (kind >= 0 && kind < KK_COUNT) ? names[kind] : "?";
 }
 
 void timing_begin(int kind, cudaStream_t s) {
     if (!g_timing_on) return;
-    TimingRec r{kind, pool_get(), pool_get()};
+    TimingRec r{kind, s, pool_get(), pool_get()};
     cudaEventRecord(r.e0, s);
     g_recs.push_back(r);
 }
@@ -222,17 +226,17 @@ cudaError_t run_bwd_state(Args a, cudaStream_t st) {
 
 // The per-chunk gradients of one piece (after its reverse pass).
 cudaError_t run_bwd_chunk_grads(const Args& a, cudaStream_t st) {
+    if (tc_eligible(a)) return a.beta ? launch_grad_fused_tc(a, st) : launch_grad_attn_tc(a, st);
     cudaError_t e = cudaSuccess;
-    if (a.beta) e = tc_eligible(a) ? launch_grad_delta_tc(a, st) : launch_grad_delta(a, st);
-    if (e == cudaSuccess) e = tc_eligible(a) ? launch_grad_attn_tc(a, st) : launch_grad_attn(a, st);
+    if (a.beta) e = launch_grad_delta(a, st);
+    if (e == cudaSuccess) e = launch_grad_attn(a, st);
     return e;
 }
 
 // The dS-dependent part: reverse state pass, then the per-chunk gradients.
 cudaError_t run_bwd_grads(const Args& a, cudaStream_t st) {
     cudaError_t e = tc_eligible(a) ? launch_state_bwd_tc(a, st) : launch_state_bwd(a, st);
-    if (e == cudaSuccess && a.beta) e = tc_eligible(a) ? launch_grad_delta_tc(a, st) : launch_grad_delta(a, st);
-    if (e == cudaSuccess) e = tc_eligible(a) ? launch_grad_attn_tc(a, st) : launch_grad_attn(a, st);
+    if (e == cudaSuccess) e = run_bwd_chunk_grads(a, st);
     return e;
 }
 
@@ -284,6 +288,32 @@ struct EventSet {
         return cudaSuccess;
     }
 };
+
+// The sequential state passes of the sub-sequence drivers run on a stream of
+// the device's greatest priority, created on first use (one per device, kept
+// for the life of the process): whenever SMs free up, the block scheduler then
+// serves the critical path before the parallel work queued on the aux stream.
+cudaError_t critical_stream(cudaStream_t* out) {
+    static std::mutex mu;
+    static std::vector<cudaStream_t> per_dev;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if ((int)per_dev.size() <= dev) per_dev.resize(dev + 1, nullptr);
+    if (!per_dev[dev]) {
+        int least = 0, greatest = 0;
+        e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+        if (e == cudaSuccess)
+            e = cudaStreamCreateWithPriority(&per_dev[dev], cudaStreamNonBlocking, greatest);
+        if (e != cudaSuccess) {
+            per_dev[dev] = nullptr;
+            return e;
+        }
+    }
+    *out = per_dev[dev];
+    return cudaSuccess;
+}
 
 }  // namespace
 
@@ -388,17 +418,21 @@ sf_status sf_fwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
     const size_t es = esize(s);
     const int ld_t = s->ld_t ? s->ld_t : s->T;
 
-    // Schedule: the main stream carries only the sequential state passes; the
-    // aux stream runs the parallel work around them (intra of pieces i+1, i+2
+    // Schedule: the critical stream carries only the sequential state passes;
+    // the aux stream runs the parallel work around them (intra of pieces i+1, i+2
     // ahead, output of piece i behind), three workspace slots in flight.
     constexpr int NS = kSeqSlots;
     EventSet evs;
-    SF_TRY(evs.make(2 * NS + 2));
+    SF_TRY(evs.make(2 * NS + 3));
     cudaEvent_t* ev_intra = &evs.ev[0];   // intra of the slot's piece done (aux)
-    cudaEvent_t* ev_state = &evs.ev[NS];  // state pass of the slot's piece done (main)
+    cudaEvent_t* ev_state = &evs.ev[NS];  // state pass of the slot's piece done (critical)
     cudaEvent_t ev_start = evs.ev[2 * NS], ev_aux_done = evs.ev[2 * NS + 1];
+    cudaEvent_t ev_crit_done = evs.ev[2 * NS + 2];
+    cudaStream_t sc = sm;  // the state passes' stream
+    if (sa != sm) SF_TRY(critical_stream(&sc));
     SF_TRY(cudaEventRecord(ev_start, sm));
     SF_TRY(cudaStreamWaitEvent(sa, ev_start, 0));
+    SF_TRY(cudaStreamWaitEvent(sc, ev_start, 0));
 
     auto piece = [&](int i) {
         Args a = make_args(s);
@@ -424,16 +458,16 @@ sf_status sf_fwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
         return a;
     };
 
-    if (S_saved) SF_TRY(copy_state(S_saved, S_in, nstate, sm));
+    if (S_saved) SF_TRY(copy_state(S_saved, S_in, nstate, sc));
     for (int j = 0; j < std::min(2, n_sub); ++j) {
         SF_TRY(run_intra(piece(j), sa));
         SF_TRY(cudaEventRecord(ev_intra[j % NS], sa));
     }
     for (int i = 0; i < n_sub; ++i) {
         const Args a = piece(i);
-        SF_TRY(cudaStreamWaitEvent(sm, ev_intra[i % NS], 0));
-        SF_TRY(run_state_output(a, sm, false));
-        SF_TRY(cudaEventRecord(ev_state[i % NS], sm));
+        SF_TRY(cudaStreamWaitEvent(sc, ev_intra[i % NS], 0));
+        SF_TRY(run_state_output(a, sc, false));
+        SF_TRY(cudaEventRecord(ev_state[i % NS], sc));
         if (i + 2 < n_sub) {  // its slot's previous piece (i-1) finished its output on this stream
             SF_TRY(run_intra(piece(i + 2), sa));
             SF_TRY(cudaEventRecord(ev_intra[(i + 2) % NS], sa));
@@ -442,7 +476,9 @@ sf_status sf_fwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
         SF_TRY(output(a, sa));
     }
     SF_TRY(cudaEventRecord(ev_aux_done, sa));
+    SF_TRY(cudaEventRecord(ev_crit_done, sc));
     SF_TRY(cudaStreamWaitEvent(sm, ev_aux_done, 0));
+    SF_TRY(cudaStreamWaitEvent(sm, ev_crit_done, 0));
     return SF_OK;
 }
 
@@ -475,18 +511,22 @@ sf_status sf_bwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
     const size_t es = esize(s);
     const int ld_t = s->ld_t ? s->ld_t : s->T;
 
-    // Schedule (pieces in reverse): the main stream carries the sequential
+    // Schedule (pieces in reverse): the critical stream carries the sequential
     // passes of each piece (forward-state recompute, then the reverse dS pass);
     // the aux stream runs the parallel work (intra recompute two pieces ahead,
     // per-chunk gradients one piece behind), three workspace slots in flight.
     constexpr int NS = kSeqSlots;
     EventSet evs;
-    SF_TRY(evs.make(2 * NS + 2));
+    SF_TRY(evs.make(2 * NS + 3));
     cudaEvent_t* ev_prep = &evs.ev[0];    // intra recompute of the slot's piece done (aux)
-    cudaEvent_t* ev_state = &evs.ev[NS];  // reverse pass of the slot's piece done (main)
+    cudaEvent_t* ev_state = &evs.ev[NS];  // reverse pass of the slot's piece done (critical)
     cudaEvent_t ev_start = evs.ev[2 * NS], ev_aux_done = evs.ev[2 * NS + 1];
+    cudaEvent_t ev_crit_done = evs.ev[2 * NS + 2];
+    cudaStream_t sc = sm;  // the state passes' stream
+    if (sa != sm) SF_TRY(critical_stream(&sc));
     SF_TRY(cudaEventRecord(ev_start, sm));
     SF_TRY(cudaStreamWaitEvent(sa, ev_start, 0));
+    SF_TRY(cudaStreamWaitEvent(sc, ev_start, 0));
 
     auto piece = [&](int i) {
         Args a = make_args(s);
@@ -520,9 +560,9 @@ sf_status sf_bwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
     }
     for (int i = n_sub - 1; i >= 0; --i) {
         const Args a = piece(i);
-        SF_TRY(cudaStreamWaitEvent(sm, ev_prep[i % NS], 0));
-        SF_TRY(run_bwd_state(a, sm));
-        SF_TRY(cudaEventRecord(ev_state[i % NS], sm));
+        SF_TRY(cudaStreamWaitEvent(sc, ev_prep[i % NS], 0));
+        SF_TRY(run_bwd_state(a, sc));
+        SF_TRY(cudaEventRecord(ev_state[i % NS], sc));
         if (i - 2 >= 0) {  // its slot's previous piece (i+1) finished its gradients on this stream
             SF_TRY(intra(piece(i - 2), true, sa));
             SF_TRY(cudaEventRecord(ev_prep[(i - 2) % NS], sa));
@@ -531,7 +571,9 @@ sf_status sf_bwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
         SF_TRY(run_bwd_chunk_grads(a, sa));
     }
     SF_TRY(cudaEventRecord(ev_aux_done, sa));
+    SF_TRY(cudaEventRecord(ev_crit_done, sc));
     SF_TRY(cudaStreamWaitEvent(sm, ev_aux_done, 0));
+    SF_TRY(cudaStreamWaitEvent(sm, ev_crit_done, 0));
     return SF_OK;
 }
 
@@ -588,6 +630,27 @@ int sf_timing_read(int cap, const char** names, int* launches, double* ms) {
         if (names) names[i] = kernel_name(i);
         if (launches) launches[i] = g_launches[i];
         if (ms) ms[i] = g_ms[i];
+    }
+    return n;
+}
+
+int sf_timing_trace(int cap, int* kinds, int* streams, double* start_ms, double* end_ms) {
+    cudaDeviceSynchronize();
+    std::vector<cudaStream_t> seen;
+    int n = 0;
+    for (const TimingRec& r : g_recs) {
+        if (n >= cap) break;
+        int si = 0;
+        while (si < (int)seen.size() && seen[si] != r.stream) ++si;
+        if (si == (int)seen.size()) seen.push_back(r.stream);
+        float t0 = -1.f, t1 = -1.f;
+        cudaEventElapsedTime(&t0, g_recs.front().e0, r.e0);
+        cudaEventElapsedTime(&t1, g_recs.front().e0, r.e1);
+        if (kinds) kinds[n] = r.kind;
+        if (streams) streams[n] = si;
+        if (start_ms) start_ms[n] = t0;
+        if (end_ms) end_ms[n] = t1;
+        ++n;
     }
     return n;
 }

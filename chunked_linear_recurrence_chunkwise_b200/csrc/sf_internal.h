@@ -86,6 +86,8 @@ cudaError_t launch_state_bwd_tc(const Args& a, cudaStream_t s);
 cudaError_t launch_grad_attn_tc(const Args& a, cudaStream_t s);
 // dv, dbeta and the delta-rule parts dKp, dGp
 cudaError_t launch_grad_delta_tc(const Args& a, cudaStream_t s);
+// every per-chunk gradient of the gated delta rule in one kernel (dq, dk, dv, dg, dbeta)
+cudaError_t launch_grad_fused_tc(const Args& a, cudaStream_t s);
 
 // Per-kernel timing registry (sf_timing_*).
 enum KernelKind {
@@ -97,6 +99,7 @@ enum KernelKind {
     KK_GRAD_DELTA,
     KK_GRAD_ATTN,
     KK_INTRA_BWD,
+    KK_GRAD_FUSED,
     KK_COUNT
 };
 const char* kernel_name(int kind);

@@ -1,0 +1,561 @@
+// Fused per-chunk gradient kernel of the gated delta rule (sm_100a).
+//
+// One CTA per chunk-head computes dq, dk, dv, dbeta and dg from one load of
+// its inputs (the algebra is the chunkwise backward of the delta rule):
+//   P = (Q K^T) .* Gamma,  dP = (dO Delta^T) .* lower,  F = dP .* Gamma
+//   dQ = diag(gamma) dO S^T + F K
+//   dVhat = T^T dDelta,  dW = -dDelta S^T,  dKhat = T^T dW
+//   dA = -(dKhat W^T + dVhat U^T) .* strictly lower,  dB = diag(beta) dA,  E = dB .* Gamma
+//   dK = F^T Q + diag(e^{G_C - G}) Delta dS'^T + diag(beta gamma) dKhat + (E + E^T) K
+//   dV = diag(beta) dVhat
+//   dbeta_r = <V_r, dVhat_r> + gamma_r <K_r, dKhat_r> + sum_t dA_rt B_rt
+//   dG_r = rowsum(dP.*P) - colsum(dP.*P) + rowsum(dB.*B) - colsum(dB.*B)
+//          + gamma_r <(Q S)_r, dO_r> + beta_r gamma_r <K_r, dKhat_r>
+//          - e^{G_C - G_r} <K_r, (Delta dS'^T)_r>
+//          + [last row] (sum_r e^{G_C - G_r} <K_r, (Delta dS'^T)_r> + gamma_C <S, dS'>)
+//   dg = reverse in-chunk cumsum of dG
+// with T = (I + diag(beta) B)^-1 taken from the backward intra kernel.
+//
+// The UMMAs (all M = 64) run in four phases; every product that needs only
+// loaded data is issued in the first.  Accumulators are paired at TMEM lane
+// offsets 0 and 16 (rows 16 w + l of the lane-0 tile sit in lanes 32 w + l,
+// those of the lane-16 tile in lanes 32 w + 16 + l):
+//   cols [0, 64):    Q K^T          | dO Delta^T, later dA
+//   cols [64, 128):  K K^T          | -
+//   cols [128, 256): dQ             | dK
+//   cols [256, 384): dW, dKhat, dKp | dVhat
+// Shared memory of operands that die after the first phase is reused for the
+// later tiles and scratch (about 209 KB in all, one CTA per SM).
+
+#include <cuda.h>
+
+#include "../../include/sf.h"
+#include "sf_internal.h"
+#include "tc_common.cuh"
+
+namespace sf {
+namespace {
+
+using namespace tc;
+
+constexpr int kD = 128;
+constexpr int kTile = 16384;
+constexpr int kHalf = 8192;
+
+struct FusedSmem {
+    static constexpr int Q = 0;                   // [dkblk][64 r][64]
+    static constexpr int K = Q + kTile;           // [dkblk][64 r][64]
+    static constexpr int dO = K + kTile;          // [dvblk][64 r][64]
+    static constexpr int Wt = dO + kTile;         // W^T [128 i][64 r]
+    static constexpr int Ut = Wt + kTile;         // U^T [128 j][64 r]
+    static constexpr int Tb = Ut + kTile;         // T [r'][64 r]
+    static constexpr int F = Tb + kHalf;          // F = dP .* Gamma [r][64 t]; later E + E^T
+    static constexpr int Dt = F + kHalf;          // Delta^T [128 j][64 t]; later dW (bf16 [iblk][r][64])
+    static constexpr int dDt = Dt + kTile;        // dDelta^T [128 j][64 r]; later dVhat (bf16)
+    static constexpr int St = dDt + kTile;        // S^T [2][128 j][64 i]; later dKhat (bf16)
+    static constexpr int dSt = St + 2 * kTile;    // dS'^T [2][128 j][64 i]; later E (fp32 [64][65])
+    static constexpr int PD = dSt + 2 * kTile;    // fp32 [64][65]: dP .* P, later dB .* B
+    static constexpr int Gs = PD + 64 * 65 * 4;   // 64 fp32
+    static constexpr int Bs = Gs + 256;           // 64 fp32
+    static constexpr int cs1 = Bs + 256;          // 64 fp32: column sums of dP .* P
+    static constexpr int part = cs1 + 256;        // fp32 [14][64] per-row partial sums
+    static constexpr int red = part + 14 * 256;   // fp32 [16]: per-warp <S, dS'> and last-row sums
+    static constexpr int Bar = red + 64;
+    static constexpr int Misc = Bar + 16;
+    static constexpr int Size = Misc + 16;
+};
+
+__device__ __forceinline__ size_t tok_index(const Args& a, int b, int t, int h) {
+    return ((size_t)b * a.ld_t + t) * a.H + h;
+}
+
+// <row r of a 128-byte-swizzled bf16 tile block, x[0..63]>
+__device__ __forceinline__ float dot_row(const uint8_t* blk, int r, const float* x) {
+    float acc = 0.f;
+#pragma unroll
+    for (int qc = 0; qc < 8; ++qc) {
+        const uint4 u = *(const uint4*)(blk + sw128(r, qc));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float2 f = unpack_bf16(w[p]);
+            acc += f.x * x[qc * 8 + 2 * p] + f.y * x[qc * 8 + 2 * p + 1];
+        }
+    }
+    return acc;
+}
+
+// n fp32 values as bf16 16-byte chunks q0 .. q0 + n/8 - 1 of row `row` of a swizzled tile.
+__device__ __forceinline__ void put_row(uint8_t* tile, int row, int q0, const float* v, int n) {
+#pragma unroll
+    for (int qq = 0; qq < n / 8; ++qq) {
+        uint4 u;
+        u.x = pack_bf16(v[qq * 8 + 0], v[qq * 8 + 1]);
+        u.y = pack_bf16(v[qq * 8 + 2], v[qq * 8 + 3]);
+        u.z = pack_bf16(v[qq * 8 + 4], v[qq * 8 + 5]);
+        u.w = pack_bf16(v[qq * 8 + 6], v[qq * 8 + 7]);
+        *(uint4*)(tile + sw128(row, q0 + qq)) = u;
+    }
+}
+
+__global__ void __launch_bounds__(256, 1)
+    grad_fused_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_wt,
+                         const __grid_constant__ CUtensorMap tm_ut, const __grid_constant__ CUtensorMap tm_t,
+                         const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_ddt,
+                         const __grid_constant__ CUtensorMap tm_sc, const __grid_constant__ CUtensorMap tm_dsc,
+                         const Args a) {
+    using L = FusedSmem;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    float* Gs = (float*)(sm + L::Gs);
+    float* Bs = (float*)(sm + L::Bs);
+    float* cs1 = (float*)(sm + L::cs1);
+    float* PD = (float*)(sm + L::PD);
+    float* Ef = (float*)(sm + L::dSt);
+    float* part = (float*)(sm + L::part);
+    float* red = (float*)(sm + L::red);
+    uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);
+    uint64_t* bar_mma = bar_ld + 1;
+    uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
+    volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
+
+    const int c = blockIdx.x, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+    const int NC = a.NC, TP = NC * kChunk;
+    const int t0 = c * kChunk, Lr = min(kChunk, a.T - t0);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, ch = warp >> 2;  // TMEM lane quadrant, column half
+    const bool hi = lane >= 16;                 // lanes 16-31: the lane-16 tiles
+    const int r = 16 * quad + (lane & 15);      // chunk row of this thread's tiles
+
+    if (tid == 0) {
+        mbar_init(bar_ld, 1);
+        mbar_init(bar_mma, 1);
+        *s_abort = 0;
+        fence_barrier_init();
+        mbar_expect_tx(bar_ld, 6 * kHalf + 2 * kTile + kHalf + 2 * kTile + 4 * kTile + 256);
+        const int rowD = (bh * NC + c) * kD, rowC = (bh * NC + c) * kChunk;
+        tma_load_4d(sm + L::Q, &tm_q, 0, h, t0, b, bar_ld);
+        tma_load_4d(sm + L::Q + kHalf, &tm_q, 64, h, t0, b, bar_ld);
+        tma_load_4d(sm + L::K, &tm_k, 0, h, t0, b, bar_ld);
+        tma_load_4d(sm + L::K + kHalf, &tm_k, 64, h, t0, b, bar_ld);
+        tma_load_4d(sm + L::dO, &tm_do, 0, h, t0, b, bar_ld);
+        tma_load_4d(sm + L::dO + kHalf, &tm_do, 64, h, t0, b, bar_ld);
+        tma_load_2d(sm + L::Wt, &tm_wt, 0, rowD, bar_ld);
+        tma_load_2d(sm + L::Ut, &tm_ut, 0, rowD, bar_ld);
+        tma_load_2d(sm + L::Tb, &tm_t, 0, rowC, bar_ld);
+        tma_load_2d(sm + L::Dt, &tm_dt, 0, rowD, bar_ld);
+        tma_load_2d(sm + L::dDt, &tm_ddt, 0, rowD, bar_ld);
+        tma_load_2d(sm + L::St, &tm_sc, 0, rowD, bar_ld);
+        tma_load_2d(sm + L::St + kTile, &tm_sc, 64, rowD, bar_ld);
+        tma_load_2d(sm + L::dSt, &tm_dsc, 0, rowD, bar_ld);
+        tma_load_2d(sm + L::dSt + kTile, &tm_dsc, 64, rowD, bar_ld);
+        bulk_load(Gs, a.G + (size_t)bh * TP + t0, 256, bar_ld);
+    }
+    if (warp == 0) tmem_alloc(s_tmem, 512);
+    if (tid < 64) Bs[tid] = (tid < Lr) ? a.beta[tok_index(a, b, t0 + tid, h)] : 0.f;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t l16 = 16u << 16;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    const uint32_t c0 = tmem, c64 = tmem + 64, c128 = tmem + 128, c256 = tmem + 256;
+
+    bool ld_pending = false, mma_pending = false;
+    uint32_t mph = 0;
+    auto mma_wait = [&]() {  // thread 0
+        mma_commit(bar_mma);
+        if (!mbar_wait(bar_mma, mph)) {
+            *s_abort = 1;
+            mma_pending = true;
+            atomicExch(a.err, kErrTimeoutMma);
+        }
+    };
+    float lastpart = 0.f;
+
+    // ---------------- phase A: every product of loaded operands
+    if (tid == 0) {
+        if (!mbar_wait(bar_ld, 0)) {
+            *s_abort = 1;
+            ld_pending = true;
+            atomicExch(a.err, kErrTimeoutTma);
+        } else {
+            tc_fence_after();
+            const uint32_t q = smem_u32(sm + L::Q), k = smem_u32(sm + L::K), dob = smem_u32(sm + L::dO);
+            const uint32_t dt = smem_u32(sm + L::Dt), ddt = smem_u32(sm + L::dDt), tb = smem_u32(sm + L::Tb);
+            const uint32_t st = smem_u32(sm + L::St), dst = smem_u32(sm + L::dSt);
+            constexpr uint32_t idKK = idesc_bf16(64, 64, false, false);
+            constexpr uint32_t idKM = idesc_bf16(64, 64, false, true);
+            constexpr uint32_t idKM2 = idesc_bf16(64, 128, false, true);
+            constexpr uint32_t idMM2 = idesc_bf16(64, 128, true, true);
+            constexpr uint32_t idMK2 = idesc_bf16(64, 128, true, false);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
+                const uint32_t m = ks * 2048;
+                mma_bf16(c0, sdesc(q + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);             // Q K^T
+                mma_bf16(c0 + l16, sdesc(dob + o, 16, 1024), sdesc(dt + m, kHalf, 1024), idKM, ks > 0);  // dO Delta^T
+                mma_bf16(c64, sdesc(k + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);            // K K^T
+                mma_bf16(c128, sdesc(dob + o, 16, 1024), sdesc(st + m, kTile, 1024), idKM2, ks > 0);     // dO S^T
+                mma_bf16(c128 + l16, sdesc(dt + m, kHalf, 1024), sdesc(dst + m, kTile, 1024), idMM2,
+                         ks > 0);                                                                        // Delta dS'^T
+                mma_bf16(c256, sdesc(ddt + m, kHalf, 1024), sdesc(st + m, kTile, 1024), idMM2, ks > 0);  // dDelta S^T
+            }
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(c256 + l16, sdesc(tb + ks * 2048, kHalf, 1024), sdesc(ddt + ks * 32, 16, 1024),
+                         idMK2, ks > 0);  // T^T dDelta
+            mma_wait();
+        }
+    }
+    mph ^= 1;
+    __syncthreads();
+    if (*s_abort) goto teardown;
+    tc_fence_after();
+    {
+        const float Gr = Gs[r];
+        float rowpart;
+        // (a) P, dP, F on columns [32 ch, 32 ch + 32); each lane of a pair finishes 16
+        {
+            float v[32];
+            tmem_ld32(c0 + lane_base + ch * 32, v);
+            tmem_ld_wait();
+            float other[32];
+#pragma unroll
+            for (int q = 0; q < 32; ++q) other[q] = __shfl_xor_sync(0xffffffffu, v[q], 16);
+            const int o = hi ? 16 : 0;
+            float rowsum = 0.f;
+            float f[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const float qk = hi ? other[o + q] : v[o + q];
+                const float dp = hi ? v[o + q] : other[o + q];
+                const int t = ch * 32 + o + q;
+                const float gam = (t <= r) ? __expf(Gr - Gs[t]) : 0.f;
+                const float pd = gam * qk * dp;
+                rowsum += pd;
+                PD[r * 65 + t] = pd;
+                f[q] = gam * dp;
+            }
+            put_row(sm + L::F, r, ch * 4 + (o >> 3), f, 16);
+            rowpart = rowsum + __shfl_xor_sync(0xffffffffu, rowsum, 16);
+        }
+        // (b) dO S^T (lanes 0-15) / Delta dS'^T (lanes 16-31), columns [64 ch, 64 ch + 64)
+        {
+            float x[64];
+            tmem_ld32(c128 + lane_base + ch * 64, *(float(*)[32]) & x[0]);
+            tmem_ld32(c128 + lane_base + ch * 64 + 32, *(float(*)[32]) & x[32]);
+            tmem_ld_wait();
+            float scale;
+            if (!hi) {
+                scale = __expf(Gr);
+                part[(0 + ch) * 64 + r] = rowpart + scale * dot_row(sm + L::Q + ch * kHalf, r, x);
+            } else {
+                scale = __expf(Gs[kChunk - 1] - Gr);
+                const float t = scale * dot_row(sm + L::K + ch * kHalf, r, x);
+                part[(2 + ch) * 64 + r] = -t;
+                lastpart = t;
+            }
+#pragma unroll
+            for (int q = 0; q < 64; ++q) x[q] *= scale;
+            tmem_st32(c128 + lane_base + ch * 64, *(const float(*)[32]) & x[0]);
+            tmem_st32(c128 + lane_base + ch * 64 + 32, *(const float(*)[32]) & x[32]);
+        }
+        // (c) dW = -(dDelta S^T) (lanes 0-15) and dVhat (lanes 16-31)
+        {
+            float x[64];
+            tmem_ld32(c256 + lane_base + ch * 64, *(float(*)[32]) & x[0]);
+            tmem_ld32(c256 + lane_base + ch * 64 + 32, *(float(*)[32]) & x[32]);
+            tmem_ld_wait();
+            if (!hi) {
+#pragma unroll
+                for (int q = 0; q < 64; ++q) x[q] = -x[q];
+                put_row(sm + L::Dt + ch * kHalf, r, 0, x, 64);  // dW, MN-major B of T^T dW
+            } else {
+                const float br = Bs[r];
+                float vd = 0.f;
+                if (r < Lr) {
+                    const size_t ti = tok_index(a, b, t0 + r, h) * kD + ch * 64;
+                    const __nv_bfloat16* vrow = (const __nv_bfloat16*)a.v + ti;
+                    __nv_bfloat16* dvrow = (__nv_bfloat16*)a.dv_ + ti;
+#pragma unroll
+                    for (int qq = 0; qq < 8; ++qq) {
+                        const uint4 u = *(const uint4*)(vrow + qq * 8);
+                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                        uint4 ov;
+                        uint32_t* ow = &ov.x;
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) {
+                            const float2 fv = unpack_bf16(w[p]);
+                            vd += fv.x * x[qq * 8 + 2 * p] + fv.y * x[qq * 8 + 2 * p + 1];
+                            ow[p] = pack_bf16(br * x[qq * 8 + 2 * p], br * x[qq * 8 + 2 * p + 1]);
+                        }
+                        *(uint4*)(dvrow + qq * 8) = ov;
+                    }
+                }
+                part[(8 + ch) * 64 + r] = vd;
+                put_row(sm + L::dDt + ch * kHalf, r, 0, x, 64);  // dVhat, K-major A of dA
+            }
+        }
+        // (d) <S, dS'> over the two identically laid out tiles; last-row sum
+        {
+            float acc = 0.f;
+#pragma unroll
+            for (int qq = 0; qq < 8; ++qq) {
+                const int off = (qq * 256 + tid) * 16;
+                const uint4 u = *(const uint4*)(sm + L::St + off);
+                const uint4 w = *(const uint4*)(sm + L::dSt + off);
+                const uint32_t uu[4] = {u.x, u.y, u.z, u.w}, ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const float2 a2 = unpack_bf16(uu[p]), b2 = unpack_bf16(ww[p]);
+                    acc += a2.x * b2.x + a2.y * b2.y;
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                lastpart += __shfl_xor_sync(0xffffffffu, lastpart, off);
+            }
+            if (lane == 0) {
+                red[warp] = acc;
+                red[8 + warp] = lastpart;
+            }
+        }
+    }
+    tmem_st_wait();
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---------------- phase B: F K, F^T Q onto the rescaled partials; dKhat = T^T dW
+    if (tid == 0) {
+        tc_fence_after();
+        const uint32_t f = smem_u32(sm + L::F), k = smem_u32(sm + L::K), q = smem_u32(sm + L::Q);
+        const uint32_t tb = smem_u32(sm + L::Tb), dw = smem_u32(sm + L::Dt);
+        constexpr uint32_t idKM2 = idesc_bf16(64, 128, false, true);
+        constexpr uint32_t idMM2 = idesc_bf16(64, 128, true, true);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            mma_bf16(c128, sdesc(f + ks * 32, 16, 1024), sdesc(k + ks * 2048, kHalf, 1024), idKM2, 1);
+            mma_bf16(c128 + l16, sdesc(f + ks * 2048, kHalf, 1024), sdesc(q + ks * 2048, kHalf, 1024), idMM2, 1);
+            mma_bf16(c256, sdesc(tb + ks * 2048, kHalf, 1024), sdesc(dw + ks * 2048, kHalf, 1024), idMM2, ks > 0);
+        }
+        mma_wait();
+    }
+    mph ^= 1;
+    __syncthreads();
+    if (*s_abort) goto teardown;
+    tc_fence_after();
+    if (tid < 64) {  // column sums of dP .* P (PD is reused below)
+        float s = 0.f;
+        for (int i = 0; i < kChunk; ++i) s += PD[i * 65 + tid];
+        cs1[tid] = s;
+    }
+    {
+        float x[64];
+        tmem_ld32(c256 + lane_base + ch * 64, *(float(*)[32]) & x[0]);  // lanes 0-15: dKhat
+        tmem_ld32(c256 + lane_base + ch * 64 + 32, *(float(*)[32]) & x[32]);
+        tmem_ld_wait();
+        if (!hi) {
+            const float gam = __expf(Gs[r]), br = Bs[r];
+            const float kd = dot_row(sm + L::K + ch * kHalf, r, x);
+            part[(10 + ch) * 64 + r] = gam * kd;        // dbeta term
+            part[(4 + ch) * 64 + r] = br * gam * kd;    // dG term
+            put_row(sm + L::St + ch * kHalf, r, 0, x, 64);  // dKhat, K-major A of dA
+#pragma unroll
+            for (int q = 0; q < 64; ++q) x[q] *= br * gam;
+        }
+        tmem_st32(c256 + lane_base + ch * 64, *(const float(*)[32]) & x[0]);
+        tmem_st32(c256 + lane_base + ch * 64 + 32, *(const float(*)[32]) & x[32]);
+    }
+    tmem_st_wait();
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---------------- phase C: dA = dKhat W^T + dVhat U^T
+    if (tid == 0) {
+        tc_fence_after();
+        const uint32_t dk = smem_u32(sm + L::St), dvb = smem_u32(sm + L::dDt);
+        const uint32_t wt = smem_u32(sm + L::Wt), ut = smem_u32(sm + L::Ut);
+        constexpr uint32_t id = idesc_bf16(64, 64, false, true);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
+            mma_bf16(c0 + l16, sdesc(dk + o, 16, 1024), sdesc(wt + ks * 2048, kHalf, 1024), id, ks > 0);
+        }
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
+            mma_bf16(c0 + l16, sdesc(dvb + o, 16, 1024), sdesc(ut + ks * 2048, kHalf, 1024), id, 1);
+        }
+        mma_wait();
+    }
+    mph ^= 1;
+    __syncthreads();
+    if (*s_abort) goto teardown;
+    tc_fence_after();
+    {
+        float va[32], vb[32];
+        tmem_ld32(c0 + lane_base + ch * 32, va);   // lanes 16-31: dA
+        tmem_ld32(c64 + lane_base + ch * 32, vb);  // lanes 0-15: K K^T
+        tmem_ld_wait();
+        float da_raw[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) da_raw[q] = __shfl_xor_sync(0xffffffffu, va[q], 16);
+        if (!hi) {
+            const float Gr = Gs[r], br = Bs[r];
+            float sab = 0.f, sbb = 0.f;
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                const int t = ch * 32 + q;
+                const float gam = (t < r) ? __expf(Gr - Gs[t]) : 0.f;
+                const float bv = gam * vb[q];
+                const float da = (t < r) ? -da_raw[q] : 0.f;
+                sab += da * bv;
+                const float dbb = br * da * bv;
+                sbb += dbb;
+                PD[r * 65 + t] = dbb;           // dB .* B (column sums below)
+                Ef[r * 65 + t] = br * da * gam; // E = dB .* Gamma
+            }
+            part[(12 + ch) * 64 + r] = sab;
+            part[(6 + ch) * 64 + r] = sbb;
+        }
+    }
+    __syncthreads();
+    {
+        // E + E^T as a bf16 K-major tile [r][64 t] (in the F slot)
+        const int rr = tid >> 2, q0 = (tid & 3) * 2;
+        float e[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int t = q0 * 8 + i;
+            e[i] = Ef[rr * 65 + t] + Ef[t * 65 + rr];
+        }
+        put_row(sm + L::F, rr, q0, e, 16);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---------------- phase D: dKp = diag(beta gamma) dKhat + (E + E^T) K
+    if (tid == 0) {
+        tc_fence_after();
+        const uint32_t f = smem_u32(sm + L::F), k = smem_u32(sm + L::K);
+        constexpr uint32_t id = idesc_bf16(64, 128, false, true);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16(c256, sdesc(f + ks * 32, 16, 1024), sdesc(k + ks * 2048, kHalf, 1024), id, 1);
+        mma_wait();
+    }
+    mph ^= 1;
+    __syncthreads();
+    if (*s_abort) goto teardown;
+    tc_fence_after();
+
+    // ---------------- epilogue
+    if (warp == 0) {
+        float sdot = 0.f, last = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            sdot += red[w];
+            last += red[8 + w];
+        }
+        float v2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int rr = 2 * lane + e;
+            float cs2 = 0.f;
+            for (int i = 0; i < kChunk; ++i) cs2 += PD[i * 65 + rr];
+            float g = -cs1[rr] - cs2;
+#pragma unroll
+            for (int pi = 0; pi < 8; ++pi) g += part[pi * 64 + rr];
+            if (rr == kChunk - 1) g += last + __expf(Gs[kChunk - 1]) * sdot;
+            v2[e] = g;
+        }
+        float incl = v2[0] + v2[1];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_down_sync(0xffffffffu, incl, off);
+            if (lane + off < 32) incl += y;
+        }
+        if (a.g) {
+            if (2 * lane < Lr) a.dg[tok_index(a, b, t0 + 2 * lane, h)] = incl;
+            if (2 * lane + 1 < Lr) a.dg[tok_index(a, b, t0 + 2 * lane + 1, h)] = incl - v2[0];
+        }
+    } else if (warp == 1 || warp == 2) {
+        const int rr = tid - 32;
+        if (rr < Lr) {
+            float db = 0.f;
+#pragma unroll
+            for (int pi = 8; pi < 14; ++pi) db += part[pi * 64 + rr];
+            a.dbeta[tok_index(a, b, t0 + rr, h)] = db;
+        }
+    }
+    {
+        float x[64], y[64];
+        tmem_ld32(c128 + lane_base + ch * 64, *(float(*)[32]) & x[0]);  // lanes 0-15 dQ, 16-31 dK
+        tmem_ld32(c128 + lane_base + ch * 64 + 32, *(float(*)[32]) & x[32]);
+        tmem_ld32(c256 + lane_base + ch * 64, *(float(*)[32]) & y[0]);  // lanes 0-15 dKp
+        tmem_ld32(c256 + lane_base + ch * 64 + 32, *(float(*)[32]) & y[32]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 64; ++q) {
+            const float kp = __shfl_xor_sync(0xffffffffu, y[q], 16);  // lanes 16-31 get dKp
+            if (hi) x[q] += kp;
+        }
+        if (r < Lr) {
+            __nv_bfloat16* dst = (__nv_bfloat16*)(hi ? a.dk_ : a.dq) + tok_index(a, b, t0 + r, h) * kD + ch * 64;
+#pragma unroll
+            for (int qq = 0; qq < 8; ++qq) {
+                uint4 u;
+                u.x = pack_bf16(x[qq * 8 + 0], x[qq * 8 + 1]);
+                u.y = pack_bf16(x[qq * 8 + 2], x[qq * 8 + 3]);
+                u.z = pack_bf16(x[qq * 8 + 4], x[qq * 8 + 5]);
+                u.w = pack_bf16(x[qq * 8 + 6], x[qq * 8 + 7]);
+                *(uint4*)(dst + qq * 8) = u;
+            }
+        }
+    }
+
+teardown:
+    if (tid == 0) {
+        if (ld_pending) mbar_wait(bar_ld, 0);
+        if (mma_pending) mbar_wait(bar_mma, mph ^ 1);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_grad_fused_tc(const Args& a, cudaStream_t s) {
+    const int BH = a.B * a.H;
+    if (BH == 0 || a.NC == 0) return cudaSuccess;
+    const uint64_t rows = (uint64_t)BH * a.NC * kD, rowsC = (uint64_t)BH * a.NC * kChunk;
+    CUtensorMap tm_q{}, tm_k{}, tm_do{}, tm_wt{}, tm_ut{}, tm_t{}, tm_dt{}, tm_ddt{}, tm_sc{}, tm_dsc{};
+    const bool ok = tmap_tokens(&tm_q, a.q, a, kD) && tmap_tokens(&tm_k, a.k, a, kD) &&
+                    tmap_tokens(&tm_do, a.dO, a, kD) && tmap_2d(&tm_wt, a.Wt, 64, rows, 128) &&
+                    tmap_2d(&tm_ut, a.Ut, 64, rows, 128) && tmap_2d(&tm_t, a.Tm, 64, rowsC, 64) &&
+                    tmap_2d(&tm_dt, a.Dt, 64, rows, 128) && tmap_2d(&tm_ddt, a.dDt, 64, rows, 128) &&
+                    tmap_2d(&tm_sc, a.Sc, kD, rows, 128) && tmap_2d(&tm_dsc, a.dSc, kD, rows, 128);
+    if (!ok) return cudaErrorInvalidValue;
+    const size_t smem = FusedSmem::Size + 1024;
+    cudaError_t e = cudaFuncSetAttribute(grad_fused_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    timing_begin(KK_GRAD_FUSED, s);
+    grad_fused_tc_kernel<<<dim3(a.NC, BH), 256, smem, s>>>(tm_q, tm_k, tm_do, tm_wt, tm_ut, tm_t, tm_dt, tm_ddt,
+                                                           tm_sc, tm_dsc, a);
+    e = cudaGetLastError();
+    timing_end(KK_GRAD_FUSED, s);
+    return e;
+}
+
+}  // namespace sf

@@ -48,6 +48,8 @@ _SIGS = {
     "sf_timing_reset": (None, []),
     "sf_timing_read": (_I, [_I, ctypes.POINTER(ctypes.c_char_p), _IP,
                             ctypes.POINTER(ctypes.c_double)]),
+    "sf_timing_trace": (_I, [_I, _IP, _IP, ctypes.POINTER(ctypes.c_double),
+                             ctypes.POINTER(ctypes.c_double)]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -175,6 +177,16 @@ def sf_timing_read() -> dict:
     ms = (ctypes.c_double * cap)()
     n = _lib.sf_timing_read(cap, names, launches, ms)
     return {names[i].decode(): (launches[i], ms[i]) for i in range(n)}
+
+
+def sf_timing_trace(cap: int = 4096) -> list:
+    """[(kernel kind index, stream index, start ms, end ms)] of the recorded launches."""
+    kinds = (ctypes.c_int * cap)()
+    streams = (ctypes.c_int * cap)()
+    t0 = (ctypes.c_double * cap)()
+    t1 = (ctypes.c_double * cap)()
+    n = _lib.sf_timing_trace(cap, kinds, streams, t0, t1)
+    return [(kinds[i], streams[i], t0[i], t1[i]) for i in range(n)]
 
 
 def raw_call(name: str, *args):

@@ -101,8 +101,13 @@ size_t sf_seq_workspace_bytes(const sf_shape* shape, int n_sub, const int* lens,
  * state entering each piece, which sf_bwd_seq consumes.  The intra-chunk work
  * of piece i+1 is issued on stream_aux while the state pass of piece i runs
  * on stream_main (state overlap: StateFlow Abstract and 术语表 "状态重叠");
- * events order them.  On return all work is ordered before later work on
- * stream_main.  stream_aux may equal stream_main (no overlap). */
+ * events order them.  When the two streams differ, the state passes run on
+ * an internal stream of the device's greatest priority, forked from and
+ * joined back to stream_main by events, so that the sequential critical path
+ * is scheduled ahead of the parallel work (the first such call on a device
+ * creates that stream; make it before any stream capture).  On return all
+ * work is ordered before later work on stream_main.  stream_aux may equal
+ * stream_main (no overlap, everything on stream_main). */
 sf_status sf_fwd_seq(const sf_shape* shape, int n_sub, const int* lens, const void* q,
                      const void* k, const void* v, const float* g, const float* beta,
                      const float* S_in, void* o, float* S_out, float* S_saved, void* ws,
@@ -159,6 +164,14 @@ const char* sf_status_string(sf_status status);
 void sf_timing_enable(int on);
 void sf_timing_reset(void);
 int sf_timing_read(int cap, const char** names, int* launches, double* ms);
+
+/* Timeline of the launches recorded since the last reset or read, in launch
+ * order (profiling aid): synchronises the device, then for the first `cap`
+ * records writes the kernel kind (an index into sf_timing_read's names), the
+ * stream as a small index in order of first appearance, and the start and end
+ * in milliseconds after the start of the first record.  Records are kept (a
+ * later sf_timing_read still totals them).  Returns the number written. */
+int sf_timing_trace(int cap, int* kinds, int* streams, double* start_ms, double* end_ms);
 
 #ifdef __cplusplus
 }
