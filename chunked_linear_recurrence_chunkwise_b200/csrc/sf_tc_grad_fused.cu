@@ -25,7 +25,10 @@
 //   cols [128, 256): dQ             | dK
 //   cols [256, 384): dW, dKhat, dKp | dVhat
 // Shared memory of operands that die after the first phase is reused for the
-// later tiles and scratch (about 209 KB in all, one CTA per SM).
+// later tiles and scratch (about 218 KB in all, one CTA per SM).  Sixteen
+// warps share the element-wise work: warp w reads TMEM lane quadrant w % 4
+// and a quarter of the columns, w / 4; the operands arrive in two groups so
+// that the first products start while the state tiles are still in flight.
 
 #include <cuda.h>
 
@@ -41,6 +44,20 @@ using namespace tc;
 constexpr int kD = 128;
 constexpr int kTile = 16384;
 constexpr int kHalf = 8192;
+constexpr int kThreads = 512;
+
+// Per-row partial sums, each kept per column quarter: [term][quarter][64 rows].
+enum PartTerm {
+    P_ROWQ = 0,  // dG: rowsum(dP .* P) + gamma_r <Q_r, (dO S^T)_r>
+    P_KD,        // dG: -e^{G_C - G_r} <K_r, (Delta dS'^T)_r>
+    P_BGK,       // dG: beta_r gamma_r <K_r, dKhat_r>
+    P_SBB,       // dG: rowsum(dB .* B)
+    P_VD,        // dbeta: <V_r, dVhat_r>
+    P_GK,        // dbeta: gamma_r <K_r, dKhat_r>
+    P_SAB,       // dbeta: sum_t dA_rt B_rt
+    P_COUNT
+};
+constexpr int kDgTerms = P_VD;  // terms [0, kDgTerms) go to dG, the rest to dbeta
 
 struct FusedSmem {
     static constexpr int Q = 0;                   // [dkblk][64 r][64]
@@ -54,14 +71,14 @@ struct FusedSmem {
     static constexpr int dDt = Dt + kTile;        // dDelta^T [128 j][64 r]; later dVhat (bf16)
     static constexpr int St = dDt + kTile;        // S^T [2][128 j][64 i]; later dKhat (bf16)
     static constexpr int dSt = St + 2 * kTile;    // dS'^T [2][128 j][64 i]; later E (fp32 [64][65])
-    static constexpr int PD = dSt + 2 * kTile;    // fp32 [64][65]: dP .* P, later dB .* B
+    static constexpr int PD = dSt + 2 * kTile;    // fp32 [64][65]: dP .* P, then + dB .* B
     static constexpr int Gs = PD + 64 * 65 * 4;   // 64 fp32
     static constexpr int Bs = Gs + 256;           // 64 fp32
-    static constexpr int cs1 = Bs + 256;          // 64 fp32: column sums of dP .* P
-    static constexpr int part = cs1 + 256;        // fp32 [14][64] per-row partial sums
-    static constexpr int red = part + 14 * 256;   // fp32 [16]: per-warp <S, dS'> and last-row sums
-    static constexpr int Bar = red + 64;
-    static constexpr int Misc = Bar + 16;
+    static constexpr int csp = Bs + 256;          // fp32 [8][64]: column sums of PD over 8-row groups
+    static constexpr int part = csp + 8 * 256;    // fp32 [P_COUNT][4][64]
+    static constexpr int red = part + P_COUNT * 4 * 256;  // fp32 [32]: per-warp <S, dS'>, last-row sums
+    static constexpr int Bar = red + 128;         // 3 mbarriers
+    static constexpr int Misc = Bar + 24;
     static constexpr int Size = Misc + 16;
 };
 
@@ -69,12 +86,12 @@ __device__ __forceinline__ size_t tok_index(const Args& a, int b, int t, int h) 
     return ((size_t)b * a.ld_t + t) * a.H + h;
 }
 
-// <row r of a 128-byte-swizzled bf16 tile block, x[0..63]>
-__device__ __forceinline__ float dot_row(const uint8_t* blk, int r, const float* x) {
+// <row r, 16-byte chunks q0 .. q0 + 3 of a 128-byte-swizzled bf16 tile block, x[0..31]>
+__device__ __forceinline__ float dot_row32(const uint8_t* blk, int r, int q0, const float* x) {
     float acc = 0.f;
 #pragma unroll
-    for (int qc = 0; qc < 8; ++qc) {
-        const uint4 u = *(const uint4*)(blk + sw128(r, qc));
+    for (int qc = 0; qc < 4; ++qc) {
+        const uint4 u = *(const uint4*)(blk + sw128(r, q0 + qc));
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
@@ -98,7 +115,7 @@ __device__ __forceinline__ void put_row(uint8_t* tile, int row, int q0, const fl
     }
 }
 
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     grad_fused_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_wt,
                          const __grid_constant__ CUtensorMap tm_ut, const __grid_constant__ CUtensorMap tm_t,
@@ -110,13 +127,14 @@ __global__ void __launch_bounds__(256, 1)
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     float* Gs = (float*)(sm + L::Gs);
     float* Bs = (float*)(sm + L::Bs);
-    float* cs1 = (float*)(sm + L::cs1);
+    float* csp = (float*)(sm + L::csp);
     float* PD = (float*)(sm + L::PD);
     float* Ef = (float*)(sm + L::dSt);
     float* part = (float*)(sm + L::part);
     float* red = (float*)(sm + L::red);
-    uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);
-    uint64_t* bar_mma = bar_ld + 1;
+    uint64_t* bar_ld0 = (uint64_t*)(sm + L::Bar);
+    uint64_t* bar_ld1 = bar_ld0 + 1;
+    uint64_t* bar_mma = bar_ld0 + 2;
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
     volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
 
@@ -124,36 +142,48 @@ __global__ void __launch_bounds__(256, 1)
     const int NC = a.NC, TP = NC * kChunk;
     const int t0 = c * kChunk, Lr = min(kChunk, a.T - t0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, ch = warp >> 2;  // TMEM lane quadrant, column half
+    const int quad = warp & 3, cq = warp >> 2;  // TMEM lane quadrant, column quarter
     const bool hi = lane >= 16;                 // lanes 16-31: the lane-16 tiles
     const int r = 16 * quad + (lane & 15);      // chunk row of this thread's tiles
+    auto P = [&](int term) { return part + (term * 4 + cq) * 64; };
 
     if (tid == 0) {
-        mbar_init(bar_ld, 1);
+        mbar_init(bar_ld0, 1);
+        mbar_init(bar_ld1, 1);
         mbar_init(bar_mma, 1);
         *s_abort = 0;
         fence_barrier_init();
-        mbar_expect_tx(bar_ld, 6 * kHalf + 2 * kTile + kHalf + 2 * kTile + 4 * kTile + 256);
         const int rowD = (bh * NC + c) * kD, rowC = (bh * NC + c) * kChunk;
-        tma_load_4d(sm + L::Q, &tm_q, 0, h, t0, b, bar_ld);
-        tma_load_4d(sm + L::Q + kHalf, &tm_q, 64, h, t0, b, bar_ld);
-        tma_load_4d(sm + L::K, &tm_k, 0, h, t0, b, bar_ld);
-        tma_load_4d(sm + L::K + kHalf, &tm_k, 64, h, t0, b, bar_ld);
-        tma_load_4d(sm + L::dO, &tm_do, 0, h, t0, b, bar_ld);
-        tma_load_4d(sm + L::dO + kHalf, &tm_do, 64, h, t0, b, bar_ld);
-        tma_load_2d(sm + L::Wt, &tm_wt, 0, rowD, bar_ld);
-        tma_load_2d(sm + L::Ut, &tm_ut, 0, rowD, bar_ld);
-        tma_load_2d(sm + L::Tb, &tm_t, 0, rowC, bar_ld);
-        tma_load_2d(sm + L::Dt, &tm_dt, 0, rowD, bar_ld);
-        tma_load_2d(sm + L::dDt, &tm_ddt, 0, rowD, bar_ld);
-        tma_load_2d(sm + L::St, &tm_sc, 0, rowD, bar_ld);
-        tma_load_2d(sm + L::St + kTile, &tm_sc, 64, rowD, bar_ld);
-        tma_load_2d(sm + L::dSt, &tm_dsc, 0, rowD, bar_ld);
-        tma_load_2d(sm + L::dSt + kTile, &tm_dsc, 64, rowD, bar_ld);
-        bulk_load(Gs, a.G + (size_t)bh * TP + t0, 256, bar_ld);
+        // group 0: the operands of the first products
+        mbar_expect_tx(bar_ld0, 6 * kHalf + kTile + 256);
+        tma_load_4d(sm + L::Q, &tm_q, 0, h, t0, b, bar_ld0);
+        tma_load_4d(sm + L::Q + kHalf, &tm_q, 64, h, t0, b, bar_ld0);
+        tma_load_4d(sm + L::K, &tm_k, 0, h, t0, b, bar_ld0);
+        tma_load_4d(sm + L::K + kHalf, &tm_k, 64, h, t0, b, bar_ld0);
+        tma_load_4d(sm + L::dO, &tm_do, 0, h, t0, b, bar_ld0);
+        tma_load_4d(sm + L::dO + kHalf, &tm_do, 64, h, t0, b, bar_ld0);
+        tma_load_2d(sm + L::Dt, &tm_dt, 0, rowD, bar_ld0);
+        bulk_load(Gs, a.G + (size_t)bh * TP + t0, 256, bar_ld0);
+        // group 1: the state tiles, dDelta, T, W^T, U^T
+        mbar_expect_tx(bar_ld1, 7 * kTile + kHalf);
+        tma_load_2d(sm + L::dDt, &tm_ddt, 0, rowD, bar_ld1);
+        tma_load_2d(sm + L::St, &tm_sc, 0, rowD, bar_ld1);
+        tma_load_2d(sm + L::St + kTile, &tm_sc, 64, rowD, bar_ld1);
+        tma_load_2d(sm + L::dSt, &tm_dsc, 0, rowD, bar_ld1);
+        tma_load_2d(sm + L::dSt + kTile, &tm_dsc, 64, rowD, bar_ld1);
+        tma_load_2d(sm + L::Tb, &tm_t, 0, rowC, bar_ld1);
+        tma_load_2d(sm + L::Wt, &tm_wt, 0, rowD, bar_ld1);
+        tma_load_2d(sm + L::Ut, &tm_ut, 0, rowD, bar_ld1);
     }
     if (warp == 0) tmem_alloc(s_tmem, 512);
     if (tid < 64) Bs[tid] = (tid < Lr) ? a.beta[tok_index(a, b, t0 + tid, h)] : 0.f;
+    // this thread's quarter of V's row r (lanes 16-31), read while the tiles load
+    uint4 vpre[4] = {};
+    if (hi && r < Lr) {
+        const uint4* src = (const uint4*)((const __nv_bfloat16*)a.v + tok_index(a, b, t0 + r, h) * kD + cq * 32);
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) vpre[qq] = __ldg(src + qq);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -176,38 +206,49 @@ __global__ void __launch_bounds__(256, 1)
 
     // ---------------- phase A: every product of loaded operands
     if (tid == 0) {
-        if (!mbar_wait(bar_ld, 0)) {
-            *s_abort = 1;
-            ld_pending = true;
-            atomicExch(a.err, kErrTimeoutTma);
-        } else {
+        const uint32_t q = smem_u32(sm + L::Q), k = smem_u32(sm + L::K), dob = smem_u32(sm + L::dO);
+        const uint32_t dt = smem_u32(sm + L::Dt), ddt = smem_u32(sm + L::dDt), tb = smem_u32(sm + L::Tb);
+        const uint32_t st = smem_u32(sm + L::St), dst = smem_u32(sm + L::dSt);
+        constexpr uint32_t idKK = idesc_bf16(64, 64, false, false);
+        constexpr uint32_t idKM = idesc_bf16(64, 64, false, true);
+        constexpr uint32_t idKM2 = idesc_bf16(64, 128, false, true);
+        constexpr uint32_t idMM2 = idesc_bf16(64, 128, true, true);
+        constexpr uint32_t idMK2 = idesc_bf16(64, 128, true, false);
+        bool ok = mbar_wait(bar_ld0, 0);
+        if (ok) {
             tc_fence_after();
-            const uint32_t q = smem_u32(sm + L::Q), k = smem_u32(sm + L::K), dob = smem_u32(sm + L::dO);
-            const uint32_t dt = smem_u32(sm + L::Dt), ddt = smem_u32(sm + L::dDt), tb = smem_u32(sm + L::Tb);
-            const uint32_t st = smem_u32(sm + L::St), dst = smem_u32(sm + L::dSt);
-            constexpr uint32_t idKK = idesc_bf16(64, 64, false, false);
-            constexpr uint32_t idKM = idesc_bf16(64, 64, false, true);
-            constexpr uint32_t idKM2 = idesc_bf16(64, 128, false, true);
-            constexpr uint32_t idMM2 = idesc_bf16(64, 128, true, true);
-            constexpr uint32_t idMK2 = idesc_bf16(64, 128, true, false);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
+                mma_bf16(c0, sdesc(q + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);  // Q K^T
+                mma_bf16(c0 + l16, sdesc(dob + o, 16, 1024), sdesc(dt + ks * 2048, kHalf, 1024), idKM,
+                         ks > 0);                                                             // dO Delta^T
+                mma_bf16(c64, sdesc(k + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);  // K K^T
+            }
+            ok = mbar_wait(bar_ld1, 0);
+        }
+        if (ok) {
+            tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
                 const uint32_t m = ks * 2048;
-                mma_bf16(c0, sdesc(q + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);             // Q K^T
-                mma_bf16(c0 + l16, sdesc(dob + o, 16, 1024), sdesc(dt + m, kHalf, 1024), idKM, ks > 0);  // dO Delta^T
-                mma_bf16(c64, sdesc(k + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);            // K K^T
-                mma_bf16(c128, sdesc(dob + o, 16, 1024), sdesc(st + m, kTile, 1024), idKM2, ks > 0);     // dO S^T
+                mma_bf16(c128, sdesc(dob + o, 16, 1024), sdesc(st + m, kTile, 1024), idKM2, ks > 0);  // dO S^T
                 mma_bf16(c128 + l16, sdesc(dt + m, kHalf, 1024), sdesc(dst + m, kTile, 1024), idMM2,
-                         ks > 0);                                                                        // Delta dS'^T
-                mma_bf16(c256, sdesc(ddt + m, kHalf, 1024), sdesc(st + m, kTile, 1024), idMM2, ks > 0);  // dDelta S^T
+                         ks > 0);                                                              // Delta dS'^T
+                mma_bf16(c256, sdesc(ddt + m, kHalf, 1024), sdesc(st + m, kTile, 1024), idMM2,
+                         ks > 0);                                                              // dDelta S^T
             }
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(c256 + l16, sdesc(tb + ks * 2048, kHalf, 1024), sdesc(ddt + ks * 32, 16, 1024),
                          idMK2, ks > 0);  // T^T dDelta
-            mma_wait();
+        } else {
+            *s_abort = 1;
+            ld_pending = true;
+            atomicExch(a.err, kErrTimeoutTma);
         }
+        mma_wait();  // also drains the products issued before a load gave up
     }
     mph ^= 1;
     __syncthreads();
@@ -216,94 +257,90 @@ __global__ void __launch_bounds__(256, 1)
     {
         const float Gr = Gs[r];
         float rowpart;
-        // (a) P, dP, F on columns [32 ch, 32 ch + 32); each lane of a pair finishes 16
+        // (a) P, dP, F on columns [16 cq, 16 cq + 16): lane l < 16 holds (Q K^T)[r], lane
+        // l + 16 (dO Delta^T)[r]; after one exchange each finishes 8 columns (the low
+        // lane the first 8, the high lane the last 8)
         {
-            float v[32];
-            tmem_ld32(c0 + lane_base + ch * 32, v);
+            float v[16];
+            tmem_ld16(c0 + lane_base + cq * 16, v);
             tmem_ld_wait();
-            float other[32];
-#pragma unroll
-            for (int q = 0; q < 32; ++q) other[q] = __shfl_xor_sync(0xffffffffu, v[q], 16);
-            const int o = hi ? 16 : 0;
+            const int tb = 16 * cq + (hi ? 8 : 0);
             float rowsum = 0.f;
-            float f[16];
+            float f[8];
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const float qk = hi ? other[o + q] : v[o + q];
-                const float dp = hi ? v[o + q] : other[o + q];
-                const int t = ch * 32 + o + q;
+            for (int q = 0; q < 8; ++q) {
+                const float recv = __shfl_xor_sync(0xffffffffu, hi ? v[q] : v[8 + q], 16);
+                const float qk = hi ? recv : v[q];
+                const float dp = hi ? v[8 + q] : recv;
+                const int t = tb + q;
                 const float gam = (t <= r) ? __expf(Gr - Gs[t]) : 0.f;
                 const float pd = gam * qk * dp;
                 rowsum += pd;
                 PD[r * 65 + t] = pd;
                 f[q] = gam * dp;
             }
-            put_row(sm + L::F, r, ch * 4 + (o >> 3), f, 16);
+            put_row(sm + L::F, r, tb >> 3, f, 8);
             rowpart = rowsum + __shfl_xor_sync(0xffffffffu, rowsum, 16);
         }
-        // (b) dO S^T (lanes 0-15) / Delta dS'^T (lanes 16-31), columns [64 ch, 64 ch + 64)
+        // (b) dO S^T (lanes 0-15) / Delta dS'^T (lanes 16-31), columns [32 cq, 32 cq + 32),
+        // rescaled in TMEM by gamma_r / e^{G_C - G_r}
         {
-            float x[64];
-            tmem_ld32(c128 + lane_base + ch * 64, *(float(*)[32]) & x[0]);
-            tmem_ld32(c128 + lane_base + ch * 64 + 32, *(float(*)[32]) & x[32]);
+            float x[32];
+            tmem_ld32(c128 + lane_base + cq * 32, x);
             tmem_ld_wait();
+            const float dot = dot_row32(sm + (hi ? L::K : L::Q) + (cq >> 1) * kHalf, r, (cq & 1) * 4, x);
             float scale;
             if (!hi) {
                 scale = __expf(Gr);
-                part[(0 + ch) * 64 + r] = rowpart + scale * dot_row(sm + L::Q + ch * kHalf, r, x);
+                P(P_ROWQ)[r] = rowpart + scale * dot;
             } else {
                 scale = __expf(Gs[kChunk - 1] - Gr);
-                const float t = scale * dot_row(sm + L::K + ch * kHalf, r, x);
-                part[(2 + ch) * 64 + r] = -t;
-                lastpart = t;
+                lastpart = scale * dot;
+                P(P_KD)[r] = -lastpart;
             }
 #pragma unroll
-            for (int q = 0; q < 64; ++q) x[q] *= scale;
-            tmem_st32(c128 + lane_base + ch * 64, *(const float(*)[32]) & x[0]);
-            tmem_st32(c128 + lane_base + ch * 64 + 32, *(const float(*)[32]) & x[32]);
+            for (int q = 0; q < 32; ++q) x[q] *= scale;
+            tmem_st32(c128 + lane_base + cq * 32, x);
         }
         // (c) dW = -(dDelta S^T) (lanes 0-15) and dVhat (lanes 16-31)
         {
-            float x[64];
-            tmem_ld32(c256 + lane_base + ch * 64, *(float(*)[32]) & x[0]);
-            tmem_ld32(c256 + lane_base + ch * 64 + 32, *(float(*)[32]) & x[32]);
+            float x[32];
+            tmem_ld32(c256 + lane_base + cq * 32, x);
             tmem_ld_wait();
             if (!hi) {
 #pragma unroll
-                for (int q = 0; q < 64; ++q) x[q] = -x[q];
-                put_row(sm + L::Dt + ch * kHalf, r, 0, x, 64);  // dW, MN-major B of T^T dW
+                for (int q = 0; q < 32; ++q) x[q] = -x[q];
+                put_row(sm + L::Dt + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);  // MN-major B of T^T dW
             } else {
                 const float br = Bs[r];
                 float vd = 0.f;
-                if (r < Lr) {
-                    const size_t ti = tok_index(a, b, t0 + r, h) * kD + ch * 64;
-                    const __nv_bfloat16* vrow = (const __nv_bfloat16*)a.v + ti;
-                    __nv_bfloat16* dvrow = (__nv_bfloat16*)a.dv_ + ti;
+                uint4 ov[4];
 #pragma unroll
-                    for (int qq = 0; qq < 8; ++qq) {
-                        const uint4 u = *(const uint4*)(vrow + qq * 8);
-                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-                        uint4 ov;
-                        uint32_t* ow = &ov.x;
+                for (int qq = 0; qq < 4; ++qq) {
+                    const uint32_t w[4] = {vpre[qq].x, vpre[qq].y, vpre[qq].z, vpre[qq].w};
+                    uint32_t* ow = &ov[qq].x;
 #pragma unroll
-                        for (int p = 0; p < 4; ++p) {
-                            const float2 fv = unpack_bf16(w[p]);
-                            vd += fv.x * x[qq * 8 + 2 * p] + fv.y * x[qq * 8 + 2 * p + 1];
-                            ow[p] = pack_bf16(br * x[qq * 8 + 2 * p], br * x[qq * 8 + 2 * p + 1]);
-                        }
-                        *(uint4*)(dvrow + qq * 8) = ov;
+                    for (int p = 0; p < 4; ++p) {
+                        const float2 fv = unpack_bf16(w[p]);
+                        vd += fv.x * x[qq * 8 + 2 * p] + fv.y * x[qq * 8 + 2 * p + 1];
+                        ow[p] = pack_bf16(br * x[qq * 8 + 2 * p], br * x[qq * 8 + 2 * p + 1]);
                     }
                 }
-                part[(8 + ch) * 64 + r] = vd;
-                put_row(sm + L::dDt + ch * kHalf, r, 0, x, 64);  // dVhat, K-major A of dA
+                if (r < Lr) {
+                    uint4* dst = (uint4*)((__nv_bfloat16*)a.dv_ + tok_index(a, b, t0 + r, h) * kD + cq * 32);
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) dst[qq] = ov[qq];
+                }
+                P(P_VD)[r] = vd;
+                put_row(sm + L::dDt + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);  // K-major A of dA
             }
         }
         // (d) <S, dS'> over the two identically laid out tiles; last-row sum
         {
             float acc = 0.f;
 #pragma unroll
-            for (int qq = 0; qq < 8; ++qq) {
-                const int off = (qq * 256 + tid) * 16;
+            for (int qq = 0; qq < 4; ++qq) {
+                const int off = (qq * kThreads + tid) * 16;
                 const uint4 u = *(const uint4*)(sm + L::St + off);
                 const uint4 w = *(const uint4*)(sm + L::dSt + off);
                 const uint32_t uu[4] = {u.x, u.y, u.z, u.w}, ww[4] = {w.x, w.y, w.z, w.w};
@@ -320,7 +357,7 @@ __global__ void __launch_bounds__(256, 1)
             }
             if (lane == 0) {
                 red[warp] = acc;
-                red[8 + warp] = lastpart;
+                red[16 + warp] = lastpart;
             }
         }
     }
@@ -338,9 +375,9 @@ __global__ void __launch_bounds__(256, 1)
         constexpr uint32_t idMM2 = idesc_bf16(64, 128, true, true);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
+            mma_bf16(c256, sdesc(tb + ks * 2048, kHalf, 1024), sdesc(dw + ks * 2048, kHalf, 1024), idMM2, ks > 0);
             mma_bf16(c128, sdesc(f + ks * 32, 16, 1024), sdesc(k + ks * 2048, kHalf, 1024), idKM2, 1);
             mma_bf16(c128 + l16, sdesc(f + ks * 2048, kHalf, 1024), sdesc(q + ks * 2048, kHalf, 1024), idMM2, 1);
-            mma_bf16(c256, sdesc(tb + ks * 2048, kHalf, 1024), sdesc(dw + ks * 2048, kHalf, 1024), idMM2, ks > 0);
         }
         mma_wait();
     }
@@ -348,27 +385,20 @@ __global__ void __launch_bounds__(256, 1)
     __syncthreads();
     if (*s_abort) goto teardown;
     tc_fence_after();
-    if (tid < 64) {  // column sums of dP .* P (PD is reused below)
-        float s = 0.f;
-        for (int i = 0; i < kChunk; ++i) s += PD[i * 65 + tid];
-        cs1[tid] = s;
-    }
     {
-        float x[64];
-        tmem_ld32(c256 + lane_base + ch * 64, *(float(*)[32]) & x[0]);  // lanes 0-15: dKhat
-        tmem_ld32(c256 + lane_base + ch * 64 + 32, *(float(*)[32]) & x[32]);
+        float x[32];
+        tmem_ld32(c256 + lane_base + cq * 32, x);  // lanes 0-15: dKhat
         tmem_ld_wait();
         if (!hi) {
             const float gam = __expf(Gs[r]), br = Bs[r];
-            const float kd = dot_row(sm + L::K + ch * kHalf, r, x);
-            part[(10 + ch) * 64 + r] = gam * kd;        // dbeta term
-            part[(4 + ch) * 64 + r] = br * gam * kd;    // dG term
-            put_row(sm + L::St + ch * kHalf, r, 0, x, 64);  // dKhat, K-major A of dA
+            const float kd = dot_row32(sm + L::K + (cq >> 1) * kHalf, r, (cq & 1) * 4, x);
+            P(P_GK)[r] = gam * kd;
+            P(P_BGK)[r] = br * gam * kd;
+            put_row(sm + L::St + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);  // K-major A of dA
 #pragma unroll
-            for (int q = 0; q < 64; ++q) x[q] *= br * gam;
+            for (int q = 0; q < 32; ++q) x[q] *= br * gam;
         }
-        tmem_st32(c256 + lane_base + ch * 64, *(const float(*)[32]) & x[0]);
-        tmem_st32(c256 + lane_base + ch * 64 + 32, *(const float(*)[32]) & x[32]);
+        tmem_st32(c256 + lane_base + cq * 32, x);
     }
     tmem_st_wait();
     fence_async_smem();
@@ -398,43 +428,55 @@ __global__ void __launch_bounds__(256, 1)
     if (*s_abort) goto teardown;
     tc_fence_after();
     {
-        float va[32], vb[32];
-        tmem_ld32(c0 + lane_base + ch * 32, va);   // lanes 16-31: dA
-        tmem_ld32(c64 + lane_base + ch * 32, vb);  // lanes 0-15: K K^T
+        // B, dA, dB .* B (added onto PD), E on columns [16 cq, 16 cq + 16): lane l < 16
+        // holds (K K^T)[r], lane l + 16 dA[r]; each finishes 8 columns as in (a)
+        float va[16], vb[16];
+        tmem_ld16(c0 + lane_base + cq * 16, va);   // lanes 16-31: dA (before the sign)
+        tmem_ld16(c64 + lane_base + cq * 16, vb);  // lanes 0-15: K K^T
         tmem_ld_wait();
-        float da_raw[32];
+        const int tb = 16 * cq + (hi ? 8 : 0);
+        const float Gr = Gs[r], br = Bs[r];
+        float sab = 0.f, sbb = 0.f;
 #pragma unroll
-        for (int q = 0; q < 32; ++q) da_raw[q] = __shfl_xor_sync(0xffffffffu, va[q], 16);
+        for (int q = 0; q < 8; ++q) {
+            const float recv = __shfl_xor_sync(0xffffffffu, hi ? va[q] : vb[8 + q], 16);
+            const float kk = hi ? recv : vb[q];
+            const float dar = hi ? va[8 + q] : recv;
+            const int t = tb + q;
+            const bool lower = t < r;
+            const float gam = lower ? __expf(Gr - Gs[t]) : 0.f;
+            const float bv = gam * kk;
+            const float da = lower ? -dar : 0.f;
+            sab += da * bv;
+            const float dbb = br * da * bv;
+            sbb += dbb;
+            PD[r * 65 + t] += dbb;  // the same thread wrote dP .* P here in (a)
+            Ef[r * 65 + t] = br * da * gam;
+        }
+        sab += __shfl_xor_sync(0xffffffffu, sab, 16);
+        sbb += __shfl_xor_sync(0xffffffffu, sbb, 16);
         if (!hi) {
-            const float Gr = Gs[r], br = Bs[r];
-            float sab = 0.f, sbb = 0.f;
-#pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const int t = ch * 32 + q;
-                const float gam = (t < r) ? __expf(Gr - Gs[t]) : 0.f;
-                const float bv = gam * vb[q];
-                const float da = (t < r) ? -da_raw[q] : 0.f;
-                sab += da * bv;
-                const float dbb = br * da * bv;
-                sbb += dbb;
-                PD[r * 65 + t] = dbb;           // dB .* B (column sums below)
-                Ef[r * 65 + t] = br * da * gam; // E = dB .* Gamma
-            }
-            part[(12 + ch) * 64 + r] = sab;
-            part[(6 + ch) * 64 + r] = sbb;
+            P(P_SAB)[r] = sab;
+            P(P_SBB)[r] = sbb;
         }
     }
     __syncthreads();
     {
-        // E + E^T as a bf16 K-major tile [r][64 t] (in the F slot)
-        const int rr = tid >> 2, q0 = (tid & 3) * 2;
-        float e[16];
+        // E + E^T as a bf16 K-major tile [r][64 t] (in the F slot), and the column
+        // sums of PD = dP .* P + dB .* B over 8-row groups
+        const int rr = tid >> 3, cc = tid & 7;
+        float e[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int t = q0 * 8 + i;
+        for (int i = 0; i < 8; ++i) {
+            const int t = cc * 8 + i;
             e[i] = Ef[rr * 65 + t] + Ef[t * 65 + rr];
         }
-        put_row(sm + L::F, rr, q0, e, 16);
+        put_row(sm + L::F, rr, cc, e, 8);
+        const int col = tid & 63, g = tid >> 6;
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s += PD[(8 * g + i) * 65 + col];
+        csp[g * 64 + col] = s;
     }
     fence_async_smem();
     tc_fence_before();
@@ -456,22 +498,22 @@ __global__ void __launch_bounds__(256, 1)
     tc_fence_after();
 
     // ---------------- epilogue
-    if (warp == 0) {
+    if (warp == 0) {  // dG and dg = reverse in-chunk cumsum
         float sdot = 0.f, last = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {
+        for (int w = 0; w < 16; ++w) {
             sdot += red[w];
-            last += red[8 + w];
+            last += red[16 + w];
         }
         float v2[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int rr = 2 * lane + e;
-            float cs2 = 0.f;
-            for (int i = 0; i < kChunk; ++i) cs2 += PD[i * 65 + rr];
-            float g = -cs1[rr] - cs2;
+            float g = 0.f;
 #pragma unroll
-            for (int pi = 0; pi < 8; ++pi) g += part[pi * 64 + rr];
+            for (int i = 0; i < 8; ++i) g -= csp[i * 64 + rr];
+#pragma unroll
+            for (int pi = 0; pi < kDgTerms * 4; ++pi) g += part[pi * 64 + rr];
             if (rr == kChunk - 1) g += last + __expf(Gs[kChunk - 1]) * sdot;
             v2[e] = g;
         }
@@ -485,44 +527,46 @@ __global__ void __launch_bounds__(256, 1)
             if (2 * lane < Lr) a.dg[tok_index(a, b, t0 + 2 * lane, h)] = incl;
             if (2 * lane + 1 < Lr) a.dg[tok_index(a, b, t0 + 2 * lane + 1, h)] = incl - v2[0];
         }
-    } else if (warp == 1 || warp == 2) {
+    } else if (warp == 1 || warp == 2) {  // dbeta
         const int rr = tid - 32;
         if (rr < Lr) {
             float db = 0.f;
 #pragma unroll
-            for (int pi = 8; pi < 14; ++pi) db += part[pi * 64 + rr];
+            for (int pi = kDgTerms * 4; pi < P_COUNT * 4; ++pi) db += part[pi * 64 + rr];
             a.dbeta[tok_index(a, b, t0 + rr, h)] = db;
         }
     }
     {
-        float x[64], y[64];
-        tmem_ld32(c128 + lane_base + ch * 64, *(float(*)[32]) & x[0]);  // lanes 0-15 dQ, 16-31 dK
-        tmem_ld32(c128 + lane_base + ch * 64 + 32, *(float(*)[32]) & x[32]);
-        tmem_ld32(c256 + lane_base + ch * 64, *(float(*)[32]) & y[0]);  // lanes 0-15 dKp
-        tmem_ld32(c256 + lane_base + ch * 64 + 32, *(float(*)[32]) & y[32]);
+        // dq (lanes 0-15) and dk = dK + dKp (lanes 16-31), columns [32 cq, 32 cq + 32)
+        float x[32], y[32];
+        tmem_ld32(c128 + lane_base + cq * 32, x);
+        tmem_ld32(c256 + lane_base + cq * 32, y);  // lanes 0-15: dKp
         tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < 64; ++q) {
-            const float kp = __shfl_xor_sync(0xffffffffu, y[q], 16);  // lanes 16-31 get dKp
+        for (int q = 0; q < 32; ++q) {
+            const float kp = __shfl_xor_sync(0xffffffffu, y[q], 16);
             if (hi) x[q] += kp;
         }
         if (r < Lr) {
-            __nv_bfloat16* dst = (__nv_bfloat16*)(hi ? a.dk_ : a.dq) + tok_index(a, b, t0 + r, h) * kD + ch * 64;
+            uint4* dst = (uint4*)((__nv_bfloat16*)(hi ? a.dk_ : a.dq) + tok_index(a, b, t0 + r, h) * kD + cq * 32);
 #pragma unroll
-            for (int qq = 0; qq < 8; ++qq) {
+            for (int qq = 0; qq < 4; ++qq) {
                 uint4 u;
                 u.x = pack_bf16(x[qq * 8 + 0], x[qq * 8 + 1]);
                 u.y = pack_bf16(x[qq * 8 + 2], x[qq * 8 + 3]);
                 u.z = pack_bf16(x[qq * 8 + 4], x[qq * 8 + 5]);
                 u.w = pack_bf16(x[qq * 8 + 6], x[qq * 8 + 7]);
-                *(uint4*)(dst + qq * 8) = u;
+                dst[qq] = u;
             }
         }
     }
 
 teardown:
     if (tid == 0) {
-        if (ld_pending) mbar_wait(bar_ld, 0);
+        if (ld_pending) {
+            mbar_wait(bar_ld0, 0);
+            mbar_wait(bar_ld1, 0);
+        }
         if (mma_pending) mbar_wait(bar_mma, mph ^ 1);
     }
     tc_fence_before();
@@ -551,8 +595,8 @@ cudaError_t launch_grad_fused_tc(const Args& a, cudaStream_t s) {
                                          (int)smem);
     if (e != cudaSuccess) return e;
     timing_begin(KK_GRAD_FUSED, s);
-    grad_fused_tc_kernel<<<dim3(a.NC, BH), 256, smem, s>>>(tm_q, tm_k, tm_do, tm_wt, tm_ut, tm_t, tm_dt, tm_ddt,
-                                                           tm_sc, tm_dsc, a);
+    grad_fused_tc_kernel<<<dim3(a.NC, BH), kThreads, smem, s>>>(tm_q, tm_k, tm_do, tm_wt, tm_ut, tm_t, tm_dt,
+                                                                tm_ddt, tm_sc, tm_dsc, a);
     e = cudaGetLastError();
     timing_end(KK_GRAD_FUSED, s);
     return e;
