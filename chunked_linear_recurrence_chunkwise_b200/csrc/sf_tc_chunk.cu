@@ -1,11 +1,13 @@
 // Tensor-core per-chunk kernels (sm_100a; bf16 operands, fp32 accumulate):
 // the intra-chunk kernel and the output kernel.  Both are fully parallel over
-// (chunk, batch, head); one CTA of 4 warps per chunk-head, two CTAs per SM.
+// (chunk, batch, head), one CTA per chunk-head (8 warps for the intra kernel,
+// 4 for the output kernel), several CTAs per SM.
 //
 // Intra-chunk kernel ("a linear-recurrence kernel inside each block", the
 // StateFlow summary on gptget.net, section 方法详解), per chunk:
 //   B  = (K K^T) .* Gamma (strictly lower)        UMMA, fp32 in TMEM
-//   A  = diag(beta) B,   T = (I + A)^-1           fp32, blocked 16x16 inverse
+//   A  = diag(beta) B,   T = (I + A)^-1           16x16 diagonal blocks by fp32
+//                                                 substitution, the rest by UMMAs
 //   W^T = (diag(beta gamma) K)^T T^T              UMMA (A operand MN-major)
 //   U^T = (diag(beta) V)^T T^T                    UMMA
 // For the backward recompute the same CTA stacks [Q; K] into one M = 128
@@ -34,91 +36,6 @@ __device__ __forceinline__ size_t tok_index(const Args& a, int b, int t, int h) 
     return ((size_t)b * a.ld_t + t) * a.H + h;
 }
 
-// T = (I + A)^-1 for a 64 x 64 strictly lower A (fp32, row stride 65), by
-// inverting the four 16 x 16 diagonal blocks with substitution and filling the
-// off-diagonal blocks by distance: T_ij = -T_ii sum_{i>k>=j} A_ik T_kj.
-// T is written with row stride 68 (16-byte aligned rows).  Each thread of the
-// off-diagonal phases computes a strip of 4 adjacent columns of one row, so
-// its four multiply-add chains are independent.  Called by all 128 threads of
-// the CTA; ends with a barrier.
-constexpr int kTS = 68;  // row stride of T in floats (16-byte aligned rows)
-constexpr int kMS = 20;  // row stride of the 16 x 16 scratch blocks (16-byte aligned)
-constexpr int kMB = 16 * kMS;
-__device__ void tri_inverse64(const float* Af, float* Tf, float* Mb, int tid) {
-    for (int e = tid; e < 64 * kTS; e += 128) Tf[e] = 0.f;
-    __syncthreads();
-    if (tid < 64) {
-        // column `col` of the inverse of diagonal block `o`: right-looking substitution
-        const int o = (tid >> 4) * 16, col = tid & 15;
-        float v[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) v[r] = (r == col) ? 1.f : 0.f;
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            const float x = (r < col) ? 0.f : v[r];
-            v[r] = x;
-#pragma unroll
-            for (int r2 = r + 1; r2 < 16; ++r2) v[r2] -= Af[(o + r2) * 65 + o + r] * x;
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) Tf[(o + r) * kTS + o + col] = v[r];
-    }
-    __syncthreads();
-    for (int d = 1; d < 4; ++d) {
-        const int nstrip = (4 - d) * 64;  // blocks (bi, bj) = (m + d, m), 16 rows x 4 strips
-        for (int e = tid; e < nstrip; e += 128) {
-            const int m = e >> 6, rr = (e >> 2) & 15, c4 = (e & 3) * 4;
-            const int bi = m + d, bj = m;
-            const float* arow = Af + (16 * bi + rr) * 65;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int k = 16 * bj; k < 16 * bi; ++k) {
-                const float a = arow[k];
-                const float4 t = *(const float4*)(Tf + k * kTS + 16 * bj + c4);
-                acc.x += a * t.x;
-                acc.y += a * t.y;
-                acc.z += a * t.z;
-                acc.w += a * t.w;
-            }
-            *(float4*)(Mb + m * kMB + rr * kMS + c4) = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < nstrip; e += 128) {
-            const int m = e >> 6, rr = (e >> 2) & 15, c4 = (e & 3) * 4;
-            const int bi = m + d, bj = m;
-            const float* trow = Tf + (16 * bi + rr) * kTS + 16 * bi;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int k = 0; k <= rr; ++k) {
-                const float t = trow[k];
-                const float4 mv = *(const float4*)(Mb + m * kMB + k * kMS + c4);
-                acc.x += t * mv.x;
-                acc.y += t * mv.y;
-                acc.z += t * mv.z;
-                acc.w += t * mv.w;
-            }
-            *(float4*)(Tf + (16 * bi + rr) * kTS + 16 * bj + c4) =
-                make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-        }
-        __syncthreads();
-    }
-}
-
-// Scales the 128-byte line (64 bf16) of row `row` of a tile by f, in place.
-// Lanes of a warp handle different rows; starting each row at a different
-// 16-byte chunk keeps the warp's accesses on distinct banks.
-__device__ __forceinline__ void scale_line(uint8_t* line, int row, float f) {
-#pragma unroll
-    for (int qq = 0; qq < 8; ++qq) {
-        const int q = (qq + row) & 7;
-        uint4 u = *(uint4*)(line + q * 16);
-        uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const float2 x = unpack_bf16(w[p]);
-            w[p] = pack_bf16(x.x * f, x.y * f);
-        }
-        *(uint4*)(line + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
 
 // Writes 64 fp32 values as one bf16 row of a K-major 128-byte-swizzled tile.
 __device__ __forceinline__ void store_row64(uint8_t* tile, int row, const float* v) {
@@ -133,6 +50,26 @@ __device__ __forceinline__ void store_row64(uint8_t* tile, int row, const float*
     }
 }
 
+
+// n fp32 values as bf16 16-byte chunks q0 .. q0 + n/8 - 1 of row `row` of a
+// 128-byte-swizzled tile with 128-byte rows.
+__device__ __forceinline__ void put_row(uint8_t* tile, int row, int q0, const float* v, int n) {
+#pragma unroll
+    for (int qq = 0; qq < n / 8; ++qq) {
+        uint4 u;
+        u.x = pack_bf16(v[qq * 8 + 0], v[qq * 8 + 1]);
+        u.y = pack_bf16(v[qq * 8 + 2], v[qq * 8 + 3]);
+        u.z = pack_bf16(v[qq * 8 + 4], v[qq * 8 + 5]);
+        u.w = pack_bf16(v[qq * 8 + 6], v[qq * 8 + 7]);
+        *(uint4*)(tile + sw128(row, q0 + qq)) = u;
+    }
+}
+
+// The 64 x 64 bf16 tiles (X1, X2, X3) are row-major with 128-byte rows, so one
+// tile serves as a K-major A operand and as an MN-major B operand.
+constexpr int kIntraThreads = 256;
+constexpr int kDS = 17;  // row stride (floats) of the fp32 16 x 16 diagonal blocks
+
 template <bool kP>
 struct IntraSmem {
     static constexpr int QK = 0;                              // kP: [kblk][Q 0-63 | K 64-127][64]
@@ -140,20 +77,31 @@ struct IntraSmem {
     static constexpr int Kb = kP ? QK + kHalf : QK;           // K, d_k block 0
     static constexpr int Kblk = kP ? kTile : kHalf;           // distance between K's d_k blocks
     static constexpr int V = QK + QKBytes;                    // [dvblk][64][64]
-    static constexpr int Tb = V + kTile;                      // T, bf16 K-major [r][64 i]
-    static constexpr int Pst = Tb + kHalf;                    // P staging (kP)
-    static constexpr int Af = Pst + (kP ? kHalf : 0);         // fp32 [64][65]
-    static constexpr int Tf = Af + 64 * 65 * 4;               // fp32 [64][68]
-    static constexpr int Mb = Tf + 64 * 68 * 4;               // fp32 [3][16][20]
-    static constexpr int Gs = Mb + 3 * 320 * 4;
-    static constexpr int Bs = Gs + 256;
-    static constexpr int Bar = Bs + 256;
+    static constexpr int X1 = V + kTile;                      // A_o, then N^2, then T diag(beta gamma)
+    static constexpr int X2 = X1 + kHalf;                     // D, then E, then T diag(beta) (I without beta)
+    static constexpr int X3 = X2 + kHalf;                     // N, then T (kP)
+    static constexpr int Pst = X3 + kHalf;                    // P staging (kP)
+    static constexpr int Adf = Pst + (kP ? kHalf : 0);        // fp32 [4][16][kDS]: diagonal blocks of A
+    static constexpr int Dfp = Adf + 4 * 16 * kDS * 4;        // fp32 [4][16][kDS]: their inverses
+    static constexpr int Gs = Dfp + 4 * 16 * kDS * 4;         // G
+    static constexpr int Bs = Gs + 256;                       // beta
+    static constexpr int BGs = Bs + 256;                      // beta gamma
+    static constexpr int Bar = BGs + 256;
     static constexpr int Misc = Bar + 16;
     static constexpr int Size = Misc + 16;
 };
 
+// Intra-chunk kernel.  With A = diag(beta) (K K^T .* Gamma) strictly lower, split
+// into its 16 x 16 diagonal blocks A_d and the rest A_o:
+//   I + A = (I + A_d)(I + N),  D = (I + A_d)^-1,  N = D A_o  (strictly block-lower,
+//   N^4 = 0), so  T = (I - N + N^2 - N^3) D = E + N^2 E  with  E = D - N D.
+// D comes from substitution in fp32; N, N^2, N D and N^2 E are 64 x 64 UMMAs
+// (bf16 operands, fp32 accumulate), E is added in fp32 in TMEM.  Then
+//   W^T = K^T (T diag(beta gamma))^T,  U^T = V^T (T diag(beta))^T.
+// TMEM (128 columns): [0, 64) K K^T ([Q; K] K^T with P), then N^2 | N D, then W^T;
+// [64, 128) N, then T (lane offset 16), then U^T.
 template <bool kDelta, bool kP>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kIntraThreads)
     intra_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_wt,
                     const __grid_constant__ CUtensorMap tm_ut, const __grid_constant__ CUtensorMap tm_p,
@@ -164,9 +112,9 @@ __global__ void __launch_bounds__(128)
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     float* Gs = (float*)(sm + L::Gs);
     float* Bs = (float*)(sm + L::Bs);
-    float* Af = (float*)(sm + L::Af);
-    float* Tf = (float*)(sm + L::Tf);
-    float* Mb = (float*)(sm + L::Mb);
+    float* BGs = (float*)(sm + L::BGs);
+    float* Adf = (float*)(sm + L::Adf);
+    float* Dfp = (float*)(sm + L::Dfp);
     uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);
     uint64_t* bar_mma = bar_ld + 1;
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
@@ -176,6 +124,9 @@ __global__ void __launch_bounds__(128)
     const int NC = a.NC, TP = NC * kChunk;
     const int t0 = c * kChunk, Lr = min(kChunk, a.T - t0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, wh = warp >> 2;  // TMEM lane quadrant, column half
+    const bool hi = lane >= 16;
+    const int r = 16 * quad + (lane & 15);      // row of this thread in the M = 64 tiles
 
     if (tid == 0) {
         mbar_init(bar_ld, 1);
@@ -196,7 +147,7 @@ __global__ void __launch_bounds__(128)
         tma_load_4d(sm + L::V + kHalf, &tm_v, 64, h, t0, b, bar_ld);
     }
     if (warp == 0) {
-        tmem_alloc(s_tmem, 256);
+        tmem_alloc(s_tmem, 128);
         // in-chunk inclusive cumsum of g, two tokens per lane
         const int r0 = 2 * lane, r1 = r0 + 1;
         const float g0 = (a.g && r0 < Lr) ? a.g[tok_index(a, b, t0 + r0, h)] : 0.f;
@@ -214,29 +165,65 @@ __global__ void __launch_bounds__(128)
         // decay table of the chunk for the state passes: e^{G_C - G_r}, then e^{G_r}
         const float gC = __shfl_sync(0xffffffffu, G1, 31);
         float* ed = a.Ed + ((size_t)bh * NC + c) * 128;
+        const float e0 = __expf(G0), e1 = __expf(G1);
         ed[r0] = __expf(gC - G0);
         ed[r1] = __expf(gC - G1);
-        ed[64 + r0] = __expf(G0);
-        ed[64 + r1] = __expf(G1);
-    } else if (warp == 1) {
-        const int r0 = 2 * lane, r1 = r0 + 1;
-        if (kDelta) {
-            Bs[r0] = (r0 < Lr) ? a.beta[tok_index(a, b, t0 + r0, h)] : 0.f;
-            Bs[r1] = (r1 < Lr) ? a.beta[tok_index(a, b, t0 + r1, h)] : 0.f;
-        } else {
-            Bs[r0] = 1.f;
-            Bs[r1] = 1.f;
-        }
+        ed[64 + r0] = e0;
+        ed[64 + r1] = e1;
+        const float b0 = (kDelta && r0 < Lr) ? a.beta[tok_index(a, b, t0 + r0, h)] : 0.f;
+        const float b1 = (kDelta && r1 < Lr) ? a.beta[tok_index(a, b, t0 + r1, h)] : 0.f;
+        Bs[r0] = b0;
+        Bs[r1] = b1;
+        BGs[r0] = b0 * e0;
+        BGs[r1] = b1 * e1;
+    }
+    if (!kDelta) {  // T = I: U^T = V^T
+        const int rr = tid >> 2, q0 = (tid & 3) * 2;
+        float e[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) e[i] = (q0 * 8 + i == rr) ? 1.f : 0.f;
+        put_row(sm + L::X2, rr, q0, e, 16);
+        fence_async_smem();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    const uint32_t tD1 = tmem, tW = tmem + 64, tU = tmem + 128;
+    const uint32_t c0 = tmem, c64 = tmem + 64, l16 = 16u << 16;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     if (tid < kChunk) a.G[(size_t)bh * TP + t0 + tid] = Gs[tid];
 
     bool ld_pending = false, mma_pending = false;
     uint32_t mph = 0;
+    auto mma_wait = [&]() {  // thread 0
+        mma_commit(bar_mma);
+        if (!mbar_wait(bar_mma, mph)) {
+            *s_abort = 1;
+            mma_pending = true;
+            atomicExch(a.err, kErrTimeoutMma);
+        }
+    };
+    // A's entries of row rr, columns [g0, g0 + 16) from (K K^T) values kk: the
+    // diagonal block goes to Adf in fp32, the rest to the bf16 tile A_o (X1)
+    auto emit_A = [&](int rr, int g0, const float* kk) {
+        const float Gr = Gs[rr], br = Bs[rr];
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int t = g0 + i;
+            v[i] = (t < rr) ? br * __expf(Gr - Gs[t]) * kk[i] : 0.f;
+        }
+        if ((g0 >> 4) == (rr >> 4)) {
+            float* dst = Adf + ((rr >> 4) * 16 + (rr & 15)) * kDS;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                dst[i] = v[i];
+                v[i] = 0.f;
+            }
+        }
+        put_row(sm + L::X1, rr, g0 >> 3, v, 16);
+    };
+
     if (tid == 0 && !mbar_wait(bar_ld, 0)) {
         *s_abort = 1;
         ld_pending = true;
@@ -252,7 +239,7 @@ __global__ void __launch_bounds__(128)
                 constexpr uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_bf16(tD1, sdesc(smem_u32(sm + L::QK) + (ks >> 2) * kTile + (ks & 3) * 32, 16, 1024),
+                    mma_bf16(c0, sdesc(smem_u32(sm + L::QK) + (ks >> 2) * kTile + (ks & 3) * 32, 16, 1024),
                              sdesc(smem_u32(sm + L::Kb) + (ks >> 2) * kTile + (ks & 3) * 32, 16, 1024),
                              id, ks > 0);
             } else {
@@ -260,123 +247,227 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint64_t d = sdesc(smem_u32(sm + L::Kb) + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
-                    mma_bf16(tD1, d, d, id, ks > 0);
+                    mma_bf16(c0, d, d, id, ks > 0);
                 }
             }
-            mma_commit(bar_mma);
-            if (!mbar_wait(bar_mma, mph)) {
-                *s_abort = 1;
-                mma_pending = true;
-                atomicExch(a.err, kErrTimeoutMma);
-            }
+            mma_wait();
         }
         mph ^= 1;
         __syncthreads();
         if (*s_abort) goto teardown;
         tc_fence_after();
         {
-            float v[64];
-            tmem_ld32(taddr(tD1, 32 * warp, 0), *(float(*)[32]) & v[0]);
-            tmem_ld32(taddr(tD1, 32 * warp, 32), *(float(*)[32]) & v[32]);
+            float v[32];
+            tmem_ld32(c0 + lane_base + 32 * wh, v);
             tmem_ld_wait();
-            // accumulator row held by this thread
-            int row = -1;
-            bool is_p = false;
             if (kP) {
-                row = tid;
-                is_p = row < kChunk;
-                if (!is_p) row -= kChunk;
-            } else if (lane < 16) {
-                row = 16 * warp + lane;
-            }
-            if (row >= 0) {
-                const float Gr = Gs[row];
-                if (kP && is_p) {
-                    float p[64];
+                // [Q; K] K^T, M = 128: lane R holds row R (P rows 0-63, K K^T rows 64-127)
+                const int R = 32 * quad + lane;
+                if (R < kChunk) {
+                    const float GR = Gs[R];
+                    float p[32];
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) p[i] = (i <= row) ? __expf(Gr - Gs[i]) * v[i] : 0.f;
-                    store_row64(sm + L::Pst, row, p);
+                    for (int i = 0; i < 32; ++i) {
+                        const int t = 32 * wh + i;
+                        p[i] = (t <= R) ? __expf(GR - Gs[t]) * v[i] : 0.f;
+                    }
+                    put_row(sm + L::Pst, R, 4 * wh, p, 32);
                 } else if (kDelta) {
-                    const float br = Bs[row];
-#pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        Af[row * 65 + i] = (i < row) ? br * __expf(Gr - Gs[i]) * v[i] : 0.f;
+                    emit_A(R - kChunk, 32 * wh, v);
+                    emit_A(R - kChunk, 32 * wh + 16, v + 16);
                 }
+            } else {
+                // K K^T, M = 64: row r in lanes 0-15; lane l + 16 takes the upper 16 columns
+                float w[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float recv = __shfl_xor_sync(0xffffffffu, v[16 + i], 16);
+                    w[i] = hi ? recv : v[i];
+                }
+                emit_A(r, 32 * wh + (hi ? 16 : 0), w);
             }
         }
+        fence_async_smem();
         __syncthreads();
-    }
-    if (kDelta) tri_inverse64(Af, Tf, Mb, tid);
-    {
-        // T as a bf16 K-major tile (identity for linear attention)
-        const int r = tid >> 1, q0 = (tid & 1) * 4;
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-            const int q = q0 + qq;
-            float t[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                t[e] = kDelta ? Tf[r * kTS + q * 8 + e] : ((q * 8 + e == r) ? 1.f : 0.f);
-            uint4 u;
-            u.x = pack_bf16(t[0], t[1]);
-            u.y = pack_bf16(t[2], t[3]);
-            u.z = pack_bf16(t[4], t[5]);
-            u.w = pack_bf16(t[6], t[7]);
-            *(uint4*)(sm + L::Tb + sw128(r, q)) = u;
-        }
-        // K_hat = diag(beta gamma) K and V_hat = diag(beta) V, in place
-        const int blk = tid & 1;
-        if (kDelta) {
-            scale_line(sm + L::Kb + blk * L::Kblk + r * 128, r, Bs[r] * __expf(Gs[r]));
-            scale_line(sm + L::V + blk * kHalf + r * 128, r, Bs[r]);
-        }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-        if (kP) {
+        if (kP && tid == 0) {
             tma_store_2d(&tm_p, sm + L::Pst, 0, (bh * NC + c) * kChunk);
-            if (kDelta) tma_store_2d(&tm_t, sm + L::Tb, 0, (bh * NC + c) * kChunk);  // for the gradients
             bulk_commit();
         }
+    }
+    if (kDelta) {
+        // D = (I + A_d)^-1: thread (block, column) substitutes down one column
+        if (tid < 64) {
+            const int bk = tid >> 4, col = tid & 15;
+            const float* ab = Adf + bk * 16 * kDS;
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = (i == col) ? 1.f : 0.f;
+#pragma unroll
+            for (int j = 0; j < 15; ++j) {
+                const float x = v[j];
+#pragma unroll
+                for (int i = j + 1; i < 16; ++i) v[i] -= ab[i * kDS + j] * x;
+            }
+            float* db = Dfp + bk * 16 * kDS;
+            const int cc = 16 * bk + col;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                db[i * kDS + col] = v[i];
+                *(__nv_bfloat16*)(sm + L::X2 + sw128(16 * bk + i, cc >> 3) + (cc & 7) * 2) =
+                    __float2bfloat16_rn(v[i]);
+            }
+        } else {
+            // zeros outside the diagonal blocks of the D tile: 6 chunks per row
+            for (int k = tid - 64; k < 64 * 6; k += kIntraThreads - 64) {
+                const int row = k / 6, j = k % 6, bc = 2 * (row >> 4);
+                *(uint4*)(sm + L::X2 + sw128(row, j < bc ? j : j + 2)) = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // N = D A_o
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t x1 = smem_u32(sm + L::X1), x2 = smem_u32(sm + L::X2);
+            constexpr uint32_t id = idesc_bf16(64, 64, false, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(c64, sdesc(x2 + ks * 32, 16, 1024), sdesc(x1 + ks * 2048, kHalf, 1024), id, ks > 0);
+            mma_wait();
+        }
+        mph ^= 1;
+        __syncthreads();
+        if (*s_abort) goto teardown;
+        tc_fence_after();
+        {
+            float v[32];
+            tmem_ld32(c64 + lane_base + 32 * wh, v);
+            tmem_ld_wait();
+            float w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float recv = __shfl_xor_sync(0xffffffffu, v[16 + i], 16);
+                w[i] = hi ? recv : v[i];
+            }
+            put_row(sm + L::X3, r, 4 * wh + (hi ? 2 : 0), w, 16);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // N^2 = N N (lane offset 0) and N D (lane offset 16)
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t x2 = smem_u32(sm + L::X2), x3 = smem_u32(sm + L::X3);
+            constexpr uint32_t id = idesc_bf16(64, 64, false, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                mma_bf16(c0, sdesc(x3 + ks * 32, 16, 1024), sdesc(x3 + ks * 2048, kHalf, 1024), id, ks > 0);
+                mma_bf16(c0 + l16, sdesc(x3 + ks * 32, 16, 1024), sdesc(x2 + ks * 2048, kHalf, 1024), id,
+                         ks > 0);
+            }
+            mma_wait();
+        }
+        mph ^= 1;
+        __syncthreads();
+        if (*s_abort) goto teardown;
+        tc_fence_after();
+        {
+            // lanes 0-15: N^2 -> bf16 tile; lanes 16-31: E = D - N D -> bf16 tile and,
+            // in fp32, into T's accumulator (lane offset 16)
+            float v[32];
+            tmem_ld32(c0 + lane_base + 32 * wh, v);
+            tmem_ld_wait();
+            if (!hi) {
+                put_row(sm + L::X1, r, 4 * wh, v, 32);
+            } else {
+                const float* drow = Dfp + ((r >> 4) * 16 + (r & 15)) * kDS;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int t = 32 * wh + i;
+                    const float dv = ((t >> 4) == (r >> 4)) ? drow[t & 15] : 0.f;
+                    v[i] = dv - v[i];
+                }
+                put_row(sm + L::X2, r, 4 * wh, v, 32);
+            }
+            tmem_st32(c64 + lane_base + 32 * wh, v);
+        }
+        tmem_st_wait();
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // T = E + N^2 E
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t x1 = smem_u32(sm + L::X1), x2 = smem_u32(sm + L::X2);
+            constexpr uint32_t id = idesc_bf16(64, 64, false, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(c64 + l16, sdesc(x1 + ks * 32, 16, 1024), sdesc(x2 + ks * 2048, kHalf, 1024), id, 1);
+            mma_wait();
+        }
+        mph ^= 1;
+        __syncthreads();
+        if (*s_abort) goto teardown;
+        tc_fence_after();
+        {
+            // T rows in lanes 16-31; lane l takes the upper 16 of the 32 columns
+            float v[32];
+            tmem_ld32(c64 + lane_base + 32 * wh, v);
+            tmem_ld_wait();
+            float w[16], t1[16], t2[16];
+            const int cb = 32 * wh + (hi ? 0 : 16);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float recv = __shfl_xor_sync(0xffffffffu, v[16 + i], 16);
+                w[i] = hi ? v[i] : recv;
+                t1[i] = w[i] * BGs[cb + i];
+                t2[i] = w[i] * Bs[cb + i];
+            }
+            put_row(sm + L::X1, r, cb >> 3, t1, 16);
+            put_row(sm + L::X2, r, cb >> 3, t2, 16);
+            if (kP) put_row(sm + L::X3, r, cb >> 3, w, 16);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (kP && tid == 0) {
+            tma_store_2d(&tm_t, sm + L::X3, 0, (bh * NC + c) * kChunk);  // for the gradients
+            bulk_commit();
+        }
+    }
+    // W^T = K^T (T diag(beta gamma))^T, U^T = V^T (T diag(beta))^T; M = 128 (d rows)
+    if (tid == 0) {
         tc_fence_after();
         constexpr uint32_t id = idesc_bf16(128, 64, true, false);
-        const uint32_t tb = smem_u32(sm + L::Tb);
+        const uint32_t x1 = smem_u32(sm + L::X1), x2 = smem_u32(sm + L::X2);
         if (kDelta) {
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tW, sdesc(smem_u32(sm + L::Kb) + ks * 2048, L::Kblk, 1024),
-                         sdesc(tb + ks * 32, 16, 1024), id, ks > 0);
+                mma_bf16(c0, sdesc(smem_u32(sm + L::Kb) + ks * 2048, L::Kblk, 1024), sdesc(x1 + ks * 32, 16, 1024),
+                         id, ks > 0);
         }
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-            mma_bf16(tU, sdesc(smem_u32(sm + L::V) + ks * 2048, kHalf, 1024),
-                     sdesc(tb + ks * 32, 16, 1024), id, ks > 0);
-        mma_commit(bar_mma);
-        if (!mbar_wait(bar_mma, mph)) {
-            *s_abort = 1;
-            mma_pending = true;
-            atomicExch(a.err, kErrTimeoutMma);
-        }
+            mma_bf16(c64, sdesc(smem_u32(sm + L::V) + ks * 2048, kHalf, 1024), sdesc(x2 + ks * 32, 16, 1024), id,
+                     ks > 0);
+        mma_wait();
     }
     mph ^= 1;
     __syncthreads();
     if (*s_abort) goto teardown;
     tc_fence_after();
     {
-        const int d = tid;  // W^T / U^T row = TMEM lane
-        float v[64];
+        const int d = 32 * quad + lane;  // W^T / U^T row = TMEM lane
+        float v[32];
         if (kDelta) {
-            tmem_ld32(taddr(tW, 32 * warp, 0), *(float(*)[32]) & v[0]);
-            tmem_ld32(taddr(tW, 32 * warp, 32), *(float(*)[32]) & v[32]);
+            tmem_ld32(c0 + lane_base + 32 * wh, v);
             tmem_ld_wait();
-            store_row64(sm + L::QK, d, v);  // W^T staging (Q/K are dead)
+            put_row(sm + L::QK, d, 4 * wh, v, 32);  // W^T staging (Q/K are dead)
         }
-        tmem_ld32(taddr(tU, 32 * warp, 0), *(float(*)[32]) & v[0]);
-        tmem_ld32(taddr(tU, 32 * warp, 32), *(float(*)[32]) & v[32]);
+        tmem_ld32(c64 + lane_base + 32 * wh, v);
         tmem_ld_wait();
-        store_row64(sm + L::V, d, v);  // U^T staging (V is dead)
+        put_row(sm + L::V, d, 4 * wh, v, 32);  // U^T staging (V is dead)
     }
     fence_async_smem();
     __syncthreads();
@@ -396,7 +487,7 @@ teardown:
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 128);
     }
 }
 
@@ -582,12 +673,12 @@ cudaError_t launch_intra_tc(const Args& a, bool with_p, cudaStream_t s) {
         const size_t smem = IntraSmem<true>::Size + 1024;
         auto kern = a.beta ? intra_tc_kernel<true, true> : intra_tc_kernel<false, true>;
         e = set_smem(kern, smem);
-        if (e == cudaSuccess) kern<<<grid, 128, smem, s>>>(tm_q, tm_k, tm_v, tm_wt, tm_ut, tm_p, tm_t, a);
+        if (e == cudaSuccess) kern<<<grid, kIntraThreads, smem, s>>>(tm_q, tm_k, tm_v, tm_wt, tm_ut, tm_p, tm_t, a);
     } else {
         const size_t smem = IntraSmem<false>::Size + 1024;
         auto kern = a.beta ? intra_tc_kernel<true, false> : intra_tc_kernel<false, false>;
         e = set_smem(kern, smem);
-        if (e == cudaSuccess) kern<<<grid, 128, smem, s>>>(tm_q, tm_k, tm_v, tm_wt, tm_ut, tm_p, tm_t, a);
+        if (e == cudaSuccess) kern<<<grid, kIntraThreads, smem, s>>>(tm_q, tm_k, tm_v, tm_wt, tm_ut, tm_p, tm_t, a);
     }
     if (e == cudaSuccess) e = cudaGetLastError();
     timing_end(kind, s);
