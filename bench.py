@@ -41,6 +41,9 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="sf", choices=["sf", "reference"])
     p.add_argument("--workload", default=inputs.BENCH_WORKLOAD, choices=list(inputs.WORKLOADS))
+    p.add_argument("--mode", default="keep", choices=["keep", "recompute"],
+                   help="keep: the forward keeps its intermediates for the backward; recompute: "
+                        "the backward recomputes every piece from its stored entering state")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=16384)
@@ -115,8 +118,8 @@ def kernel_units(name: str, w) -> dict:
                           mm(C, C, d) + 2 * mm(d, C, C)),
             "intra_bwd": (3 * tile + 2 * C * f + C * f + 2 * tile + C * C * e,
                           mm(2 * C, C, d) + 2 * mm(d, C, C)),
-            # read W^T, U^T, k, G; write S^T, Delta^T
-            "state_fwd": (3 * tile + C * f + st + tile, mm(d, C, d) + mm(d, d, C)),
+            # read W^T, U^T, k, decay table; write S^T, Delta^T
+            "state_fwd": (3 * tile + 2 * C * f + st + tile, mm(d, C, d) + mm(d, d, C)),
             # read q, k, S^T, Delta^T, G; write o
             "output": (2 * tile + st + tile + C * f + tile,
                        mm(C, C, d) + mm(d, C, d) + mm(d, C, C)),
@@ -169,11 +172,9 @@ def roofline(timing: dict, w, steps: int, peaks: dict, peaks_src: str, clocks: d
         return None
     per_step = launches / steps
     chunk_heads = w.B * w.H * ((w.T + 63) // 64)  # per step, over all pieces
-    # launches of one kind per step each process one piece; their chunk-heads add up to
-    # the whole sequence once per pass (intra and the forward state pass run twice: forward
-    # and backward recompute, and are timed as separate kinds or as two launches per piece)
-    passes = 2 if (name == "state_fwd") else 1
-    units_per_launch = chunk_heads * passes / per_step
+    # every launch processes one piece (all heads, batch rows); pieces of the workload
+    # are uniform, so a launch covers chunk_heads / n_sub chunk-heads
+    units_per_launch = chunk_heads / w.n_sub
     u = kernel_units(name, w)
     per_launch_s = ms / 1e3 / launches
     gbs = u["bytes"] * units_per_launch / per_launch_s / 1e9
@@ -325,9 +326,17 @@ def run_sf(args, w, rank, world, local_rank):
     dg = None if x["g"] is None else torch.empty_like(x["g"])
     db = None if x["beta"] is None else torch.empty_like(x["beta"])
     dS_in = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+    keep = torch.empty(sf.sf_keep_bytes(sh, lens), dtype=torch.uint8, device=dev)
 
-    def step(src, serial=False):
+    def step(src, serial=False, mode=None):
         sa = main if serial else aux
+        if (mode or args.mode) == "keep":
+            sf.sf_fwd_seq_keep(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], None, o,
+                               S_out, keep, ws_f, stream_main=main, stream_aux=sa)
+            sf.sf_bwd_seq_keep(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], keep,
+                               src["dO"], None, dq, dk, dv, dg, db, dS_in, ws_b, stream_main=main,
+                               stream_aux=sa)
+            return
         sf.sf_fwd_seq(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], None, o, S_out,
                       S_saved, ws_f, stream_main=main, stream_aux=sa)
         sf.sf_bwd_seq(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], S_saved,
@@ -360,6 +369,22 @@ def run_sf(args, w, rank, world, local_rank):
     barrier()
     ms = e0.elapsed_time(e1) / args.steps
     ms_max = reduce_max(ms, device=dev)
+    sf.sf_check(ws_f, main)
+    sf.sf_check(ws_b, main)
+
+    # ---- the other driver form, timed the same way (reported beside the headline)
+    other = "recompute" if args.mode == "keep" else "keep"
+    for _ in range(args.warmup):
+        step(x, mode=other)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(main)
+    for _ in range(args.steps):
+        step(x, mode=other)
+    e1.record(main)
+    torch.cuda.synchronize()
+    barrier()
+    ms_other = reduce_max(e0.elapsed_time(e1) / args.steps, device=dev)
     sf.sf_check(ws_f, main)
     sf.sf_check(ws_b, main)
 
@@ -423,7 +448,12 @@ def run_sf(args, w, rank, world, local_rank):
             "data": "synthetic",
             "config": {"workload": w.name, "B": B, "T": T, "H": H, "d": d, "n_sub": len(lens),
                        "chunk": 64, "variant": w.variant, "l2": "inputs larger than L2, no flush",
-                       "parallelism": f"replicas{world}"},
+                       "parallelism": f"replicas{world}", "mode": args.mode,
+                       "keep_bytes": keep.numel()},
+            "modes": {args.mode: {"ms_per_step": round(ms_max, 4),
+                                  "value": round(job_tokens_per_s(world, B, T, ms_max), 1)},
+                      other: {"ms_per_step": round(ms_other, 4),
+                              "value": round(job_tokens_per_s(world, B, T, ms_other), 1)}},
             "clocks": clocks,
             "gpu_launches": launches,
             "e2e": e2e,

@@ -32,7 +32,14 @@ constexpr int kSeqSlots = 3;
 
 WsLayout ws_layout(int B, int T, int H, int dk, int dv, int dtype, bool delta, bool bwd,
                    int nslots) {
+    return ws_layout_parts(B, T, H, dk, dv, dtype, delta,
+                           bwd ? (kPartFwd | kPartPT | kPartBwd) : kPartFwd, nslots);
+}
+
+WsLayout ws_layout_parts(int B, int T, int H, int dk, int dv, int dtype, bool delta, int parts,
+                         int nslots) {
     WsLayout L{};
+    const bool fwd = parts & kPartFwd, pt = parts & kPartPT, bwd = parts & kPartBwd;
     const size_t BH = (size_t)B * H;
     const size_t NC = (size_t)(T + kChunk - 1) / kChunk;
     const size_t TP = NC * kChunk;
@@ -45,21 +52,42 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv, int dtype, bool delta, b
         off += up256(bytes);
         return o;
     };
-    L.G = take(BH * TP * 4);
-    L.Ed = take(BH * NC * 128 * 4);
-    L.Wt = take(delta ? BH * TP * dk * tw : 0);
-    L.Ut = take(BH * TP * dv * tw);
-    L.Sc = take(BH * NC * dk * dv * tw);
-    L.Dt = take(BH * TP * dv * tw);
+    L.G = take(fwd ? BH * TP * 4 : 0);
+    L.Ed = take(fwd ? BH * NC * 128 * 4 : 0);
+    L.Wt = take(fwd && delta ? BH * TP * dk * tw : 0);
+    L.Ut = take(fwd ? BH * TP * dv * tw : 0);
+    L.Sc = take(fwd ? BH * NC * dk * dv * tw : 0);
+    L.Dt = take(fwd ? BH * TP * dv * tw : 0);
     L.dDt = take(bwd ? BH * TP * dv * tw : 0);
     L.dSc = take(bwd ? BH * NC * dk * dv * tw : 0);
-    L.Pm = take(bwd ? BH * NC * kChunk * kChunk * tw : 0);
-    L.Tm = take(bwd && delta ? BH * NC * kChunk * kChunk * tw : 0);
+    L.Pm = take(pt ? BH * NC * kChunk * kChunk * tw : 0);
+    L.Tm = take(pt && delta ? BH * NC * kChunk * kChunk * tw : 0);
     L.dKp = take(bwd && delta && split_grads ? BH * TP * dk * 4 : 0);
     L.dGp = take(bwd && delta && split_grads ? BH * TP * 4 : 0);
     L.slot_bytes = off;
     L.total = kErrBytes + (size_t)nslots * L.slot_bytes;
     return L;
+}
+
+void bind_parts(Args& a, char* base, const WsLayout& L, int parts) {
+    if (parts & kPartFwd) {
+        a.G = (float*)(base + L.G);
+        a.Ed = (float*)(base + L.Ed);
+        a.Wt = base + L.Wt;
+        a.Ut = base + L.Ut;
+        a.Sc = base + L.Sc;
+        a.Dt = base + L.Dt;
+    }
+    if (parts & kPartPT) {
+        a.Pm = base + L.Pm;
+        a.Tm = base + L.Tm;
+    }
+    if (parts & kPartBwd) {
+        a.dDt = base + L.dDt;
+        a.dSc = base + L.dSc;
+        a.dKp = (float*)(base + L.dKp);
+        a.dGp = (float*)(base + L.dGp);
+    }
 }
 
 void bind_slot(Args& a, void* ws, const WsLayout& L, int slot, bool bwd) {
@@ -220,6 +248,14 @@ cudaError_t run_bwd_state(Args a, cudaStream_t st) {
     f.S_out = nullptr;
     cudaError_t e = state_fwd(f, st);
     if (e == cudaSuccess && !tc_eligible(a)) e = launch_dd_pre(a, st);
+    if (e == cudaSuccess) e = tc_eligible(a) ? launch_state_bwd_tc(a, st) : launch_state_bwd(a, st);
+    return e;
+}
+
+// The sequential part of one piece's backward when the forward kept its
+// intermediates: (on the SIMT path, the P^T dO pre-pass) then the reverse dS pass.
+cudaError_t run_bwd_state_kept(const Args& a, cudaStream_t st) {
+    cudaError_t e = tc_eligible(a) ? cudaSuccess : launch_dd_pre(a, st);
     if (e == cudaSuccess) e = tc_eligible(a) ? launch_state_bwd_tc(a, st) : launch_state_bwd(a, st);
     return e;
 }
@@ -392,10 +428,41 @@ sf_status sf_bwd(const sf_shape* s, const void* q, const void* k, const void* v,
 }
 
 
-sf_status sf_fwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* q, const void* k,
-                     const void* v, const float* g, const float* beta, const float* S_in, void* o,
-                     float* S_out, float* S_saved, void* ws, size_t ws_bytes, void* stream_main,
-                     void* stream_aux) {
+}  // extern "C"
+
+namespace {
+
+// Layout of the buffer that keeps the forward's intermediates of every piece for
+// a backward without recompute: piece i's region (the forward parts of a slot for
+// lens[i] tokens, plus P and T on the tensor-core path) follows piece i-1's.
+struct KeepPlan {
+    std::vector<size_t> off;  // byte offset of each piece's region
+    std::vector<WsLayout> lay;
+    size_t total = 0;
+};
+
+int keep_parts(const sf_shape* s) {
+    const bool tc = s->dtype == SF_BF16 && s->dk == kMaxD && s->dv == kMaxD;
+    return kPartFwd | (tc ? kPartPT : 0);
+}
+
+void plan_keep(const sf_shape* s, int n_sub, const int* lens, KeepPlan& k) {
+    k.off.resize(n_sub);
+    k.lay.resize(n_sub);
+    size_t off = 0;
+    for (int i = 0; i < n_sub; ++i) {
+        k.lay[i] = ws_layout_parts(s->B, lens[i], s->H, s->dk, s->dv, s->dtype, true, keep_parts(s), 1);
+        k.off[i] = off;
+        off += up256(k.lay[i].slot_bytes);
+    }
+    k.total = off;
+}
+
+// The forward driver; keep != NULL also stores every piece's intermediates there.
+sf_status fwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* q, const void* k,
+                  const void* v, const float* g, const float* beta, const float* S_in, void* o,
+                  float* S_out, float* S_saved, void* ws, size_t ws_bytes, void* keep,
+                  size_t keep_bytes, void* stream_main, void* stream_aux) {
     sf_status st = check_shape(s);
     if (st != SF_OK) return st;
     SeqPlan p;
@@ -406,6 +473,11 @@ sf_status sf_fwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
                             : std::initializer_list<const void*>{},
                     {q, k, v, o}, {g, beta, S_in, S_out, S_saved});
     if (st != SF_OK) return st;
+    KeepPlan kp;
+    if (keep) {
+        plan_keep(s, n_sub, lens, kp);
+        if (keep_bytes < kp.total || !aligned(keep, 256)) return SF_ERR_WORKSPACE;
+    }
     if (!work) return SF_OK;
     const size_t nstate = (size_t)s->B * s->H * s->dk * s->dv;
     const WsLayout L = ws_layout(s->B, p.lmax, s->H, s->dk, s->dv, s->dtype, beta != nullptr, false,
@@ -455,12 +527,15 @@ sf_status sf_fwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
         a.S_in = sin;
         a.S_out = sout;
         bind_slot(a, ws, L, i % kSeqSlots, false);
+        if (keep) bind_parts(a, (char*)keep + kp.off[i], kp.lay[i], keep_parts(s));
         return a;
     };
+    // with keep, the intra kernel also stores P and T (tensor-core path) for the backward
+    auto run_intra_piece = [&](const Args& a) { return intra(a, keep != nullptr, sa); };
 
     if (S_saved) SF_TRY(copy_state(S_saved, S_in, nstate, sc));
     for (int j = 0; j < std::min(2, n_sub); ++j) {
-        SF_TRY(run_intra(piece(j), sa));
+        SF_TRY(run_intra_piece(piece(j)));
         SF_TRY(cudaEventRecord(ev_intra[j % NS], sa));
     }
     for (int i = 0; i < n_sub; ++i) {
@@ -469,7 +544,7 @@ sf_status sf_fwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
         SF_TRY(run_state_output(a, sc, false));
         SF_TRY(cudaEventRecord(ev_state[i % NS], sc));
         if (i + 2 < n_sub) {  // its slot's previous piece (i-1) finished its output on this stream
-            SF_TRY(run_intra(piece(i + 2), sa));
+            SF_TRY(run_intra_piece(piece(i + 2)));
             SF_TRY(cudaEventRecord(ev_intra[(i + 2) % NS], sa));
         }
         SF_TRY(cudaStreamWaitEvent(sa, ev_state[i % NS], 0));
@@ -482,11 +557,13 @@ sf_status sf_fwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
     return SF_OK;
 }
 
-sf_status sf_bwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* q, const void* k,
-                     const void* v, const float* g, const float* beta, const float* S_saved,
-                     const void* dO, const float* dS_out, void* dq, void* dk, void* dv, float* dg,
-                     float* dbeta, float* dS_in, void* ws, size_t ws_bytes, void* stream_main,
-                     void* stream_aux) {
+// The backward driver; keep != NULL reads the forward's intermediates from there
+// (no recompute), else every piece is recomputed from S_saved.
+sf_status bwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* q, const void* k,
+                  const void* v, const float* g, const float* beta, const float* S_saved,
+                  const void* dO, const float* dS_out, void* dq, void* dk, void* dv, float* dg,
+                  float* dbeta, float* dS_in, void* ws, size_t ws_bytes, const void* keep,
+                  size_t keep_bytes, void* stream_main, void* stream_aux) {
     sf_status st = check_shape(s);
     if (st != SF_OK) return st;
     if ((g != nullptr) != (dg != nullptr) || (beta != nullptr) != (dbeta != nullptr))
@@ -495,10 +572,16 @@ sf_status sf_bwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
     st = plan_seq(s, n_sub, lens, p);
     if (st != SF_OK) return st;
     const bool work = (size_t)s->B * s->H > 0;
-    st = check_ptrs(s, work ? std::initializer_list<const void*>{q, k, v, dO, dq, dk, dv, S_saved}
+    st = check_ptrs(s, work ? (keep ? std::initializer_list<const void*>{q, k, v, dO, dq, dk, dv}
+                                    : std::initializer_list<const void*>{q, k, v, dO, dq, dk, dv, S_saved})
                             : std::initializer_list<const void*>{},
                     {q, k, v, dO, dq, dk, dv}, {g, beta, S_saved, dS_out, dg, dbeta, dS_in});
     if (st != SF_OK) return st;
+    KeepPlan kp;
+    if (keep) {
+        plan_keep(s, n_sub, lens, kp);
+        if (keep_bytes < kp.total || !aligned(keep, 256)) return SF_ERR_WORKSPACE;
+    }
     if (!work) return SF_OK;
     const size_t nstate = (size_t)s->B * s->H * s->dk * s->dv;
     const WsLayout L = ws_layout(s->B, p.lmax, s->H, s->dk, s->dv, s->dtype, beta != nullptr, true,
@@ -512,9 +595,10 @@ sf_status sf_bwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
     const int ld_t = s->ld_t ? s->ld_t : s->T;
 
     // Schedule (pieces in reverse): the critical stream carries the sequential
-    // passes of each piece (forward-state recompute, then the reverse dS pass);
-    // the aux stream runs the parallel work (intra recompute two pieces ahead,
-    // per-chunk gradients one piece behind), three workspace slots in flight.
+    // passes of each piece (forward-state recompute unless kept, then the reverse
+    // dS pass); the aux stream runs the parallel work (intra recompute two pieces
+    // ahead unless kept, per-chunk gradients one piece behind), three workspace
+    // slots in flight.
     constexpr int NS = kSeqSlots;
     EventSet evs;
     SF_TRY(evs.make(2 * NS + 3));
@@ -545,36 +629,93 @@ sf_status sf_bwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* 
         a.beta = (const float*)tok_ptr(beta, t0, s->H, 1, 4);
         a.dg = (float*)tok_ptr(dg, t0, s->H, 1, 4);
         a.dbeta = (float*)tok_ptr(dbeta, t0, s->H, 1, 4);
-        a.S_in = S_saved + (size_t)i * nstate;
+        a.S_in = S_saved ? S_saved + (size_t)i * nstate : nullptr;
         a.S_out = nullptr;
         // dS leaving piece i (from piece i+1) and dS entering it (to piece i-1)
         a.dS_out = (i == n_sub - 1) ? dS_out : pingpong + (size_t)((n_sub - 2 - i) & 1) * nstate;
         a.dS_in = (i == 0) ? dS_in : pingpong + (size_t)((n_sub - 1 - i) & 1) * nstate;
         bind_slot(a, ws, L, i % kSeqSlots, true);
+        if (keep) bind_parts(a, (char*)keep + kp.off[i], kp.lay[i], keep_parts(s));
         return a;
     };
 
-    for (int j = n_sub - 1; j >= std::max(0, n_sub - 2); --j) {
-        SF_TRY(intra(piece(j), true, sa));
-        SF_TRY(cudaEventRecord(ev_prep[j % NS], sa));
+    if (!keep) {
+        for (int j = n_sub - 1; j >= std::max(0, n_sub - 2); --j) {
+            SF_TRY(intra(piece(j), true, sa));
+            SF_TRY(cudaEventRecord(ev_prep[j % NS], sa));
+        }
     }
+    // ev_prep[slot]: without keep, the intra recompute of the slot's piece is done (it
+    // was issued on the aux stream after the gradients of the slot's previous piece);
+    // with keep, the gradients of the slot's previous piece are done.  Either way the
+    // reverse pass may then overwrite the slot's dS'^T and dDelta^T.
     for (int i = n_sub - 1; i >= 0; --i) {
         const Args a = piece(i);
-        SF_TRY(cudaStreamWaitEvent(sc, ev_prep[i % NS], 0));
-        SF_TRY(run_bwd_state(a, sc));
+        if (!keep || i + NS < n_sub) SF_TRY(cudaStreamWaitEvent(sc, ev_prep[i % NS], 0));
+        SF_TRY(keep ? run_bwd_state_kept(a, sc) : run_bwd_state(a, sc));
         SF_TRY(cudaEventRecord(ev_state[i % NS], sc));
-        if (i - 2 >= 0) {  // its slot's previous piece (i+1) finished its gradients on this stream
+        if (!keep && i - 2 >= 0) {  // its slot's previous piece (i+1) finished its gradients on this stream
             SF_TRY(intra(piece(i - 2), true, sa));
             SF_TRY(cudaEventRecord(ev_prep[(i - 2) % NS], sa));
         }
         SF_TRY(cudaStreamWaitEvent(sa, ev_state[i % NS], 0));
         SF_TRY(run_bwd_chunk_grads(a, sa));
+        if (keep) SF_TRY(cudaEventRecord(ev_prep[i % NS], sa));
     }
     SF_TRY(cudaEventRecord(ev_aux_done, sa));
     SF_TRY(cudaEventRecord(ev_crit_done, sc));
     SF_TRY(cudaStreamWaitEvent(sm, ev_aux_done, 0));
     SF_TRY(cudaStreamWaitEvent(sm, ev_crit_done, 0));
     return SF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sf_status sf_fwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* q, const void* k,
+                     const void* v, const float* g, const float* beta, const float* S_in, void* o,
+                     float* S_out, float* S_saved, void* ws, size_t ws_bytes, void* stream_main,
+                     void* stream_aux) {
+    return fwd_seq(s, n_sub, lens, q, k, v, g, beta, S_in, o, S_out, S_saved, ws, ws_bytes, nullptr, 0,
+                   stream_main, stream_aux);
+}
+
+sf_status sf_bwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* q, const void* k,
+                     const void* v, const float* g, const float* beta, const float* S_saved,
+                     const void* dO, const float* dS_out, void* dq, void* dk, void* dv, float* dg,
+                     float* dbeta, float* dS_in, void* ws, size_t ws_bytes, void* stream_main,
+                     void* stream_aux) {
+    return bwd_seq(s, n_sub, lens, q, k, v, g, beta, S_saved, dO, dS_out, dq, dk, dv, dg, dbeta, dS_in,
+                   ws, ws_bytes, nullptr, 0, stream_main, stream_aux);
+}
+
+size_t sf_keep_bytes(const sf_shape* s, int n_sub, const int* lens) {
+    if (check_shape(s) != SF_OK || n_sub <= 0 || !lens) return 0;
+    SeqPlan p;
+    if (plan_seq(s, n_sub, lens, p) != SF_OK) return 0;
+    KeepPlan kp;
+    plan_keep(s, n_sub, lens, kp);
+    return kp.total;
+}
+
+sf_status sf_fwd_seq_keep(const sf_shape* s, int n_sub, const int* lens, const void* q,
+                          const void* k, const void* v, const float* g, const float* beta,
+                          const float* S_in, void* o, float* S_out, void* keep, size_t keep_bytes,
+                          void* ws, size_t ws_bytes, void* stream_main, void* stream_aux) {
+    if (!keep) return SF_ERR_WORKSPACE;
+    return fwd_seq(s, n_sub, lens, q, k, v, g, beta, S_in, o, S_out, nullptr, ws, ws_bytes, keep,
+                   keep_bytes, stream_main, stream_aux);
+}
+
+sf_status sf_bwd_seq_keep(const sf_shape* s, int n_sub, const int* lens, const void* q,
+                          const void* k, const void* v, const float* g, const float* beta,
+                          const void* keep, size_t keep_bytes, const void* dO, const float* dS_out,
+                          void* dq, void* dk, void* dv, float* dg, float* dbeta, float* dS_in,
+                          void* ws, size_t ws_bytes, void* stream_main, void* stream_aux) {
+    if (!keep) return SF_ERR_WORKSPACE;
+    return bwd_seq(s, n_sub, lens, q, k, v, g, beta, nullptr, dO, dS_out, dq, dk, dv, dg, dbeta, dS_in,
+                   ws, ws_bytes, keep, keep_bytes, stream_main, stream_aux);
 }
 
 sf_status sf_check(void* ws, void* stream) {

@@ -62,7 +62,14 @@ constexpr size_t kErrBytes = 256;
 
 WsLayout ws_layout(int B, int T, int H, int dk, int dv, int dtype, bool delta, bool bwd,
                    int nslots);
+// Parts of a slot: the forward's intermediates (G, Ed, W^T, U^T, chunk states,
+// Delta^T), P and T (tensor-core backward), the backward-only scratch.
+constexpr int kPartFwd = 1, kPartPT = 2, kPartBwd = 4;
+WsLayout ws_layout_parts(int B, int T, int H, int dk, int dv, int dtype, bool delta, int parts,
+                         int nslots);
 void bind_slot(Args& a, void* ws, const WsLayout& L, int slot, bool bwd);
+// Points the arrays of `parts` at a slot that starts at `base`.
+void bind_parts(Args& a, char* base, const WsLayout& L, int parts);
 
 // Kernel launchers (SIMT fp32 arithmetic; I/O in a.dtype).  Each returns the
 // cudaError_t of its launch.

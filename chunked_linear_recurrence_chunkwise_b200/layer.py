@@ -76,3 +76,43 @@ def backward(q, k, v, g, beta, dO, S_in=None, S_saved=None, dS_out=None, lens=No
         sf.sf_bwd_seq(sh, lens, q, k, v, g, beta, S_saved, dO, dS_out, dq, dk_, dv_, dg, db, dS_in,
                       ws, stream_main=stream, stream_aux=aux_stream)
     return {"dq": dq, "dk": dk_, "dv": dv_, "dg": dg, "dbeta": db, "dS_in": dS_in}
+
+
+def forward_keep(q, k, v, g=None, beta=None, S_in=None, lens=None, stream=None, aux_stream=None,
+                 ws=None, keep=None):
+    """Forward that keeps every piece's intermediates for :func:`backward_keep`
+    (no activation recompute).  Returns ``(o, S_out, keep)``; ``lens`` defaults
+    to one piece."""
+    _check_inputs(q, k, v, g, beta, S_in)
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    lens = [T] if lens is None else list(lens)
+    sh = sf.shape_of(q, v)
+    o = torch.empty_like(v)
+    S_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    keep = _ws(sf.sf_keep_bytes(sh, lens), q.device) if keep is None else keep
+    ws = _ws(sf.sf_seq_workspace_bytes(sh, lens, sf.SF_OP_FWD), q.device) if ws is None else ws
+    sf.sf_fwd_seq_keep(sh, lens, q, k, v, g, beta, S_in, o, S_out, keep, ws, stream_main=stream,
+                       stream_aux=aux_stream)
+    return o, S_out, keep
+
+
+def backward_keep(q, k, v, g, beta, dO, keep, dS_out=None, lens=None, stream=None, aux_stream=None,
+                  ws=None):
+    """Gradients from the intermediates :func:`forward_keep` kept (same inputs
+    and ``lens``).  Returns a dict with dq, dk, dv, dg, dbeta, dS_in."""
+    _check_inputs(q, k, v, g, beta, dO, dS_out)
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    lens = [T] if lens is None else list(lens)
+    sh = sf.shape_of(q, v)
+    dq = torch.empty_like(q)
+    dk_ = torch.empty_like(k)
+    dv_ = torch.empty_like(v)
+    dg = None if g is None else torch.empty_like(g)
+    db = None if beta is None else torch.empty_like(beta)
+    dS_in = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    ws = _ws(sf.sf_seq_workspace_bytes(sh, lens, sf.SF_OP_BWD), q.device) if ws is None else ws
+    sf.sf_bwd_seq_keep(sh, lens, q, k, v, g, beta, keep, dO, dS_out, dq, dk_, dv_, dg, db, dS_in, ws,
+                       stream_main=stream, stream_aux=aux_stream)
+    return {"dq": dq, "dk": dk_, "dv": dv_, "dg": dg, "dbeta": db, "dS_in": dS_in}

@@ -41,6 +41,9 @@ _SIGS = {
     "sf_bwd": (_I, [_SP] + [_P] * 14 + [_P, _S, _P]),
     "sf_fwd_seq": (_I, [_SP, _I, _IP] + [_P] * 9 + [_P, _S, _P, _P]),
     "sf_bwd_seq": (_I, [_SP, _I, _IP] + [_P] * 14 + [_P, _S, _P, _P]),
+    "sf_keep_bytes": (_S, [_SP, _I, _IP]),
+    "sf_fwd_seq_keep": (_I, [_SP, _I, _IP] + [_P] * 8 + [_P, _S, _P, _S, _P, _P]),
+    "sf_bwd_seq_keep": (_I, [_SP, _I, _IP] + [_P] * 5 + [_P, _S] + [_P] * 8 + [_P, _S, _P, _P]),
     "sf_fwd_noalloc": (_I, [_SP] + [_P] * 8 + [_P]),
     "sf_check": (_I, [_P, _P]),
     "sf_status_string": (ctypes.c_char_p, [_I]),
@@ -149,6 +152,33 @@ def sf_bwd_seq(sh, lens, q, k, v, g, beta, S_saved, dO, dS_out, dq, dk, dv, dg, 
                            _ptr(g), _ptr(beta), _ptr(S_saved), _ptr(dO), _ptr(dS_out), _ptr(dq),
                            _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(dS_in), _ptr(ws),
                            ws_bytes, sm, sa), "sf_bwd_seq")
+
+
+def sf_keep_bytes(sh: sf_shape, lens) -> int:
+    return int(_lib.sf_keep_bytes(ctypes.byref(sh), len(lens), _lens(lens)))
+
+
+def sf_fwd_seq_keep(sh, lens, q, k, v, g, beta, S_in, o, S_out, keep, ws, keep_bytes=None,
+                    ws_bytes=None, stream_main=None, stream_aux=None):
+    keep_bytes = keep.numel() * keep.element_size() if keep_bytes is None else keep_bytes
+    ws_bytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
+    sm = _stream(stream_main)
+    sa = sm if stream_aux is None else _stream(stream_aux)
+    _check(_lib.sf_fwd_seq_keep(ctypes.byref(sh), len(lens), _lens(lens), _ptr(q), _ptr(k), _ptr(v),
+                                _ptr(g), _ptr(beta), _ptr(S_in), _ptr(o), _ptr(S_out), _ptr(keep),
+                                keep_bytes, _ptr(ws), ws_bytes, sm, sa), "sf_fwd_seq_keep")
+
+
+def sf_bwd_seq_keep(sh, lens, q, k, v, g, beta, keep, dO, dS_out, dq, dk, dv, dg, dbeta, dS_in, ws,
+                    keep_bytes=None, ws_bytes=None, stream_main=None, stream_aux=None):
+    keep_bytes = keep.numel() * keep.element_size() if keep_bytes is None else keep_bytes
+    ws_bytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
+    sm = _stream(stream_main)
+    sa = sm if stream_aux is None else _stream(stream_aux)
+    _check(_lib.sf_bwd_seq_keep(ctypes.byref(sh), len(lens), _lens(lens), _ptr(q), _ptr(k), _ptr(v),
+                                _ptr(g), _ptr(beta), _ptr(keep), keep_bytes, _ptr(dO), _ptr(dS_out),
+                                _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(dS_in),
+                                _ptr(ws), ws_bytes, sm, sa), "sf_bwd_seq_keep")
 
 
 def sf_fwd_noalloc(sh, q, k, v, g, beta, S_in, o, S_out, stream=None):

@@ -122,6 +122,39 @@ sf_status sf_bwd_seq(const sf_shape* shape, int n_sub, const int* lens, const vo
                      void* dk, void* dv, float* dg, float* dbeta, float* dS_in, void* ws,
                      size_t ws_bytes, void* stream_main, void* stream_aux);
 
+/* Sub-sequence drivers without activation recompute.  The StateFlow summary
+ * (gptget.net, sections 关键结果 and 方法详解) reports its pipeline both without
+ * and with activation recompute; sf_fwd_seq / sf_bwd_seq are the recompute
+ * form (the backward re-runs every piece from its stored entering state), these
+ * are the other: the forward keeps every piece's intermediates in `keep` and
+ * the backward reads them instead of recomputing.  That skips the intra-chunk
+ * kernel and the forward state pass of every piece in the backward at the cost
+ * of device memory that grows with T.
+ *
+ * sf_keep_bytes: bytes of `keep` for this shape and cut (0 on an invalid
+ * argument).  On the bf16 path with d_k = d_v = 128 that is about 97 KB per
+ * 64-token chunk and head: the cumulative decay, W^T, U^T, the chunk states,
+ * Delta^T, P and T; on the other paths the same minus P and T, at fp32.
+ *
+ * sf_fwd_seq_keep: as sf_fwd_seq, with `keep` (device, 256-byte aligned,
+ * keep_bytes >= sf_keep_bytes) receiving the intermediates; ws is the same
+ * workspace as sf_fwd_seq's (sf_seq_workspace_bytes(..., SF_OP_FWD)).
+ * sf_bwd_seq_keep: as sf_bwd_seq, reading `keep` as the forward left it (same
+ * q, k, v, g, beta, shape and lens) instead of S_saved; ws as sf_bwd_seq's.
+ * `keep` NULL or too small, or misaligned: SF_ERR_WORKSPACE. */
+size_t sf_keep_bytes(const sf_shape* shape, int n_sub, const int* lens);
+
+sf_status sf_fwd_seq_keep(const sf_shape* shape, int n_sub, const int* lens, const void* q,
+                          const void* k, const void* v, const float* g, const float* beta,
+                          const float* S_in, void* o, float* S_out, void* keep, size_t keep_bytes,
+                          void* ws, size_t ws_bytes, void* stream_main, void* stream_aux);
+
+sf_status sf_bwd_seq_keep(const sf_shape* shape, int n_sub, const int* lens, const void* q,
+                          const void* k, const void* v, const float* g, const float* beta,
+                          const void* keep, size_t keep_bytes, const void* dO, const float* dS_out,
+                          void* dq, void* dk, void* dv, float* dg, float* dbeta, float* dS_in,
+                          void* ws, size_t ws_bytes, void* stream_main, void* stream_aux);
+
 /* Forward without a caller workspace, for callers that cannot allocate device
  * memory (a plugin that is handed only its input and output buffers by a
  * framework that plans all memory up front, code running inside an

@@ -98,6 +98,38 @@ def test_sequence_lengths_must_sum_to_T(sf):
     assert rc == sf.SF_ERR_INVALID
 
 
+def test_keep_drivers_check_the_kept_buffer(sf):
+    """The no-recompute drivers reject a missing, short or misaligned keep buffer
+    (and a bad cut) before any CUDA call."""
+    sh = sf.shape(1, 300, 2, 64, 64, sf.SF_F32)
+    assert sf.sf_keep_bytes(sh, [100, 100]) == 0
+    need = sf.sf_keep_bytes(sh, [100, 200])
+    assert need > 0
+    # more pieces keep more (each piece's chunks are padded to 64 tokens)
+    assert sf.sf_keep_bytes(sh, [100] * 3) > sf.sf_keep_bytes(sh, [300])
+    tc = sf.shape(1, 256, 2, 128, 128, sf.SF_BF16)
+    assert sf.sf_keep_bytes(tc, [256]) > 0
+    lens = (ctypes.c_int * 2)(100, 200)
+    P, S = ctypes.c_void_p, ctypes.c_size_t
+
+    def fwd(keep, keep_bytes, lens_=lens):
+        return sf.raw_call("sf_fwd_seq_keep", ctypes.byref(sh), 2, lens_, P(16), P(16), P(16), None,
+                           None, None, P(16), None, P(keep) if keep else None, S(keep_bytes),
+                           P(256), S(1 << 30), None, None)
+
+    def bwd(keep, keep_bytes):
+        return sf.raw_call("sf_bwd_seq_keep", ctypes.byref(sh), 2, lens, P(16), P(16), P(16), None,
+                           None, P(keep) if keep else None, S(keep_bytes), P(16), None, P(16), P(16),
+                           P(16), None, None, None, P(256), S(1 << 30), None, None)
+
+    assert fwd(0, need) == sf.SF_ERR_WORKSPACE
+    assert fwd(256, need - 1) == sf.SF_ERR_WORKSPACE
+    assert fwd(272, need) == sf.SF_ERR_WORKSPACE       # not 256-byte aligned
+    assert fwd(256, need, (ctypes.c_int * 2)(100, 100)) == sf.SF_ERR_INVALID
+    assert bwd(0, need) == sf.SF_ERR_WORKSPACE
+    assert bwd(256, need - 1) == sf.SF_ERR_WORKSPACE
+
+
 def test_product_path_does_not_reference_the_oracle():
     pkg = os.path.join(ROOT, "chunked_linear_recurrence_chunkwise_b200")
     for dirpath, _, files in os.walk(pkg):

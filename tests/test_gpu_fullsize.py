@@ -25,15 +25,25 @@ def rel_l2(x, ref):
     return float(np.linalg.norm(x - ref) / (n if n > 0 else 1.0))
 
 
-def run_gpu(w, x, lens, stream_aux=True):
+def run_gpu(w, x, lens, stream_aux=True, keep=False):
+    """The workload through the sub-sequence drivers: with activation recompute
+    (keep=False) or with the forward's intermediates kept for the backward."""
     from chunked_linear_recurrence_chunkwise_b200 import layer
     aux = torch.cuda.Stream() if stream_aux else None
-    o, S_out, S_saved = layer.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], lens=lens,
-                                      aux_stream=aux)
+    if keep:
+        o, S_out, kept = layer.forward_keep(x["q"], x["k"], x["v"], x["g"], x["beta"], lens=lens,
+                                            aux_stream=aux)
+    else:
+        o, S_out, S_saved = layer.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], lens=lens,
+                                          aux_stream=aux)
     gr = None
     if x["dO"] is not None:
-        gr = layer.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["dO"], S_saved=S_saved,
-                            lens=lens, aux_stream=aux)
+        if keep:
+            gr = layer.backward_keep(x["q"], x["k"], x["v"], x["g"], x["beta"], x["dO"], kept,
+                                     lens=lens, aux_stream=aux)
+        else:
+            gr = layer.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["dO"], S_saved=S_saved,
+                                lens=lens, aux_stream=aux)
     torch.cuda.synchronize()
     return o, S_out, gr
 
@@ -46,13 +56,19 @@ def sampled(t, heads, has_batch=True):
     return outs
 
 
-@pytest.mark.parametrize("name", list(inputs.WORKLOADS))
-def test_full_size_sampled_heads_match_oracle(name):
+# every workload with activation recompute; the kept-intermediates drivers (the
+# bench's configuration) on the gated-delta-rule workloads
+CASES = [(name, False) for name in inputs.WORKLOADS] + [
+    (name, True) for name in inputs.WORKLOADS if inputs.WORKLOADS[name].variant == "gdn"]
+
+
+@pytest.mark.parametrize("name,keep", CASES)
+def test_full_size_sampled_heads_match_oracle(name, keep):
     w = inputs.WORKLOADS[name]
     lens = inputs.sub_lengths(w)
     heads = [(0, 0), (w.B - 1, w.H - 1)]
     x = inputs.to_torch(w, device="cuda", keep_heads=heads)
-    o, S_out, gr = run_gpu(w, x, lens)
+    o, S_out, gr = run_gpu(w, x, lens, keep=keep)
     tol = TOL[w.dtype]
     # both sampled heads as a batch of two single-head problems (the oracle runs them in parallel)
     cat = lambda key: (None if x["kept"][0][key] is None
