@@ -121,7 +121,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                          const __grid_constant__ CUtensorMap tm_ut, const __grid_constant__ CUtensorMap tm_t,
                          const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_ddt,
                          const __grid_constant__ CUtensorMap tm_sc, const __grid_constant__ CUtensorMap tm_dsc,
-                         const Args a) {
+                         const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
+                         const __grid_constant__ CUtensorMap tm_dv, const Args a) {
     using L = FusedSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -326,11 +327,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ow[p] = pack_bf16(br * x[qq * 8 + 2 * p], br * x[qq * 8 + 2 * p + 1]);
                     }
                 }
-                if (r < Lr) {
-                    uint4* dst = (uint4*)((__nv_bfloat16*)a.dv_ + tok_index(a, b, t0 + r, h) * kD + cq * 32);
+                // dv row r into the dO tile (dead after phase A) for one TMA store
 #pragma unroll
-                    for (int qq = 0; qq < 4; ++qq) dst[qq] = ov[qq];
-                }
+                for (int qq = 0; qq < 4; ++qq)
+                    *(uint4*)(sm + L::dO + (cq >> 1) * kHalf + sw128(r, (cq & 1) * 4 + qq)) = ov[qq];
                 P(P_VD)[r] = vd;
                 put_row(sm + L::dDt + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);  // K-major A of dA
             }
@@ -368,6 +368,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------- phase B: F K, F^T Q onto the rescaled partials; dKhat = T^T dW
     if (tid == 0) {
+        tma_store_4d(&tm_dv, sm + L::dO, 0, h, t0, b);  // rows past the piece's end are clipped
+        tma_store_4d(&tm_dv, sm + L::dO + kHalf, 64, h, t0, b);
+        bulk_commit();
         tc_fence_after();
         const uint32_t f = smem_u32(sm + L::F), k = smem_u32(sm + L::K), q = smem_u32(sm + L::Q);
         const uint32_t tb = smem_u32(sm + L::Tb), dw = smem_u32(sm + L::Dt);
@@ -547,18 +550,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float kp = __shfl_xor_sync(0xffffffffu, y[q], 16);
             if (hi) x[q] += kp;
         }
-        if (r < Lr) {
-            uint4* dst = (uint4*)((__nv_bfloat16*)(hi ? a.dk_ : a.dq) + tok_index(a, b, t0 + r, h) * kD + cq * 32);
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                uint4 u;
-                u.x = pack_bf16(x[qq * 8 + 0], x[qq * 8 + 1]);
-                u.y = pack_bf16(x[qq * 8 + 2], x[qq * 8 + 3]);
-                u.z = pack_bf16(x[qq * 8 + 4], x[qq * 8 + 5]);
-                u.w = pack_bf16(x[qq * 8 + 6], x[qq * 8 + 7]);
-                dst[qq] = u;
-            }
-        }
+        // dq rows into the W^T tile, dk rows into the U^T tile (both dead after phase C)
+        put_row(sm + (hi ? L::Ut : L::Wt) + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {  // rows past the piece's end are clipped by the stores
+        tma_store_4d(&tm_dq, sm + L::Wt, 0, h, t0, b);
+        tma_store_4d(&tm_dq, sm + L::Wt + kHalf, 64, h, t0, b);
+        tma_store_4d(&tm_dk, sm + L::Ut, 0, h, t0, b);
+        tma_store_4d(&tm_dk, sm + L::Ut + kHalf, 64, h, t0, b);
+        bulk_commit();
     }
 
 teardown:
@@ -568,6 +570,7 @@ teardown:
             mbar_wait(bar_ld1, 0);
         }
         if (mma_pending) mbar_wait(bar_mma, mph ^ 1);
+        bulk_wait<0>();  // the output stores have finished
     }
     tc_fence_before();
     __syncthreads();
@@ -584,11 +587,14 @@ cudaError_t launch_grad_fused_tc(const Args& a, cudaStream_t s) {
     if (BH == 0 || a.NC == 0) return cudaSuccess;
     const uint64_t rows = (uint64_t)BH * a.NC * kD, rowsC = (uint64_t)BH * a.NC * kChunk;
     CUtensorMap tm_q{}, tm_k{}, tm_do{}, tm_wt{}, tm_ut{}, tm_t{}, tm_dt{}, tm_ddt{}, tm_sc{}, tm_dsc{};
+    CUtensorMap tm_dq{}, tm_dk{}, tm_dv{};
     const bool ok = tmap_tokens(&tm_q, a.q, a, kD) && tmap_tokens(&tm_k, a.k, a, kD) &&
                     tmap_tokens(&tm_do, a.dO, a, kD) && tmap_2d(&tm_wt, a.Wt, 64, rows, 128) &&
                     tmap_2d(&tm_ut, a.Ut, 64, rows, 128) && tmap_2d(&tm_t, a.Tm, 64, rowsC, 64) &&
                     tmap_2d(&tm_dt, a.Dt, 64, rows, 128) && tmap_2d(&tm_ddt, a.dDt, 64, rows, 128) &&
-                    tmap_2d(&tm_sc, a.Sc, kD, rows, 128) && tmap_2d(&tm_dsc, a.dSc, kD, rows, 128);
+                    tmap_2d(&tm_sc, a.Sc, kD, rows, 128) && tmap_2d(&tm_dsc, a.dSc, kD, rows, 128) &&
+                    tmap_tokens(&tm_dq, a.dq, a, kD) && tmap_tokens(&tm_dk, a.dk_, a, kD) &&
+                    tmap_tokens(&tm_dv, a.dv_, a, kD);
     if (!ok) return cudaErrorInvalidValue;
     const size_t smem = FusedSmem::Size + 1024;
     cudaError_t e = cudaFuncSetAttribute(grad_fused_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -596,7 +602,7 @@ cudaError_t launch_grad_fused_tc(const Args& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     timing_begin(KK_GRAD_FUSED, s);
     grad_fused_tc_kernel<<<dim3(a.NC, BH), kThreads, smem, s>>>(tm_q, tm_k, tm_do, tm_wt, tm_ut, tm_t, tm_dt,
-                                                                tm_ddt, tm_sc, tm_dsc, a);
+                                                                tm_ddt, tm_sc, tm_dsc, tm_dq, tm_dk, tm_dv, a);
     e = cudaGetLastError();
     timing_end(KK_GRAD_FUSED, s);
     return e;
