@@ -86,6 +86,7 @@ bool tc_eligible(const Args& a);
 cudaError_t launch_state_fwd_tc(const Args& a, cudaStream_t s);
 // with_p: also store P (backward recompute)
 cudaError_t launch_intra_tc(const Args& a, bool with_p, cudaStream_t s);
+// reads P from a.Pm when it is set (the forward that keeps its intermediates)
 cudaError_t launch_output_tc(const Args& a, cudaStream_t s);
 // reverse dS pass; consumes P from the backward intra kernel (no dDelta pre-pass)
 cudaError_t launch_state_bwd_tc(const Args& a, cudaStream_t s);

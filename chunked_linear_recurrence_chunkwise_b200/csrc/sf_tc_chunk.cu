@@ -646,6 +646,125 @@ teardown:
     }
 }
 
+// Output kernel when the intra kernel has stored P (the forward that keeps its
+// intermediates): O^T = gamma-scaled (S^T Q^T) + Delta^T P^T with P read, not
+// recomputed, so both products go out at once and K is not needed.
+struct OutPSmem {
+    static constexpr int Q = 0;                // [dkblk][64 r][64]; later the O^T staging
+    static constexpr int St = Q + kTile;       // S^T [kblk][128 j][64]
+    static constexpr int Dt = St + 2 * kTile;  // Delta^T [128 j][64 r]
+    static constexpr int Pb = Dt + kTile;      // P, K-major [r][64 i]
+    static constexpr int Gs = Pb + kHalf;
+    static constexpr int Bar = Gs + 256;
+    static constexpr int Misc = Bar + 16;
+    static constexpr int Size = Misc + 16;
+};
+
+__global__ void __launch_bounds__(128)
+    output_p_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_p,
+                       const __grid_constant__ CUtensorMap tm_sc, const __grid_constant__ CUtensorMap tm_dt,
+                       const __grid_constant__ CUtensorMap tm_o, const Args a) {
+    using L = OutPSmem;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    float* Gs = (float*)(sm + L::Gs);
+    uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);
+    uint64_t* bar_mma = bar_ld + 1;
+    uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
+    volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
+
+    const int c = blockIdx.x, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+    const int NC = a.NC, TP = NC * kChunk;
+    const int t0 = c * kChunk;
+    const int tid = threadIdx.x, warp = tid >> 5;
+
+    if (tid == 0) {
+        mbar_init(bar_ld, 1);
+        mbar_init(bar_mma, 1);
+        *s_abort = 0;
+        fence_barrier_init();
+        mbar_expect_tx(bar_ld, kTile + 2 * kTile + kTile + kHalf + 256);
+        tma_load_4d(sm + L::Q, &tm_q, 0, h, t0, b, bar_ld);
+        tma_load_4d(sm + L::Q + kHalf, &tm_q, 64, h, t0, b, bar_ld);
+        tma_load_2d(sm + L::St, &tm_sc, 0, (bh * NC + c) * kD, bar_ld);
+        tma_load_2d(sm + L::St + kTile, &tm_sc, 64, (bh * NC + c) * kD, bar_ld);
+        tma_load_2d(sm + L::Dt, &tm_dt, 0, (bh * NC + c) * kD, bar_ld);
+        tma_load_2d(sm + L::Pb, &tm_p, 0, (bh * NC + c) * kChunk, bar_ld);
+        bulk_load(Gs, a.G + (size_t)bh * TP + t0, 256, bar_ld);
+    }
+    if (warp == 0) tmem_alloc(s_tmem, 128);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t tX2 = tmem, tX3 = tmem + 64;
+    bool ld_pending = false, mma_pending = false;
+    if (tid == 0) {
+        if (!mbar_wait(bar_ld, 0)) {
+            *s_abort = 1;
+            ld_pending = true;
+            atomicExch(a.err, kErrTimeoutTma);
+        } else {
+            tc_fence_after();
+            const uint32_t q = smem_u32(sm + L::Q), st = smem_u32(sm + L::St);
+            const uint32_t dt = smem_u32(sm + L::Dt), pb = smem_u32(sm + L::Pb);
+            constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(tX2, sdesc(st + (ks >> 2) * kTile + (ks & 3) * 32, 16, 1024),
+                         sdesc(q + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024), id, ks > 0);  // S^T Q^T
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tX3, sdesc(dt + ks * 32, 16, 1024), sdesc(pb + ks * 32, 16, 1024), id, ks > 0);  // Delta^T P^T
+            mma_commit(bar_mma);
+            if (!mbar_wait(bar_mma, 0)) {
+                *s_abort = 1;
+                mma_pending = true;
+                atomicExch(a.err, kErrTimeoutMma);
+            }
+        }
+    }
+    __syncthreads();
+    if (*s_abort) goto teardown;
+    tc_fence_after();
+    {
+        const int j = tid;  // O^T row = d_v index = TMEM lane
+        float x2[64], x3[64];
+        tmem_ld32(taddr(tX2, 32 * warp, 0), *(float(*)[32]) & x2[0]);
+        tmem_ld32(taddr(tX2, 32 * warp, 32), *(float(*)[32]) & x2[32]);
+        tmem_ld32(taddr(tX3, 32 * warp, 0), *(float(*)[32]) & x3[0]);
+        tmem_ld32(taddr(tX3, 32 * warp, 32), *(float(*)[32]) & x3[32]);
+        tmem_ld_wait();
+        uint8_t* ost = sm + L::Q;  // [jblk][64 r][64 j] staging (Q is dead: the products are done)
+        const uint32_t jb = (uint32_t)(j >> 6) * kHalf, jq = (j & 63) >> 3, je = (j & 7) * 2;
+#pragma unroll
+        for (int r = 0; r < 64; ++r) {
+            const float o = __expf(Gs[r]) * x2[r] + x3[r];
+            *(__nv_bfloat16*)(ost + jb + sw128(r, jq) + je) = __float2bfloat16_rn(o);
+        }
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        tma_store_4d(&tm_o, sm + L::Q, 0, h, t0, b);
+        tma_store_4d(&tm_o, sm + L::Q + kHalf, 64, h, t0, b);
+        bulk_commit();
+    }
+
+teardown:
+    if (tid == 0) {
+        if (ld_pending) mbar_wait(bar_ld, 0);
+        if (mma_pending) mbar_wait(bar_mma, 0);
+        bulk_wait<0>();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
 template <typename K>
 cudaError_t set_smem(K kern, size_t smem) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -689,6 +808,22 @@ cudaError_t launch_output_tc(const Args& a, cudaStream_t s) {
     const int BH = a.B * a.H;
     if (BH == 0 || a.NC == 0) return cudaSuccess;
     const uint64_t rows = (uint64_t)BH * a.NC * kD;
+    if (a.Pm) {  // P stored by the intra kernel of this forward
+        CUtensorMap tm_q{}, tm_p{}, tm_sc{}, tm_dt{}, tm_o{};
+        const bool ok = tmap_tokens(&tm_q, a.q, a, kD) &&
+                        tmap_2d(&tm_p, a.Pm, 64, (uint64_t)BH * a.NC * kChunk, 64) &&
+                        tmap_2d(&tm_sc, a.Sc, kD, rows, 128) && tmap_2d(&tm_dt, a.Dt, 64, rows, 128) &&
+                        tmap_tokens(&tm_o, a.o, a, kD);
+        if (!ok) return cudaErrorInvalidValue;
+        const size_t smem = OutPSmem::Size + 1024;
+        cudaError_t e = set_smem(output_p_tc_kernel, smem);
+        if (e != cudaSuccess) return e;
+        timing_begin(KK_OUTPUT, s);
+        output_p_tc_kernel<<<dim3(a.NC, BH), 128, smem, s>>>(tm_q, tm_p, tm_sc, tm_dt, tm_o, a);
+        e = cudaGetLastError();
+        timing_end(KK_OUTPUT, s);
+        return e;
+    }
     CUtensorMap tm_q{}, tm_k{}, tm_sc{}, tm_dt{}, tm_o{};
     const bool ok = tmap_tokens(&tm_q, a.q, a, kD) && tmap_tokens(&tm_k, a.k, a, kD) &&
                     tmap_2d(&tm_sc, a.Sc, kD, rows, 128) && tmap_2d(&tm_dt, a.Dt, 64, rows, 128) &&
