@@ -44,6 +44,8 @@ def parse_args(argv=None):
     p.add_argument("--mode", default="keep", choices=["keep", "recompute"],
                    help="keep: the forward keeps its intermediates for the backward; recompute: "
                         "the backward recomputes every piece from its stored entering state")
+    p.add_argument("--no-other-mode", action="store_true",
+                   help="do not time the other driver form beside the headline one")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=16384)
@@ -95,7 +97,7 @@ def tc_path(w) -> bool:
     return w.dtype == "bf16" and w.d == 128
 
 
-def kernel_units(name: str, w) -> dict:
+def kernel_units(name: str, w, mode: str = "keep") -> dict:
     """Algorithmic bytes and flops of one chunk-head (64 tokens of one head) per kernel.
 
     Bytes count each tensor the kernel must read or write once, at the
@@ -120,9 +122,11 @@ def kernel_units(name: str, w) -> dict:
                           mm(2 * C, C, d) + 2 * mm(d, C, C)),
             # read W^T, U^T, k, decay table; write S^T, Delta^T
             "state_fwd": (3 * tile + 2 * C * f + st + tile, mm(d, C, d) + mm(d, d, C)),
-            # read q, k, S^T, Delta^T, G; write o
+            # read q, k, S^T, Delta^T, G; write o (P recomputed on chip)
             "output": (2 * tile + st + tile + C * f + tile,
                        mm(C, C, d) + mm(d, C, d) + mm(d, C, C)),
+            # read q, S^T, Delta^T, the stored P, G; write o
+            "output_p": (tile + st + tile + C * C * e + C * f + tile, mm(d, C, d) + mm(d, C, C)),
             # read k, dO, q, W^T, P, G; write dS'^T, dDelta^T
             "state_bwd": (4 * tile + C * C * e + C * f + st + tile,
                           mm(d, C, d) + mm(d, C, C) + 2 * mm(d, d, C)),
@@ -153,11 +157,26 @@ def kernel_units(name: str, w) -> dict:
             "grad_attn": (5 * C * d * e + 2 * d * d * e + C * d * f + 2 * C * f,
                           tri_i * 8 * d + 4 * C * d * d),
         }
+    if tc_path(w) and name == "output" and mode == "keep":
+        name = "output_p"  # the forward that keeps P runs the output kernel that reads it
     b, fl = tab.get(name, (0, 0))
     return {"bytes": b, "flops": fl}
 
 
-def roofline(timing: dict, w, steps: int, peaks: dict, peaks_src: str, clocks: dict):
+# DRAM bytes (read + write) per launch of one 4096-token piece of the 32-head, d = 128
+# workload (2048 chunk-heads), from the committed ncu captures of the current kernels
+# (profiles/<kernel>_gdn_bf16_h32.md); per launch they scale with the chunk-heads covered.
+NCU_TRAFFIC_2048 = {
+    "grad_fused": 504.110e6,
+    "state_bwd": 222.702e6,
+    "state_fwd": 162.303e6,
+    "intra_bwd": 158.974e6,
+    "output": 167.309e6,  # output_p_tc_kernel (the keep form)
+}
+
+
+def roofline(timing: dict, w, steps: int, peaks: dict, peaks_src: str, clocks: dict,
+             mode: str = "keep"):
     """Roofline object of the kernel with the largest total time (serialized pass).
 
     Every kernel of this layer moves more bytes than its arithmetic can hide
@@ -175,14 +194,16 @@ def roofline(timing: dict, w, steps: int, peaks: dict, peaks_src: str, clocks: d
     # every launch processes one piece (all heads, batch rows); pieces of the workload
     # are uniform, so a launch covers chunk_heads / n_sub chunk-heads
     units_per_launch = chunk_heads / w.n_sub
-    u = kernel_units(name, w)
+    u = kernel_units(name, w, mode)
     per_launch_s = ms / 1e3 / launches
     gbs = u["bytes"] * units_per_launch / per_launch_s / 1e9
     tfs = u["flops"] * units_per_launch / per_launch_s / 1e12
     hbm = float(peaks["hbm_gbs"])
     bf16 = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1590.0)))
     obj = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
-           "frac": round(gbs / hbm, 4), "traffic": None,
+           "frac": round(gbs / hbm, 4),
+           "traffic": (round(NCU_TRAFFIC_2048[name] * units_per_launch / 2048)
+                       if (tc_path(w) and mode == "keep" and name in NCU_TRAFFIC_2048) else None),
            "kernel": name, "launches": launches, "avg_launch_ms": round(ms / launches, 4),
            "bytes_per_launch": int(u["bytes"] * units_per_launch),
            "tensor_tflops": round(tfs, 2), "tensor_frac": round(tfs / bf16, 4),
@@ -374,19 +395,21 @@ def run_sf(args, w, rank, world, local_rank):
 
     # ---- the other driver form, timed the same way (reported beside the headline)
     other = "recompute" if args.mode == "keep" else "keep"
-    for _ in range(args.warmup):
-        step(x, mode=other)
-    barrier()
-    torch.cuda.synchronize()
-    e0.record(main)
-    for _ in range(args.steps):
-        step(x, mode=other)
-    e1.record(main)
-    torch.cuda.synchronize()
-    barrier()
-    ms_other = reduce_max(e0.elapsed_time(e1) / args.steps, device=dev)
-    sf.sf_check(ws_f, main)
-    sf.sf_check(ws_b, main)
+    ms_other = None
+    if not args.no_other_mode:
+        for _ in range(args.warmup):
+            step(x, mode=other)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(main)
+        for _ in range(args.steps):
+            step(x, mode=other)
+        e1.record(main)
+        torch.cuda.synchronize()
+        barrier()
+        ms_other = reduce_max(e0.elapsed_time(e1) / args.steps, device=dev)
+        sf.sf_check(ws_f, main)
+        sf.sf_check(ws_b, main)
 
     # ---- per-kernel durations: the same steps with both driver streams on one
     # stream, every launch bracketed by CUDA events on its stream (with two
@@ -452,12 +475,13 @@ def run_sf(args, w, rank, world, local_rank):
                        "keep_bytes": keep.numel()},
             "modes": {args.mode: {"ms_per_step": round(ms_max, 4),
                                   "value": round(job_tokens_per_s(world, B, T, ms_max), 1)},
-                      other: {"ms_per_step": round(ms_other, 4),
-                              "value": round(job_tokens_per_s(world, B, T, ms_other), 1)}},
+                      other: None if ms_other is None else
+                      {"ms_per_step": round(ms_other, 4),
+                       "value": round(job_tokens_per_s(world, B, T, ms_other), 1)}},
             "clocks": clocks,
             "gpu_launches": launches,
             "e2e": e2e,
-            "roofline": roofline(timing, w, args.steps, peaks, src, clocks),
+            "roofline": roofline(timing, w, args.steps, peaks, src, clocks, args.mode),
             "kernels": {k_: {"launches": v[0] // max(1, args.steps),
                              "ms_per_step": round(v[1] / args.steps, 4)} for k_, v in timing.items()
                         if v[0] > 0},
