@@ -118,7 +118,9 @@ def kernel_units(name: str, w, mode: str = "keep") -> dict:
             # read k, v (+ q), g, beta; write G, W^T, U^T (+ P)
             "intra_fwd": (2 * tile + 2 * C * f + C * f + 2 * tile,
                           mm(C, C, d) + 2 * mm(d, C, C)),
-            "intra_bwd": (3 * tile + 2 * C * f + C * f + 2 * tile + C * C * e,
+            # as intra_fwd, also reading q and writing P (and T for the delta rule)
+            "intra_bwd": (3 * tile + 2 * C * f + C * f + 2 * tile
+                          + (2 if w.has_beta else 1) * C * C * e,
                           mm(2 * C, C, d) + 2 * mm(d, C, C)),
             # read W^T, U^T, k, decay table; write S^T, Delta^T
             "state_fwd": (3 * tile + 2 * C * f + st + tile, mm(d, C, d) + mm(d, d, C)),
