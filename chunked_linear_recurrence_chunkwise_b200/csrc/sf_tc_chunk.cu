@@ -481,7 +481,7 @@ teardown:
     if (tid == 0) {
         if (ld_pending) mbar_wait(bar_ld, 0);
         if (mma_pending) mbar_wait(bar_mma, mph ^ 1);
-        bulk_wait<0>();
+        bulk_wait_read<0>();  // stores have read shared memory (their writes land before the grid completes)
     }
     tc_fence_before();
     __syncthreads();
@@ -636,7 +636,7 @@ teardown:
     if (tid == 0) {
         if (ld_pending) mbar_wait(bar_ld, 0);
         if (mma_pending) mbar_wait(bar_mma, mph ^ 1);
-        bulk_wait<0>();
+        bulk_wait_read<0>();  // stores have read shared memory (their writes land before the grid completes)
     }
     tc_fence_before();
     __syncthreads();
@@ -755,7 +755,7 @@ teardown:
     if (tid == 0) {
         if (ld_pending) mbar_wait(bar_ld, 0);
         if (mma_pending) mbar_wait(bar_mma, 0);
-        bulk_wait<0>();
+        bulk_wait_read<0>();  // stores have read shared memory (their writes land before the grid completes)
     }
     tc_fence_before();
     __syncthreads();

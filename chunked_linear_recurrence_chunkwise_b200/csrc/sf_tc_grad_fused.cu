@@ -27,8 +27,11 @@
 // Shared memory of operands that die after the first phase is reused for the
 // later tiles and scratch (about 218 KB in all, one CTA per SM).  Sixteen
 // warps share the element-wise work: warp w reads TMEM lane quadrant w % 4
-// and a quarter of the columns, w / 4; the operands arrive in two groups so
-// that the first products start while the state tiles are still in flight.
+// and a quarter of the columns, w / 4.  A seventeenth warp issues the copies
+// and the UMMAs.  The operands arrive in six groups and the first phase's
+// products are committed in three, so that each product starts as soon as
+// its tiles have landed and the element-wise work on the first products
+// runs while the later ones are still on the tensor core.
 
 #include <cuda.h>
 
@@ -44,7 +47,10 @@ using namespace tc;
 constexpr int kD = 128;
 constexpr int kTile = 16384;
 constexpr int kHalf = 8192;
-constexpr int kThreads = 512;
+constexpr int kThreads = 512;          // element-wise warps 0-15
+constexpr int kBlock = kThreads + 32;  // + the issuing warp
+constexpr int kIss = kThreads;         // the thread that issues copies and UMMAs
+constexpr int kLoads = 6;              // operand groups, in the order they are needed
 
 // Per-row partial sums, each kept per column quarter: [term][quarter][64 rows].
 enum PartTerm {
@@ -77,8 +83,8 @@ struct FusedSmem {
     static constexpr int csp = Bs + 256;          // fp32 [8][64]: column sums of PD over 8-row groups
     static constexpr int part = csp + 8 * 256;    // fp32 [P_COUNT][4][64]
     static constexpr int red = part + P_COUNT * 4 * 256;  // fp32 [32]: per-warp <S, dS'>, last-row sums
-    static constexpr int Bar = red + 128;         // 3 mbarriers
-    static constexpr int Misc = Bar + 24;
+    static constexpr int Bar = red + 128;         // kLoads load + 3 first-phase + 2 mbarriers
+    static constexpr int Misc = Bar + (kLoads + 5) * 8;
     static constexpr int Size = Misc + 16;
 };
 
@@ -115,7 +121,7 @@ __device__ __forceinline__ void put_row(uint8_t* tile, int row, int q0, const fl
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kBlock, 1)
     grad_fused_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_wt,
                          const __grid_constant__ CUtensorMap tm_ut, const __grid_constant__ CUtensorMap tm_t,
@@ -133,9 +139,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* Ef = (float*)(sm + L::dSt);
     float* part = (float*)(sm + L::part);
     float* red = (float*)(sm + L::red);
-    uint64_t* bar_ld0 = (uint64_t*)(sm + L::Bar);
-    uint64_t* bar_ld1 = bar_ld0 + 1;
-    uint64_t* bar_mma = bar_ld0 + 2;
+    uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);  // [kLoads]
+    uint64_t* bar_a = bar_ld + kLoads;            // first-phase products, three groups
+    uint64_t* bar_mma = bar_a + 3;                // later phases
+    uint64_t* bar_fin = bar_a + 4;                // teardown after an abort
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
     volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
 
@@ -148,39 +155,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = 16 * quad + (lane & 15);      // chunk row of this thread's tiles
     auto P = [&](int term) { return part + (term * 4 + cq) * 64; };
 
-    if (tid == 0) {
-        mbar_init(bar_ld0, 1);
-        mbar_init(bar_ld1, 1);
-        mbar_init(bar_mma, 1);
+    if (tid == kIss) {
+        for (int i = 0; i < kLoads + 5; ++i) mbar_init(bar_ld + i, 1);
         *s_abort = 0;
         fence_barrier_init();
         const int rowD = (bh * NC + c) * kD, rowC = (bh * NC + c) * kChunk;
-        // group 0: the operands of the first products
-        mbar_expect_tx(bar_ld0, 6 * kHalf + kTile + 256);
-        tma_load_4d(sm + L::Q, &tm_q, 0, h, t0, b, bar_ld0);
-        tma_load_4d(sm + L::Q + kHalf, &tm_q, 64, h, t0, b, bar_ld0);
-        tma_load_4d(sm + L::K, &tm_k, 0, h, t0, b, bar_ld0);
-        tma_load_4d(sm + L::K + kHalf, &tm_k, 64, h, t0, b, bar_ld0);
-        tma_load_4d(sm + L::dO, &tm_do, 0, h, t0, b, bar_ld0);
-        tma_load_4d(sm + L::dO + kHalf, &tm_do, 64, h, t0, b, bar_ld0);
-        tma_load_2d(sm + L::Dt, &tm_dt, 0, rowD, bar_ld0);
-        bulk_load(Gs, a.G + (size_t)bh * TP + t0, 256, bar_ld0);
-        // group 1: the state tiles, dDelta, T, W^T, U^T
-        mbar_expect_tx(bar_ld1, 7 * kTile + kHalf);
-        tma_load_2d(sm + L::dDt, &tm_ddt, 0, rowD, bar_ld1);
-        tma_load_2d(sm + L::St, &tm_sc, 0, rowD, bar_ld1);
-        tma_load_2d(sm + L::St + kTile, &tm_sc, 64, rowD, bar_ld1);
-        tma_load_2d(sm + L::dSt, &tm_dsc, 0, rowD, bar_ld1);
-        tma_load_2d(sm + L::dSt + kTile, &tm_dsc, 64, rowD, bar_ld1);
-        tma_load_2d(sm + L::Tb, &tm_t, 0, rowC, bar_ld1);
-        tma_load_2d(sm + L::Wt, &tm_wt, 0, rowD, bar_ld1);
-        tma_load_2d(sm + L::Ut, &tm_ut, 0, rowD, bar_ld1);
+        // 0: Q, K, G (Q K^T, K K^T)
+        mbar_expect_tx(&bar_ld[0], 4 * kHalf + 256);
+        tma_load_4d(sm + L::Q, &tm_q, 0, h, t0, b, &bar_ld[0]);
+        tma_load_4d(sm + L::Q + kHalf, &tm_q, 64, h, t0, b, &bar_ld[0]);
+        tma_load_4d(sm + L::K, &tm_k, 0, h, t0, b, &bar_ld[0]);
+        tma_load_4d(sm + L::K + kHalf, &tm_k, 64, h, t0, b, &bar_ld[0]);
+        bulk_load(Gs, a.G + (size_t)bh * TP + t0, 256, &bar_ld[0]);
+        // 1: dO, Delta^T (dO Delta^T)
+        mbar_expect_tx(&bar_ld[1], 2 * kHalf + kTile);
+        tma_load_4d(sm + L::dO, &tm_do, 0, h, t0, b, &bar_ld[1]);
+        tma_load_4d(sm + L::dO + kHalf, &tm_do, 64, h, t0, b, &bar_ld[1]);
+        tma_load_2d(sm + L::Dt, &tm_dt, 0, rowD, &bar_ld[1]);
+        // 2: S^T (dO S^T)
+        mbar_expect_tx(&bar_ld[2], 2 * kTile);
+        tma_load_2d(sm + L::St, &tm_sc, 0, rowD, &bar_ld[2]);
+        tma_load_2d(sm + L::St + kTile, &tm_sc, 64, rowD, &bar_ld[2]);
+        // 3: dS'^T (Delta dS'^T)
+        mbar_expect_tx(&bar_ld[3], 2 * kTile);
+        tma_load_2d(sm + L::dSt, &tm_dsc, 0, rowD, &bar_ld[3]);
+        tma_load_2d(sm + L::dSt + kTile, &tm_dsc, 64, rowD, &bar_ld[3]);
+        // 4: dDelta^T, T (dDelta S^T, T^T dDelta)
+        mbar_expect_tx(&bar_ld[4], kTile + kHalf);
+        tma_load_2d(sm + L::dDt, &tm_ddt, 0, rowD, &bar_ld[4]);
+        tma_load_2d(sm + L::Tb, &tm_t, 0, rowC, &bar_ld[4]);
+        // 5: W^T, U^T (third phase)
+        mbar_expect_tx(&bar_ld[5], 2 * kTile);
+        tma_load_2d(sm + L::Wt, &tm_wt, 0, rowD, &bar_ld[5]);
+        tma_load_2d(sm + L::Ut, &tm_ut, 0, rowD, &bar_ld[5]);
     }
     if (warp == 0) tmem_alloc(s_tmem, 512);
     if (tid < 64) Bs[tid] = (tid < Lr) ? a.beta[tok_index(a, b, t0 + tid, h)] : 0.f;
     // this thread's quarter of V's row r (lanes 16-31), read while the tiles load
     uint4 vpre[4] = {};
-    if (hi && r < Lr) {
+    if (warp < 16 && hi && r < Lr) {
         const uint4* src = (const uint4*)((const __nv_bfloat16*)a.v + tok_index(a, b, t0 + r, h) * kD + cq * 32);
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) vpre[qq] = __ldg(src + qq);
@@ -193,20 +206,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const uint32_t c0 = tmem, c64 = tmem + 64, c128 = tmem + 128, c256 = tmem + 256;
 
-    bool ld_pending = false, mma_pending = false;
+    bool ld_pending = false;
     uint32_t mph = 0;
-    auto mma_wait = [&]() {  // thread 0
+    auto mma_wait = [&]() {  // the issuer
         mma_commit(bar_mma);
         if (!mbar_wait(bar_mma, mph)) {
             *s_abort = 1;
-            mma_pending = true;
             atomicExch(a.err, kErrTimeoutMma);
+        }
+    };
+    // element-wise threads: a wait that gives up flags the abort, checked at the next barrier
+    auto wait_flag = [&](uint64_t* bar, int err) {
+        if (!mbar_wait(bar, 0)) {
+            *s_abort = 1;
+            atomicExch(a.err, err);
         }
     };
     float lastpart = 0.f;
 
-    // ---------------- phase A: every product of loaded operands
-    if (tid == 0) {
+    // ---------------- phase A: every product of loaded operands, committed in three groups
+    if (tid == kIss) {
         const uint32_t q = smem_u32(sm + L::Q), k = smem_u32(sm + L::K), dob = smem_u32(sm + L::dO);
         const uint32_t dt = smem_u32(sm + L::Dt), ddt = smem_u32(sm + L::dDt), tb = smem_u32(sm + L::Tb);
         const uint32_t st = smem_u32(sm + L::St), dst = smem_u32(sm + L::dSt);
@@ -215,47 +234,71 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t idKM2 = idesc_bf16(64, 128, false, true);
         constexpr uint32_t idMM2 = idesc_bf16(64, 128, true, true);
         constexpr uint32_t idMK2 = idesc_bf16(64, 128, true, false);
-        bool ok = mbar_wait(bar_ld0, 0);
+        // a group whose tiles did not land is skipped, its commit still issued so
+        // that no element-wise thread waits on it for long
+        bool ok = mbar_wait(&bar_ld[0], 0);
         if (ok) {
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
                 mma_bf16(c0, sdesc(q + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);  // Q K^T
-                mma_bf16(c0 + l16, sdesc(dob + o, 16, 1024), sdesc(dt + ks * 2048, kHalf, 1024), idKM,
-                         ks > 0);                                                             // dO Delta^T
                 mma_bf16(c64, sdesc(k + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);  // K K^T
             }
-            ok = mbar_wait(bar_ld1, 0);
+            ok = mbar_wait(&bar_ld[1], 0);
         }
         if (ok) {
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
-                const uint32_t m = ks * 2048;
-                mma_bf16(c128, sdesc(dob + o, 16, 1024), sdesc(st + m, kTile, 1024), idKM2, ks > 0);  // dO S^T
-                mma_bf16(c128 + l16, sdesc(dt + m, kHalf, 1024), sdesc(dst + m, kTile, 1024), idMM2,
-                         ks > 0);                                                              // Delta dS'^T
-                mma_bf16(c256, sdesc(ddt + m, kHalf, 1024), sdesc(st + m, kTile, 1024), idMM2,
-                         ks > 0);                                                              // dDelta S^T
+                mma_bf16(c0 + l16, sdesc(dob + o, 16, 1024), sdesc(dt + ks * 2048, kHalf, 1024), idKM,
+                         ks > 0);  // dO Delta^T
             }
+        }
+        mma_commit(&bar_a[0]);
+        if (ok) ok = mbar_wait(&bar_ld[2], 0);
+        if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
+                mma_bf16(c128, sdesc(dob + o, 16, 1024), sdesc(st + ks * 2048, kTile, 1024), idKM2,
+                         ks > 0);  // dO S^T
+            }
+            ok = mbar_wait(&bar_ld[3], 0);
+        }
+        if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(c128 + l16, sdesc(dt + ks * 2048, kHalf, 1024), sdesc(dst + ks * 2048, kTile, 1024),
+                         idMM2, ks > 0);  // Delta dS'^T
+        }
+        mma_commit(&bar_a[1]);
+        if (ok) ok = mbar_wait(&bar_ld[4], 0);
+        if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(c256, sdesc(ddt + ks * 2048, kHalf, 1024), sdesc(st + ks * 2048, kTile, 1024), idMM2,
+                         ks > 0);  // dDelta S^T
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(c256 + l16, sdesc(tb + ks * 2048, kHalf, 1024), sdesc(ddt + ks * 32, 16, 1024),
                          idMK2, ks > 0);  // T^T dDelta
-        } else {
+        }
+        mma_commit(&bar_a[2]);
+        if (!ok) {
             *s_abort = 1;
             ld_pending = true;
             atomicExch(a.err, kErrTimeoutTma);
         }
-        mma_wait();  // also drains the products issued before a load gave up
     }
-    mph ^= 1;
-    __syncthreads();
-    if (*s_abort) goto teardown;
-    tc_fence_after();
-    {
+    if (warp < 16) {
+        wait_flag(&bar_ld[0], kErrTimeoutTma);  // G, Q, K are read below
+        wait_flag(&bar_a[0], kErrTimeoutMma);
+        tc_fence_after();
         const float Gr = Gs[r];
         float rowpart;
         // (a) P, dP, F on columns [16 cq, 16 cq + 16): lane l < 16 holds (Q K^T)[r], lane
@@ -285,6 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // (b) dO S^T (lanes 0-15) / Delta dS'^T (lanes 16-31), columns [32 cq, 32 cq + 32),
         // rescaled in TMEM by gamma_r / e^{G_C - G_r}
+        wait_flag(&bar_a[1], kErrTimeoutMma);
+        tc_fence_after();
         {
             float x[32];
             tmem_ld32(c128 + lane_base + cq * 32, x);
@@ -304,6 +349,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(c128 + lane_base + cq * 32, x);
         }
         // (c) dW = -(dDelta S^T) (lanes 0-15) and dVhat (lanes 16-31)
+        wait_flag(&bar_a[2], kErrTimeoutMma);
+        tc_fence_after();
         {
             float x[32];
             tmem_ld32(c256 + lane_base + cq * 32, x);
@@ -336,6 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         // (d) <S, dS'> over the two identically laid out tiles; last-row sum
+        wait_flag(&bar_ld[2], kErrTimeoutTma);
+        wait_flag(&bar_ld[3], kErrTimeoutTma);
         {
             float acc = 0.f;
 #pragma unroll
@@ -365,9 +414,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (*s_abort) goto teardown;
 
     // ---------------- phase B: F K, F^T Q onto the rescaled partials; dKhat = T^T dW
-    if (tid == 0) {
+    if (tid == kIss) {
         tma_store_4d(&tm_dv, sm + L::dO, 0, h, t0, b);  // rows past the piece's end are clipped
         tma_store_4d(&tm_dv, sm + L::dO + kHalf, 64, h, t0, b);
         bulk_commit();
@@ -388,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (*s_abort) goto teardown;
     tc_fence_after();
-    {
+    if (warp < 16) {
         float x[32];
         tmem_ld32(c256 + lane_base + cq * 32, x);  // lanes 0-15: dKhat
         tmem_ld_wait();
@@ -409,28 +459,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
 
     // ---------------- phase C: dA = dKhat W^T + dVhat U^T
-    if (tid == 0) {
-        tc_fence_after();
-        const uint32_t dk = smem_u32(sm + L::St), dvb = smem_u32(sm + L::dDt);
-        const uint32_t wt = smem_u32(sm + L::Wt), ut = smem_u32(sm + L::Ut);
-        constexpr uint32_t id = idesc_bf16(64, 64, false, true);
+    if (tid == kIss) {
+        if (mbar_wait(&bar_ld[5], 0)) {  // W^T, U^T
+            tc_fence_after();
+            const uint32_t dk = smem_u32(sm + L::St), dvb = smem_u32(sm + L::dDt);
+            const uint32_t wt = smem_u32(sm + L::Wt), ut = smem_u32(sm + L::Ut);
+            constexpr uint32_t id = idesc_bf16(64, 64, false, true);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
-            mma_bf16(c0 + l16, sdesc(dk + o, 16, 1024), sdesc(wt + ks * 2048, kHalf, 1024), id, ks > 0);
-        }
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
+                mma_bf16(c0 + l16, sdesc(dk + o, 16, 1024), sdesc(wt + ks * 2048, kHalf, 1024), id, ks > 0);
+            }
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
-            mma_bf16(c0 + l16, sdesc(dvb + o, 16, 1024), sdesc(ut + ks * 2048, kHalf, 1024), id, 1);
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
+                mma_bf16(c0 + l16, sdesc(dvb + o, 16, 1024), sdesc(ut + ks * 2048, kHalf, 1024), id, 1);
+            }
+            mma_wait();
+        } else {
+            *s_abort = 1;
+            ld_pending = true;
+            atomicExch(a.err, kErrTimeoutTma);
         }
-        mma_wait();
     }
     mph ^= 1;
     __syncthreads();
     if (*s_abort) goto teardown;
     tc_fence_after();
-    {
+    if (warp < 16) {
         // B, dA, dB .* B (added onto PD), E on columns [16 cq, 16 cq + 16): lane l < 16
         // holds (K K^T)[r], lane l + 16 dA[r]; each finishes 8 columns as in (a)
         float va[16], vb[16];
@@ -464,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     __syncthreads();
-    {
+    if (warp < 16) {
         // E + E^T as a bf16 K-major tile [r][64 t] (in the F slot), and the column
         // sums of PD = dP .* P + dB .* B over 8-row groups
         const int rr = tid >> 3, cc = tid & 7;
@@ -486,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
 
     // ---------------- phase D: dKp = diag(beta gamma) dKhat + (E + E^T) K
-    if (tid == 0) {
+    if (tid == kIss) {
         tc_fence_after();
         const uint32_t f = smem_u32(sm + L::F), k = smem_u32(sm + L::K);
         constexpr uint32_t id = idesc_bf16(64, 128, false, true);
@@ -539,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             a.dbeta[tok_index(a, b, t0 + rr, h)] = db;
         }
     }
-    {
+    if (warp < 16) {
         // dq (lanes 0-15) and dk = dK + dKp (lanes 16-31), columns [32 cq, 32 cq + 32)
         float x[32], y[32];
         tmem_ld32(c128 + lane_base + cq * 32, x);
@@ -555,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_async_smem();
     __syncthreads();
-    if (tid == 0) {  // rows past the piece's end are clipped by the stores
+    if (tid == kIss) {  // rows past the piece's end are clipped by the stores
         tma_store_4d(&tm_dq, sm + L::Wt, 0, h, t0, b);
         tma_store_4d(&tm_dq, sm + L::Wt + kHalf, 64, h, t0, b);
         tma_store_4d(&tm_dk, sm + L::Ut, 0, h, t0, b);
@@ -564,13 +620,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
 teardown:
-    if (tid == 0) {
-        if (ld_pending) {
-            mbar_wait(bar_ld0, 0);
-            mbar_wait(bar_ld1, 0);
+    if (tid == kIss) {
+        if (ld_pending)
+            for (int i = 0; i < kLoads; ++i) mbar_wait(&bar_ld[i], 0);
+        if (*s_abort) {  // every UMMA issued has finished before the TMEM is freed
+            mma_commit(bar_fin);
+            mbar_wait(bar_fin, 0);
         }
-        if (mma_pending) mbar_wait(bar_mma, mph ^ 1);
-        bulk_wait<0>();  // the output stores have finished
+        bulk_wait_read<0>();  // the output stores have read shared memory
     }
     tc_fence_before();
     __syncthreads();
@@ -601,7 +658,7 @@ cudaError_t launch_grad_fused_tc(const Args& a, cudaStream_t s) {
                                          (int)smem);
     if (e != cudaSuccess) return e;
     timing_begin(KK_GRAD_FUSED, s);
-    grad_fused_tc_kernel<<<dim3(a.NC, BH), kThreads, smem, s>>>(tm_q, tm_k, tm_do, tm_wt, tm_ut, tm_t, tm_dt,
+    grad_fused_tc_kernel<<<dim3(a.NC, BH), kBlock, smem, s>>>(tm_q, tm_k, tm_do, tm_wt, tm_ut, tm_t, tm_dt,
                                                                 tm_ddt, tm_sc, tm_dsc, tm_dq, tm_dk, tm_dv, a);
     e = cudaGetLastError();
     timing_end(KK_GRAD_FUSED, s);

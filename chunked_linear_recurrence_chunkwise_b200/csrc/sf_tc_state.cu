@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int cc = c; cc < issued; ++cc) mbar_wait(&bar_ld[cc % kStages], (cc / kStages) & 1);
             if (mma_pending) mbar_wait(bar_mma, mma_phase ^ 1);
         }
-        bulk_wait<0>();
+        bulk_wait_read<0>();  // stores have read shared memory (their writes land before the grid completes)
     }
     tc_fence_before();
     __syncthreads();
@@ -552,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int m = n; m < issued; ++m) mbar_wait(&bar_ld[m % kBStages], (m / kBStages) & 1);
             if (mma_pending) mbar_wait(bar_mma, mma_phase ^ 1);
         }
-        bulk_wait<0>();
+        bulk_wait_read<0>();  // stores have read shared memory (their writes land before the grid completes)
     }
     tc_fence_before();
     __syncthreads();
