@@ -16,22 +16,25 @@
 //   dg = reverse in-chunk cumsum of dG
 // with T = (I + diag(beta) B)^-1 taken from the backward intra kernel.
 //
-// The UMMAs (all M = 64) run in four phases; every product that needs only
-// loaded data is issued in the first.  Accumulators are paired at TMEM lane
-// offsets 0 and 16 (rows 16 w + l of the lane-0 tile sit in lanes 32 w + l,
-// those of the lane-16 tile in lanes 32 w + 16 + l):
+// The UMMAs are all M = 64, their accumulators paired at TMEM lane offsets 0
+// and 16 (rows 16 w + l of the lane-0 tile sit in lanes 32 w + l, those of the
+// lane-16 tile in lanes 32 w + 16 + l):
 //   cols [0, 64):    Q K^T          | dO Delta^T, later dA
 //   cols [64, 128):  K K^T          | -
 //   cols [128, 256): dQ             | dK
 //   cols [256, 384): dW, dKhat, dKp | dVhat
-// Shared memory of operands that die after the first phase is reused for the
-// later tiles and scratch (about 218 KB in all, one CTA per SM).  Sixteen
-// warps share the element-wise work: warp w reads TMEM lane quadrant w % 4
-// and a quarter of the columns, w / 4.  A seventeenth warp issues the copies
-// and the UMMAs.  The operands arrive in six groups and the first phase's
-// products are committed in three, so that each product starts as soon as
-// its tiles have landed and the element-wise work on the first products
-// runs while the later ones are still on the tensor core.
+// Shared memory of operands that die early is reused for the later tiles and
+// scratch (about 218 KB in all, one CTA per SM).
+//
+// One thread of a seventeenth warp issues the copies and every UMMA, each as
+// soon as its operands are in place: the products of loaded tiles as their six
+// copy groups land (committed in three groups), F K and F^T Q once F is
+// written, T^T dW and dVhat U^T once dW and dVhat are, dKhat W^T once dKhat
+// is, (E + E^T) K once E is.  Sixteen warps share the element-wise work (warp
+// w reads TMEM lane quadrant w % 4 and a quarter of the columns, w / 4); they
+// hand each stage over through an mbarrier (one arrival per warp) and wait for
+// the products they read on the commit barriers, so that the tensor core and
+// the element-wise work of the chunk overlap.
 
 #include <cuda.h>
 
@@ -83,8 +86,8 @@ struct FusedSmem {
     static constexpr int csp = Bs + 256;          // fp32 [8][64]: column sums of PD over 8-row groups
     static constexpr int part = csp + 8 * 256;    // fp32 [P_COUNT][4][64]
     static constexpr int red = part + P_COUNT * 4 * 256;  // fp32 [32]: per-warp <S, dS'>, last-row sums
-    static constexpr int Bar = red + 128;         // kLoads load + 3 first-phase + 2 mbarriers
-    static constexpr int Misc = Bar + (kLoads + 5) * 8;
+    static constexpr int Bar = red + 128;         // kLoads + 11 mbarriers
+    static constexpr int Misc = Bar + (kLoads + 11) * 8;
     static constexpr int Size = Misc + 16;
 };
 
@@ -139,10 +142,11 @@ __global__ void __launch_bounds__(kBlock, 1)
     float* Ef = (float*)(sm + L::dSt);
     float* part = (float*)(sm + L::part);
     float* red = (float*)(sm + L::red);
-    uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);  // [kLoads]
-    uint64_t* bar_a = bar_ld + kLoads;            // first-phase products, three groups
-    uint64_t* bar_mma = bar_a + 3;                // later phases
-    uint64_t* bar_fin = bar_a + 4;                // teardown after an abort
+    uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);  // [kLoads] operand groups landed
+    uint64_t* bar_a = bar_ld + kLoads;            // [3] products of loaded tiles done
+    uint64_t* bar_c = bar_a + 3;                  // [3] later products done
+    uint64_t* bar_s = bar_c + 3;                  // [4] element-wise stages handed over (16 warps)
+    uint64_t* bar_fin = bar_s + 4;                // teardown after an abort
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
     volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
 
@@ -156,7 +160,7 @@ __global__ void __launch_bounds__(kBlock, 1)
     auto P = [&](int term) { return part + (term * 4 + cq) * 64; };
 
     if (tid == kIss) {
-        for (int i = 0; i < kLoads + 5; ++i) mbar_init(bar_ld + i, 1);
+        for (int i = 0; i < kLoads + 11; ++i) mbar_init(bar_ld + i, (i >= kLoads + 6 && i < kLoads + 10) ? 16 : 1);
         *s_abort = 0;
         fence_barrier_init();
         const int rowD = (bh * NC + c) * kD, rowC = (bh * NC + c) * kChunk;
@@ -184,7 +188,7 @@ __global__ void __launch_bounds__(kBlock, 1)
         mbar_expect_tx(&bar_ld[4], kTile + kHalf);
         tma_load_2d(sm + L::dDt, &tm_ddt, 0, rowD, &bar_ld[4]);
         tma_load_2d(sm + L::Tb, &tm_t, 0, rowC, &bar_ld[4]);
-        // 5: W^T, U^T (third phase)
+        // 5: W^T, U^T (dVhat U^T, dKhat W^T)
         mbar_expect_tx(&bar_ld[5], 2 * kTile);
         tma_load_2d(sm + L::Wt, &tm_wt, 0, rowD, &bar_ld[5]);
         tma_load_2d(sm + L::Ut, &tm_ut, 0, rowD, &bar_ld[5]);
@@ -206,25 +210,26 @@ __global__ void __launch_bounds__(kBlock, 1)
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const uint32_t c0 = tmem, c64 = tmem + 64, c128 = tmem + 128, c256 = tmem + 256;
 
-    bool ld_pending = false;
-    uint32_t mph = 0;
-    auto mma_wait = [&]() {  // the issuer
-        mma_commit(bar_mma);
-        if (!mbar_wait(bar_mma, mph)) {
-            *s_abort = 1;
-            atomicExch(a.err, kErrTimeoutMma);
-        }
-    };
-    // element-wise threads: a wait that gives up flags the abort, checked at the next barrier
+    // Element-wise warps: a wait that gives up flags the abort (checked before the
+    // final stores); every warp passes every barrier whatever happened, so that no
+    // wait of another thread runs to its limit.
     auto wait_flag = [&](uint64_t* bar, int err) {
         if (!mbar_wait(bar, 0)) {
             *s_abort = 1;
             atomicExch(a.err, err);
         }
     };
+    // Element-wise warps hand their shared- and tensor-memory writes to the issuer.
+    auto hand_over = [&](uint64_t* bar) {
+        tmem_st_wait();
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar);
+    };
     float lastpart = 0.f;
 
-    // ---------------- phase A: every product of loaded operands, committed in three groups
+    // ---------------- the issuer: every UMMA, each as soon as its operands are ready
     if (tid == kIss) {
         const uint32_t q = smem_u32(sm + L::Q), k = smem_u32(sm + L::K), dob = smem_u32(sm + L::dO);
         const uint32_t dt = smem_u32(sm + L::Dt), ddt = smem_u32(sm + L::dDt), tb = smem_u32(sm + L::Tb);
@@ -289,13 +294,72 @@ __global__ void __launch_bounds__(kBlock, 1)
                          idMK2, ks > 0);  // T^T dDelta
         }
         mma_commit(&bar_a[2]);
-        if (!ok) {
-            *s_abort = 1;
-            ld_pending = true;
-            atomicExch(a.err, kErrTimeoutTma);
+        // F K and F^T Q accumulate onto the rescaled dO S^T / Delta dS'^T once the
+        // element-wise warps have written F and rescaled those ((a), (b))
+        bool sok = ok && mbar_wait(&bar_s[0], 0);
+        if (sok) {
+            tc_fence_after();
+            const uint32_t f = smem_u32(sm + L::F);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                mma_bf16(c128, sdesc(f + ks * 32, 16, 1024), sdesc(k + ks * 2048, kHalf, 1024), idKM2, 1);
+                mma_bf16(c128 + l16, sdesc(f + ks * 2048, kHalf, 1024), sdesc(q + ks * 2048, kHalf, 1024),
+                         idMM2, 1);
+            }
         }
-    }
-    if (warp < 16) {
+        // dv is staged, dW and dVhat are written ((c), (d)): dKhat = T^T dW, then dVhat U^T
+        sok = sok && mbar_wait(&bar_s[1], 0);
+        if (sok) {
+            tma_store_4d(&tm_dv, sm + L::dO, 0, h, t0, b);  // rows past the piece's end are clipped
+            tma_store_4d(&tm_dv, sm + L::dO + kHalf, 64, h, t0, b);
+            bulk_commit();
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(c256, sdesc(tb + ks * 2048, kHalf, 1024), sdesc(dt + ks * 2048, kHalf, 1024), idMM2,
+                         ks > 0);
+        }
+        mma_commit(&bar_c[0]);
+        const bool sok_pre5 = sok;
+        const bool ok5 = sok && mbar_wait(&bar_ld[5], 0);  // W^T, U^T
+        if (ok5) {
+            tc_fence_after();
+            const uint32_t ut = smem_u32(sm + L::Ut);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
+                mma_bf16(c0 + l16, sdesc(ddt + o, 16, 1024), sdesc(ut + ks * 2048, kHalf, 1024), idKM,
+                         ks > 0);  // dVhat U^T
+            }
+        }
+        // dA += dKhat W^T once dKhat is written (second element-wise stage)
+        sok = ok5 && mbar_wait(&bar_s[2], 0);
+        if (sok) {
+            tc_fence_after();
+            const uint32_t wt = smem_u32(sm + L::Wt);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
+                mma_bf16(c0 + l16, sdesc(st + o, 16, 1024), sdesc(wt + ks * 2048, kHalf, 1024), idKM, 1);
+            }
+        }
+        mma_commit(&bar_c[1]);
+        // dKp = diag(beta gamma) dKhat + (E + E^T) K once E + E^T is written
+        sok = sok && mbar_wait(&bar_s[3], 0);
+        if (sok) {
+            tc_fence_after();
+            const uint32_t f = smem_u32(sm + L::F);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(c256, sdesc(f + ks * 32, 16, 1024), sdesc(k + ks * 2048, kHalf, 1024), idKM2, 1);
+        }
+        mma_commit(&bar_c[2]);
+        if (!sok) {  // a copy or an element-wise stage did not arrive in time
+            *s_abort = 1;
+            atomicExch(a.err, (!ok || (sok_pre5 && !ok5)) ? kErrTimeoutTma : kErrTimeoutMma);
+        }
+    } else if (warp < 16) {
+        // ---------------- the element-wise warps
         wait_flag(&bar_ld[0], kErrTimeoutTma);  // G, Q, K are read below
         wait_flag(&bar_a[0], kErrTimeoutMma);
         tc_fence_after();
@@ -348,6 +412,7 @@ __global__ void __launch_bounds__(kBlock, 1)
             for (int q = 0; q < 32; ++q) x[q] *= scale;
             tmem_st32(c128 + lane_base + cq * 32, x);
         }
+        hand_over(&bar_s[0]);
         // (c) dW = -(dDelta S^T) (lanes 0-15) and dVhat (lanes 16-31)
         wait_flag(&bar_a[2], kErrTimeoutMma);
         tc_fence_after();
@@ -374,15 +439,14 @@ __global__ void __launch_bounds__(kBlock, 1)
                         ow[p] = pack_bf16(br * x[qq * 8 + 2 * p], br * x[qq * 8 + 2 * p + 1]);
                     }
                 }
-                // dv row r into the dO tile (dead after phase A) for one TMA store
+                // dv row r into the dO tile (its products are done) for one TMA store
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq)
                     *(uint4*)(sm + L::dO + (cq >> 1) * kHalf + sw128(r, (cq & 1) * 4 + qq)) = ov[qq];
                 P(P_VD)[r] = vd;
                 put_row(sm + L::dDt + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);  // K-major A of dA
             }
-        }
-        // (d) <S, dS'> over the two identically laid out tiles; last-row sum
+        }        // (d) <S, dS'> over the two identically laid out tiles; last-row sum
         wait_flag(&bar_ld[2], kErrTimeoutTma);
         wait_flag(&bar_ld[3], kErrTimeoutTma);
         {
@@ -409,221 +473,151 @@ __global__ void __launch_bounds__(kBlock, 1)
                 red[16 + warp] = lastpart;
             }
         }
-    }
-    tmem_st_wait();
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (*s_abort) goto teardown;
-
-    // ---------------- phase B: F K, F^T Q onto the rescaled partials; dKhat = T^T dW
-    if (tid == kIss) {
-        tma_store_4d(&tm_dv, sm + L::dO, 0, h, t0, b);  // rows past the piece's end are clipped
-        tma_store_4d(&tm_dv, sm + L::dO + kHalf, 64, h, t0, b);
-        bulk_commit();
+        hand_over(&bar_s[1]);
+        // dKhat: dG and dbeta terms, the K-major A operand of dKhat W^T, and
+        // diag(beta gamma) dKhat as the start of dKp
+        wait_flag(&bar_c[0], kErrTimeoutMma);
         tc_fence_after();
-        const uint32_t f = smem_u32(sm + L::F), k = smem_u32(sm + L::K), q = smem_u32(sm + L::Q);
-        const uint32_t tb = smem_u32(sm + L::Tb), dw = smem_u32(sm + L::Dt);
-        constexpr uint32_t idKM2 = idesc_bf16(64, 128, false, true);
-        constexpr uint32_t idMM2 = idesc_bf16(64, 128, true, true);
+        {
+            float x[32];
+            tmem_ld32(c256 + lane_base + cq * 32, x);  // lanes 0-15: dKhat
+            tmem_ld_wait();
+            if (!hi) {
+                const float gam = __expf(Gs[r]), br = Bs[r];
+                const float kd = dot_row32(sm + L::K + (cq >> 1) * kHalf, r, (cq & 1) * 4, x);
+                P(P_GK)[r] = gam * kd;
+                P(P_BGK)[r] = br * gam * kd;
+                put_row(sm + L::St + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);  // K-major A of dA
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            mma_bf16(c256, sdesc(tb + ks * 2048, kHalf, 1024), sdesc(dw + ks * 2048, kHalf, 1024), idMM2, ks > 0);
-            mma_bf16(c128, sdesc(f + ks * 32, 16, 1024), sdesc(k + ks * 2048, kHalf, 1024), idKM2, 1);
-            mma_bf16(c128 + l16, sdesc(f + ks * 2048, kHalf, 1024), sdesc(q + ks * 2048, kHalf, 1024), idMM2, 1);
-        }
-        mma_wait();
-    }
-    mph ^= 1;
-    __syncthreads();
-    if (*s_abort) goto teardown;
-    tc_fence_after();
-    if (warp < 16) {
-        float x[32];
-        tmem_ld32(c256 + lane_base + cq * 32, x);  // lanes 0-15: dKhat
-        tmem_ld_wait();
-        if (!hi) {
-            const float gam = __expf(Gs[r]), br = Bs[r];
-            const float kd = dot_row32(sm + L::K + (cq >> 1) * kHalf, r, (cq & 1) * 4, x);
-            P(P_GK)[r] = gam * kd;
-            P(P_BGK)[r] = br * gam * kd;
-            put_row(sm + L::St + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);  // K-major A of dA
-#pragma unroll
-            for (int q = 0; q < 32; ++q) x[q] *= br * gam;
-        }
-        tmem_st32(c256 + lane_base + cq * 32, x);
-    }
-    tmem_st_wait();
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---------------- phase C: dA = dKhat W^T + dVhat U^T
-    if (tid == kIss) {
-        if (mbar_wait(&bar_ld[5], 0)) {  // W^T, U^T
-            tc_fence_after();
-            const uint32_t dk = smem_u32(sm + L::St), dvb = smem_u32(sm + L::dDt);
-            const uint32_t wt = smem_u32(sm + L::Wt), ut = smem_u32(sm + L::Ut);
-            constexpr uint32_t id = idesc_bf16(64, 64, false, true);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
-                mma_bf16(c0 + l16, sdesc(dk + o, 16, 1024), sdesc(wt + ks * 2048, kHalf, 1024), id, ks > 0);
+                for (int q = 0; q < 32; ++q) x[q] *= br * gam;
             }
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
-                mma_bf16(c0 + l16, sdesc(dvb + o, 16, 1024), sdesc(ut + ks * 2048, kHalf, 1024), id, 1);
-            }
-            mma_wait();
-        } else {
-            *s_abort = 1;
-            ld_pending = true;
-            atomicExch(a.err, kErrTimeoutTma);
+            tmem_st32(c256 + lane_base + cq * 32, x);
         }
-    }
-    mph ^= 1;
-    __syncthreads();
-    if (*s_abort) goto teardown;
-    tc_fence_after();
-    if (warp < 16) {
-        // B, dA, dB .* B (added onto PD), E on columns [16 cq, 16 cq + 16): lane l < 16
-        // holds (K K^T)[r], lane l + 16 dA[r]; each finishes 8 columns as in (a)
-        float va[16], vb[16];
-        tmem_ld16(c0 + lane_base + cq * 16, va);   // lanes 16-31: dA (before the sign)
-        tmem_ld16(c64 + lane_base + cq * 16, vb);  // lanes 0-15: K K^T
-        tmem_ld_wait();
-        const int tb = 16 * cq + (hi ? 8 : 0);
-        const float Gr = Gs[r], br = Bs[r];
-        float sab = 0.f, sbb = 0.f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const float recv = __shfl_xor_sync(0xffffffffu, hi ? va[q] : vb[8 + q], 16);
-            const float kk = hi ? recv : vb[q];
-            const float dar = hi ? va[8 + q] : recv;
-            const int t = tb + q;
-            const bool lower = t < r;
-            const float gam = lower ? __expf(Gr - Gs[t]) : 0.f;
-            const float bv = gam * kk;
-            const float da = lower ? -dar : 0.f;
-            sab += da * bv;
-            const float dbb = br * da * bv;
-            sbb += dbb;
-            PD[r * 65 + t] += dbb;  // the same thread wrote dP .* P here in (a)
-            Ef[r * 65 + t] = br * da * gam;
-        }
-        sab += __shfl_xor_sync(0xffffffffu, sab, 16);
-        sbb += __shfl_xor_sync(0xffffffffu, sbb, 16);
-        if (!hi) {
-            P(P_SAB)[r] = sab;
-            P(P_SBB)[r] = sbb;
-        }
-    }
-    __syncthreads();
-    if (warp < 16) {
-        // E + E^T as a bf16 K-major tile [r][64 t] (in the F slot), and the column
-        // sums of PD = dP .* P + dB .* B over 8-row groups
-        const int rr = tid >> 3, cc = tid & 7;
-        float e[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int t = cc * 8 + i;
-            e[i] = Ef[rr * 65 + t] + Ef[t * 65 + rr];
-        }
-        put_row(sm + L::F, rr, cc, e, 8);
-        const int col = tid & 63, g = tid >> 6;
-        float s = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) s += PD[(8 * g + i) * 65 + col];
-        csp[g * 64 + col] = s;
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---------------- phase D: dKp = diag(beta gamma) dKhat + (E + E^T) K
-    if (tid == kIss) {
+        hand_over(&bar_s[2]);
+        wait_flag(&bar_c[1], kErrTimeoutMma);
         tc_fence_after();
-        const uint32_t f = smem_u32(sm + L::F), k = smem_u32(sm + L::K);
-        constexpr uint32_t id = idesc_bf16(64, 128, false, true);
+        {
+            // B, dA, dB .* B (added onto PD), E on columns [16 cq, 16 cq + 16): lane l < 16
+            // holds (K K^T)[r], lane l + 16 dA[r]; each finishes 8 columns as in (a)
+            float va[16], vb[16];
+            tmem_ld16(c0 + lane_base + cq * 16, va);   // lanes 16-31: dA (before the sign)
+            tmem_ld16(c64 + lane_base + cq * 16, vb);  // lanes 0-15: K K^T
+            tmem_ld_wait();
+            const int tb = 16 * cq + (hi ? 8 : 0);
+            const float Gr = Gs[r], br = Bs[r];
+            float sab = 0.f, sbb = 0.f;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-            mma_bf16(c256, sdesc(f + ks * 32, 16, 1024), sdesc(k + ks * 2048, kHalf, 1024), id, 1);
-        mma_wait();
+            for (int q = 0; q < 8; ++q) {
+                const float recv = __shfl_xor_sync(0xffffffffu, hi ? va[q] : vb[8 + q], 16);
+                const float kk = hi ? recv : vb[q];
+                const float dar = hi ? va[8 + q] : recv;
+                const int t = tb + q;
+                const bool lower = t < r;
+                const float gam = lower ? __expf(Gr - Gs[t]) : 0.f;
+                const float bv = gam * kk;
+                const float da = lower ? -dar : 0.f;
+                sab += da * bv;
+                const float dbb = br * da * bv;
+                sbb += dbb;
+                PD[r * 65 + t] += dbb;  // the same thread wrote dP .* P here in (a)
+                Ef[r * 65 + t] = br * da * gam;
+            }
+            sab += __shfl_xor_sync(0xffffffffu, sab, 16);
+            sbb += __shfl_xor_sync(0xffffffffu, sbb, 16);
+            if (!hi) {
+                P(P_SAB)[r] = sab;
+                P(P_SBB)[r] = sbb;
+            }
+        }
+        named_sync(1, kThreads);  // PD and E of every row
+        {
+            // E + E^T as a bf16 K-major tile [r][64 t] (in the F slot), and the column
+            // sums of PD = dP .* P + dB .* B over 8-row groups
+            const int rr = tid >> 3, cc = tid & 7;
+            float e[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int t = cc * 8 + i;
+                e[i] = Ef[rr * 65 + t] + Ef[t * 65 + rr];
+            }
+            put_row(sm + L::F, rr, cc, e, 8);
+            const int col = tid & 63, g = tid >> 6;
+            float s = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) s += PD[(8 * g + i) * 65 + col];
+            csp[g * 64 + col] = s;
+        }
+        hand_over(&bar_s[3]);
+        wait_flag(&bar_c[2], kErrTimeoutMma);
+        tc_fence_after();
+        named_sync(1, kThreads);  // the per-row partial sums of every warp
+        // ---------------- epilogue
+        if (warp == 0) {  // dG and dg = reverse in-chunk cumsum
+            float sdot = 0.f, last = 0.f;
+#pragma unroll
+            for (int w = 0; w < 16; ++w) {
+                sdot += red[w];
+                last += red[16 + w];
+            }
+            float v2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int rr = 2 * lane + e;
+                float g = 0.f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) g -= csp[i * 64 + rr];
+#pragma unroll
+                for (int pi = 0; pi < kDgTerms * 4; ++pi) g += part[pi * 64 + rr];
+                if (rr == kChunk - 1) g += last + __expf(Gs[kChunk - 1]) * sdot;
+                v2[e] = g;
+            }
+            float incl = v2[0] + v2[1];
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_down_sync(0xffffffffu, incl, off);
+                if (lane + off < 32) incl += y;
+            }
+            if (a.g) {
+                if (2 * lane < Lr) a.dg[tok_index(a, b, t0 + 2 * lane, h)] = incl;
+                if (2 * lane + 1 < Lr) a.dg[tok_index(a, b, t0 + 2 * lane + 1, h)] = incl - v2[0];
+            }
+        } else if (warp == 1 || warp == 2) {  // dbeta
+            const int rr = tid - 32;
+            if (rr < Lr) {
+                float db = 0.f;
+#pragma unroll
+                for (int pi = kDgTerms * 4; pi < P_COUNT * 4; ++pi) db += part[pi * 64 + rr];
+                a.dbeta[tok_index(a, b, t0 + rr, h)] = db;
+            }
+        }
+        if (warp < 16) {
+            // dq (lanes 0-15) and dk = dK + dKp (lanes 16-31), columns [32 cq, 32 cq + 32)
+            float x[32], y[32];
+            tmem_ld32(c128 + lane_base + cq * 32, x);
+            tmem_ld32(c256 + lane_base + cq * 32, y);  // lanes 0-15: dKp
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                const float kp = __shfl_xor_sync(0xffffffffu, y[q], 16);
+                if (hi) x[q] += kp;
+            }
+            // dq rows into the W^T tile, dk rows into the U^T tile (both read by now)
+            put_row(sm + (hi ? L::Ut : L::Wt) + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);
+        }
+        fence_async_smem();
     }
-    mph ^= 1;
     __syncthreads();
-    if (*s_abort) goto teardown;
-    tc_fence_after();
-
-    // ---------------- epilogue
-    if (warp == 0) {  // dG and dg = reverse in-chunk cumsum
-        float sdot = 0.f, last = 0.f;
-#pragma unroll
-        for (int w = 0; w < 16; ++w) {
-            sdot += red[w];
-            last += red[16 + w];
-        }
-        float v2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int rr = 2 * lane + e;
-            float g = 0.f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) g -= csp[i * 64 + rr];
-#pragma unroll
-            for (int pi = 0; pi < kDgTerms * 4; ++pi) g += part[pi * 64 + rr];
-            if (rr == kChunk - 1) g += last + __expf(Gs[kChunk - 1]) * sdot;
-            v2[e] = g;
-        }
-        float incl = v2[0] + v2[1];
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const float y = __shfl_down_sync(0xffffffffu, incl, off);
-            if (lane + off < 32) incl += y;
-        }
-        if (a.g) {
-            if (2 * lane < Lr) a.dg[tok_index(a, b, t0 + 2 * lane, h)] = incl;
-            if (2 * lane + 1 < Lr) a.dg[tok_index(a, b, t0 + 2 * lane + 1, h)] = incl - v2[0];
-        }
-    } else if (warp == 1 || warp == 2) {  // dbeta
-        const int rr = tid - 32;
-        if (rr < Lr) {
-            float db = 0.f;
-#pragma unroll
-            for (int pi = kDgTerms * 4; pi < P_COUNT * 4; ++pi) db += part[pi * 64 + rr];
-            a.dbeta[tok_index(a, b, t0 + rr, h)] = db;
-        }
-    }
-    if (warp < 16) {
-        // dq (lanes 0-15) and dk = dK + dKp (lanes 16-31), columns [32 cq, 32 cq + 32)
-        float x[32], y[32];
-        tmem_ld32(c128 + lane_base + cq * 32, x);
-        tmem_ld32(c256 + lane_base + cq * 32, y);  // lanes 0-15: dKp
-        tmem_ld_wait();
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-            const float kp = __shfl_xor_sync(0xffffffffu, y[q], 16);
-            if (hi) x[q] += kp;
-        }
-        // dq rows into the W^T tile, dk rows into the U^T tile (both dead after phase C)
-        put_row(sm + (hi ? L::Ut : L::Wt) + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);
-    }
-    fence_async_smem();
-    __syncthreads();
-    if (tid == kIss) {  // rows past the piece's end are clipped by the stores
+    if (tid == kIss && !*s_abort) {  // rows past the piece's end are clipped by the stores
         tma_store_4d(&tm_dq, sm + L::Wt, 0, h, t0, b);
         tma_store_4d(&tm_dq, sm + L::Wt + kHalf, 64, h, t0, b);
         tma_store_4d(&tm_dk, sm + L::Ut, 0, h, t0, b);
         tma_store_4d(&tm_dk, sm + L::Ut + kHalf, 64, h, t0, b);
         bulk_commit();
     }
-
-teardown:
     if (tid == kIss) {
-        if (ld_pending)
+        if (*s_abort) {  // copies still in flight land, and every UMMA issued has
+                         // finished, before the CTA exits and frees the TMEM
             for (int i = 0; i < kLoads; ++i) mbar_wait(&bar_ld[i], 0);
-        if (*s_abort) {  // every UMMA issued has finished before the TMEM is freed
             mma_commit(bar_fin);
             mbar_wait(bar_fin, 0);
         }
