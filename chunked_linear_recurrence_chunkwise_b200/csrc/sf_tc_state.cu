@@ -65,23 +65,26 @@ constexpr int kD = 128;                 // d_k = d_v on this path
 constexpr int kTile = 128 * 64 * 2;     // one 128-row x 128-byte bf16 tile (16 KB)
 constexpr int kStages = 3;
 
-// Thread layout of both passes: 512 threads = 16 warps; warp w reads TMEM lane
+// Thread layout of both passes: 16 element-wise warps; warp w reads TMEM lane
 // quadrant (w & 3), i.e. d_v rows j = 32 (w & 3) + lane, and owns the column
 // quarter p = w >> 2 of every per-row tile (16 of 64 token columns, 32 of 128
 // state columns), so each step's elementwise work is split four ways per row.
 constexpr int kThreads = 512;
+// The forward pass adds a seventeenth warp whose first thread issues the
+// copies, the UMMAs and the stores.
+constexpr int kFwdThreads = kThreads + 32;
+constexpr int kFwdIss = kThreads;
 
 // Shared-memory carve-up (byte offsets from a 1024-byte aligned base).
 struct FwdSmem {
     static constexpr int Wt = 0;                          // [stage] W^T  [d_k][64 r]
     static constexpr int Kt = Wt + kStages * kTile;       // [stage] K    [2][64 r][64 d_k]
     static constexpr int Ut = Kt + kStages * kTile;       // [stage] U^T  [d_v][64 r]
-    static constexpr int St = Ut + kStages * kTile;       // S^T operand [2 kblk][d_v][64]
-    static constexpr int Dsc = St + 2 * kTile;            // (e^{G_C-G} Delta)^T operand
-    static constexpr int Dst = Dsc + kTile;               // Delta^T staging for the store
+    static constexpr int St = Ut + kStages * kTile;       // S^T staging for its store [2 kblk][d_v][64]
+    static constexpr int Dst = St + 2 * kTile;            // Delta^T staging for its store
     static constexpr int Ed = Dst + kTile;                // [stage][128] fp32 decay table
-    static constexpr int Bar = Ed + kStages * 512;        // kStages load barriers + 1 MMA
-    static constexpr int Misc = Bar + (kStages + 1) * 8;  // TMEM base, abort flag
+    static constexpr int Bar = Ed + kStages * 512;        // barriers, see the kernel
+    static constexpr int Misc = Bar + (kStages + 10) * 8;  // TMEM base, abort flag
     static constexpr int Size = Misc + 16;
 };
 
@@ -98,8 +101,21 @@ __device__ __forceinline__ void put_row32(uint8_t* tile, int row, int q0, const 
     }
 }
 
+// Forward state pass.  Both per-chunk products take their A operand from tensor
+// memory, where the element-wise warps put it as bf16 pairs: S^T (entering the
+// chunk) for X^T = S^T W^T, and (e^{G_C - G} Delta)^T for P^T = ... K.  The
+// dependent chain of a chunk is therefore UMMA -> TMEM -> registers -> TMEM ->
+// UMMA; the bf16 copies of S^T and Delta^T that go to global memory are staged
+// in shared memory and stored by TMA off that chain, while the next product
+// runs.  The warps hand over through mbarriers (one arrival per warp):
+//   bar_s    S^T of chunk c in TMEM            bar_x  X^T of chunk c done (commit)
+//   bar_d    scaled Delta^T in TMEM            bar_p  P^T of chunk c done (commit)
+//   bar_sst  S^T staged for its store          bar_sfree  that store has read the tile
+//   bar_dst  Delta^T staged for its store      bar_dfree  that store has read the tile
+// TMEM (512 columns): X^T [0, 64), P^T [64, 192), S^T operand [192, 256),
+// Delta^T operand [256, 288).
 template <bool kDelta>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     state_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_wt,
                         const __grid_constant__ CUtensorMap tm_ut,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -109,8 +125,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     float* Eds = (float*)(sm + L::Ed);
-    uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);
-    uint64_t* bar_mma = bar_ld + kStages;
+    uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);  // [kStages], count 1
+    uint64_t* bar_x = bar_ld + kStages;           // count 1 (commits)
+    uint64_t* bar_p = bar_x + 1;
+    uint64_t* bar_s = bar_x + 2;                  // count 16 (one arrival per element-wise warp)
+    uint64_t* bar_d = bar_x + 3;
+    uint64_t* bar_sst = bar_x + 4;
+    uint64_t* bar_dst = bar_x + 5;
+    uint64_t* bar_sfree = bar_x + 6;              // count 1 (the issuer)
+    uint64_t* bar_dfree = bar_x + 7;
+    uint64_t* bar_fin = bar_x + 8;
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
     volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
 
@@ -120,148 +144,189 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
     const int NC = a.NC;
 
-    if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&bar_ld[s], 1);
-        mbar_init(bar_mma, 1);
+    if (tid == kFwdIss) {
+        for (int i = 0; i < kStages + 9; ++i) {
+            const int k = i - kStages;  // 2..5: the element-wise hand-overs
+            mbar_init(bar_ld + i, (k >= 2 && k <= 5) ? 16 : 1);
+        }
         *s_abort = 0;
         fence_barrier_init();
     }
-    if (warp == 0) tmem_alloc(s_tmem, 256);
+    if (warp == 0) tmem_alloc(s_tmem, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    const uint32_t tX = tmem, tP = tmem + 64;
+    const uint32_t tX = tmem, tP = tmem + 64, tS = tmem + 192, tD = tmem + 256;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
 
-    auto issue_load = [&](int c) {  // thread 0
-        const int s = c % kStages;
-        const uint32_t bytes = (kDelta ? kTile : 0) + 2 * kTile + 512;
-        mbar_expect_tx(&bar_ld[s], bytes);
-        if (kDelta) tma_load_2d(sm + L::Wt + s * kTile, &tm_wt, 0, (bh * NC + c) * kD, &bar_ld[s]);
-        tma_load_2d(sm + L::Ut + s * kTile, &tm_ut, 0, (bh * NC + c) * kD, &bar_ld[s]);
-        tma_load_4d(sm + L::Kt + s * kTile, &tm_k, 0, h, c * kChunk, b, &bar_ld[s]);
-        tma_load_4d(sm + L::Kt + s * kTile + kTile / 2, &tm_k, 64, h, c * kChunk, b, &bar_ld[s]);
-        bulk_load(Eds + s * 128, a.Ed + ((size_t)bh * NC + c) * 128, 512, &bar_ld[s]);
-    };
-    int issued = 0;
-    if (tid == 0)
+    if (tid == kFwdIss) {
+        // ---------------- the issuer
+        auto issue_load = [&](int c) {
+            const int s = c % kStages;
+            const uint32_t bytes = (kDelta ? kTile : 0) + 2 * kTile + 512;
+            mbar_expect_tx(&bar_ld[s], bytes);
+            if (kDelta) tma_load_2d(sm + L::Wt + s * kTile, &tm_wt, 0, (bh * NC + c) * kD, &bar_ld[s]);
+            tma_load_2d(sm + L::Ut + s * kTile, &tm_ut, 0, (bh * NC + c) * kD, &bar_ld[s]);
+            tma_load_4d(sm + L::Kt + s * kTile, &tm_k, 0, h, c * kChunk, b, &bar_ld[s]);
+            tma_load_4d(sm + L::Kt + s * kTile + kTile / 2, &tm_k, 64, h, c * kChunk, b, &bar_ld[s]);
+            bulk_load(Eds + s * 128, a.Ed + ((size_t)bh * NC + c) * 128, 512, &bar_ld[s]);
+        };
+        int issued = 0;
         for (; issued < min(kStages, NC); ++issued) issue_load(issued);
-
-    // S^T row j, state columns i in [32 part, 32 part + 32): S[q] = S_{i, j}
-    float S[32];
-#pragma unroll
-    for (int q = 0; q < 32; ++q)
-        S[q] = a.S_in ? a.S_in[((size_t)bh * kD + part * 32 + q) * kD + j] : 0.f;
-    uint8_t* St = sm + L::St + (part >> 1) * kTile;
-    const int sq0 = (part & 1) * 4;  // first 16-byte chunk of this thread's 32 state columns
-    put_row32(St, j, sq0, S);
-    fence_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-        tma_store_2d(&tm_sc, sm + L::St, 0, bh * NC * kD);
-        tma_store_2d(&tm_sc, sm + L::St + kTile, 64, bh * NC * kD);
-        bulk_commit();
-    }
-
-    uint32_t mma_phase = 0;
-    bool mma_pending = false;  // thread 0: an MMA commit whose wait timed out
-    int c = 0;
-    bool aborted = false;
-    for (; c < NC; ++c) {
-        const int s = c % kStages;
-        if (tid == 0) {
-            if (!mbar_wait(&bar_ld[s], (c / kStages) & 1)) {
+        bool ok = true;
+        int err = 0;
+        auto wait = [&](uint64_t* bar, uint32_t parity, int e) {
+            if (ok && !mbar_wait_or_abort(bar, parity, s_abort)) {
+                ok = false;
+                err = e;
                 *s_abort = 1;
-                atomicExch(a.err, kErrTimeoutTma);
-            } else if (kDelta) {
+            }
+        };
+        for (int c = 0; c < NC; ++c) {
+            const int s = c % kStages;
+            const uint32_t par = c & 1;
+            wait(&bar_ld[s], (c / kStages) & 1, kErrTimeoutTma);
+            wait(bar_s, par, kErrTimeoutMma);  // S^T entering chunk c is in TMEM
+            if (ok && kDelta) {
                 tc_fence_after();
-                const uint32_t a0 = smem_u32(sm + L::St), b0 = smem_u32(sm + L::Wt + s * kTile);
+                const uint32_t b0 = smem_u32(sm + L::Wt + s * kTile);
                 constexpr uint32_t id = idesc_bf16(128, 64, false, true);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_bf16(tX, sdesc(a0 + (ks >> 2) * kTile + (ks & 3) * 32, 16, 1024),
-                             sdesc(b0 + ks * 2048, 8192, 1024), id, ks > 0);
-                mma_commit(bar_mma);
-                bulk_wait_read<1>();  // Delta^T staging of chunk c-1 has been read
-                if (!mbar_wait(bar_mma, mma_phase)) {
-                    *s_abort = 1;
-                    mma_pending = true;
-                    atomicExch(a.err, kErrTimeoutMma);
-                }
-            } else {
-                bulk_wait_read<1>();
+                    mma_bf16_ts(tX, tS + 8 * ks, sdesc(b0 + ks * 2048, 8192, 1024), id, ks > 0);
             }
-        }
-        if (kDelta) mma_phase ^= 1;
-        __syncthreads();
-        if (*s_abort) {
-            aborted = true;
-            break;
-        }
-        // Delta^T[j][r] = U^T[j][r] - X^T[j][r] for tokens r in [16 part, 16 part + 16)
-        float X[16];
-        if (kDelta) {
-            tc_fence_after();
-            tmem_ld16(tX + lane_base + part * 16, X);
-            tmem_ld_wait();
-        } else {
-#pragma unroll
-            for (int q = 0; q < 16; ++q) X[q] = 0.f;
-        }
-        const float* E = Eds + s * 128;
-        const uint8_t* Ut = sm + L::Ut + s * kTile;
-#pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-            const int q = part * 2 + qq;  // tokens 8q .. 8q + 7
-            const uint4 u = *(const uint4*)(Ut + sw128(j, q));
-            const float4 e0 = *(const float4*)(E + q * 8), e1 = *(const float4*)(E + q * 8 + 4);
-            const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
-            uint32_t dw[4], tw[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const float2 uf = unpack_bf16(uw[p]);
-                const float d0 = uf.x - X[qq * 8 + 2 * p];
-                const float d1 = uf.y - X[qq * 8 + 2 * p + 1];
-                dw[p] = pack_bf16(d0, d1);
-                tw[p] = pack_bf16(d0 * ev[2 * p], d1 * ev[2 * p + 1]);
+            mma_commit(bar_x);
+            // the chunk state entering c to global memory, staged while X^T is computed
+            wait(bar_sst, par, kErrTimeoutMma);
+            if (ok) {
+                tma_store_2d(&tm_sc, sm + L::St, 0, (bh * NC + c) * kD);
+                tma_store_2d(&tm_sc, sm + L::St + kTile, 64, (bh * NC + c) * kD);
             }
-            *(uint4*)(sm + L::Dst + sw128(j, q)) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
-            *(uint4*)(sm + L::Dsc + sw128(j, q)) = make_uint4(tw[0], tw[1], tw[2], tw[3]);
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tma_store_2d(&tm_dt, sm + L::Dst, 0, (bh * NC + c) * kD);
             bulk_commit();
-            tc_fence_after();
-            const uint32_t a0 = smem_u32(sm + L::Dsc), b0 = smem_u32(sm + L::Kt + s * kTile);
-            constexpr uint32_t id = idesc_bf16(128, 128, false, true);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tP, sdesc(a0 + ks * 32, 16, 1024), sdesc(b0 + ks * 2048, 8192, 1024),
-                         id, ks > 0);
-            mma_commit(bar_mma);
-            bulk_wait_read<1>();  // the S^T store issued after chunk c-1 has been read
-            if (!mbar_wait(bar_mma, mma_phase)) {
-                *s_abort = 1;
-                mma_pending = true;
-                atomicExch(a.err, kErrTimeoutMma);
-            } else if (issued < NC) {
-                issue_load(issued);  // stage s is free again
+            bulk_wait_read<1>();  // the Delta^T store of chunk c-1 has read its tile
+            if (c > 0) mbar_arrive(bar_dfree);
+            // the stage of chunk c-1 is free: its products are done and the element-wise
+            // warps have handed over S^T of chunk c, after their last read of it
+            if (ok && c >= 1 && issued < NC) {
+                issue_load(issued);
                 ++issued;
             }
+            wait(bar_d, par, kErrTimeoutMma);  // (e^{G_C - G} Delta)^T is in TMEM
+            if (ok) {
+                tc_fence_after();
+                const uint32_t b0 = smem_u32(sm + L::Kt + s * kTile);
+                constexpr uint32_t id = idesc_bf16(128, 128, false, true);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ts(tP, tD + 8 * ks, sdesc(b0 + ks * 2048, 8192, 1024), id, ks > 0);
+            }
+            mma_commit(bar_p);
+            wait(bar_dst, par, kErrTimeoutMma);
+            if (ok) tma_store_2d(&tm_dt, sm + L::Dst, 0, (bh * NC + c) * kD);
+            bulk_commit();
+            bulk_wait_read<1>();  // the S^T store of chunk c has read its tile
+            mbar_arrive(bar_sfree);
         }
-        mma_phase ^= 1;
-        __syncthreads();
+        if (!ok) atomicExch(a.err, err);
+        // teardown: copies still in flight land, every UMMA issued has finished and
+        // the stores have read shared memory before the CTA exits
         if (*s_abort) {
-            aborted = true;
-            break;
+            for (int cc = 0; cc < issued; ++cc) mbar_wait(&bar_ld[cc % kStages], (cc / kStages) & 1);
+            mma_commit(bar_fin);
+            mbar_wait(bar_fin, 0);
         }
-        tc_fence_after();
-        {
+        bulk_wait_read<0>();
+    } else if (warp < 16) {
+        // ---------------- the element-wise warps
+        // `bad` stays warp-uniform (the warp-collective TMEM accesses and __syncwarp
+        // below need every lane): a failed wait in any lane ends the warp's loop
+        bool bad = false;
+        auto wait = [&](uint64_t* bar, uint32_t parity, int e) {
+            if (!bad && !mbar_wait_or_abort(bar, parity, s_abort)) {
+                bad = true;
+                if (!*s_abort) atomicExch(a.err, e);
+                *s_abort = 1;
+            }
+            bad = __any_sync(0xffffffffu, bad);
+        };
+        auto hand_over_tmem = [&](uint64_t* bar) {  // after tcgen05.st of an operand
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar);
+        };
+        auto hand_over_smem = [&](uint64_t* bar) {  // after shared-memory writes a TMA store reads
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar);
+        };
+        // S^T row j, state columns i in [32 part, 32 part + 32): S[q] = S_{i, j}
+        float S[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+            S[q] = a.S_in ? a.S_in[((size_t)bh * kD + part * 32 + q) * kD + j] : 0.f;
+        uint8_t* St = sm + L::St + (part >> 1) * kTile;
+        const int sq0 = (part & 1) * 4;  // first 16-byte chunk of this thread's 32 state columns
+        for (int c = 0; c < NC && !bad; ++c) {
+            const int s = c % kStages;
+            const uint32_t par = c & 1;
+            // (1) S^T as bf16 pairs into TMEM: the A operand of X^T = S^T W^T
+            {
+                uint32_t w[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) w[q] = pack_bf16(S[2 * q], S[2 * q + 1]);
+                tmem_st16u(tS + lane_base + 16 * part, w);
+            }
+            hand_over_tmem(bar_s);
+            // (2) the same bf16 S^T staged for its store, once the last one has read the tile
+            if (c > 0) wait(bar_sfree, (c - 1) & 1, kErrTimeoutTma);
+            put_row32(St, j, sq0, S);
+            hand_over_smem(bar_sst);
+            // (3) Delta^T[j][r] = U^T[j][r] - X^T[j][r] for tokens r in [16 part, 16 part + 16);
+            // e^{G_C - G_r} Delta^T into TMEM (A operand of P^T), Delta^T kept for its store
+            wait(&bar_ld[s], (c / kStages) & 1, kErrTimeoutTma);
+            float X[16];
+            if (kDelta) {
+                wait(bar_x, par, kErrTimeoutMma);
+                tc_fence_after();
+                tmem_ld16(tX + lane_base + part * 16, X);
+                tmem_ld_wait();
+            } else {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) X[q] = 0.f;
+            }
+            const float* E = Eds + s * 128;
+            const uint8_t* Ut = sm + L::Ut + s * kTile;
+            uint32_t dw[8], tw[8];
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq) {
+                const int q = part * 2 + qq;  // tokens 8q .. 8q + 7
+                const uint4 u = *(const uint4*)(Ut + sw128(j, q));
+                const float4 e0 = *(const float4*)(E + q * 8), e1 = *(const float4*)(E + q * 8 + 4);
+                const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+                const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const float2 uf = unpack_bf16(uw[p]);
+                    const float d0 = uf.x - X[qq * 8 + 2 * p];
+                    const float d1 = uf.y - X[qq * 8 + 2 * p + 1];
+                    dw[qq * 4 + p] = pack_bf16(d0, d1);
+                    tw[qq * 4 + p] = pack_bf16(d0 * ev[2 * p], d1 * ev[2 * p + 1]);
+                }
+            }
+            tmem_st8u(tD + lane_base + 8 * part, tw);
+            hand_over_tmem(bar_d);
+            // (4) Delta^T staged for its store
+            if (c > 0) wait(bar_dfree, (c - 1) & 1, kErrTimeoutTma);
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq)
+                *(uint4*)(sm + L::Dst + sw128(j, part * 2 + qq)) =
+                    make_uint4(dw[qq * 4], dw[qq * 4 + 1], dw[qq * 4 + 2], dw[qq * 4 + 3]);
+            hand_over_smem(bar_dst);
+            // (5) S^T <- gamma_C S^T + P^T
+            wait(bar_p, par, kErrTimeoutMma);
+            tc_fence_after();
             float P[32];
             tmem_ld32(tP + lane_base + part * 32, P);
             tmem_ld_wait();
@@ -269,35 +334,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int q = 0; q < 32; ++q) S[q] = gam * S[q] + P[q];
         }
-        if (c + 1 < NC) {
-            put_row32(St, j, sq0, S);
-            fence_async_smem();
-        }
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0 && c + 1 < NC) {
-            tma_store_2d(&tm_sc, sm + L::St, 0, (bh * NC + c + 1) * kD);
-            tma_store_2d(&tm_sc, sm + L::St + kTile, 64, (bh * NC + c + 1) * kD);
-            bulk_commit();
-        }
-    }
-    if (!aborted && a.S_out) {
+        if (!bad && a.S_out) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) a.S_out[((size_t)bh * kD + part * 32 + q) * kD + j] = S[q];
-    }
-    if (tid == 0) {
-        if (aborted) {
-            // let every copy and MMA this CTA started finish before it exits (bounded)
-            for (int cc = c; cc < issued; ++cc) mbar_wait(&bar_ld[cc % kStages], (cc / kStages) & 1);
-            if (mma_pending) mbar_wait(bar_mma, mma_phase ^ 1);
+            for (int q = 0; q < 32; ++q) a.S_out[((size_t)bh * kD + part * 32 + q) * kD + j] = S[q];
         }
-        bulk_wait_read<0>();  // stores have read shared memory (their writes land before the grid completes)
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -599,7 +645,7 @@ cudaError_t launch_state_fwd_tc(const Args& a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     timing_begin(KK_STATE_FWD, s);
-    kern<<<BH, kThreads, smem, s>>>(tm_wt, tm_ut, tm_k, tm_sc, tm_dt, a);
+    kern<<<BH, kFwdThreads, smem, s>>>(tm_wt, tm_ut, tm_k, tm_sc, tm_dt, a);
     e = cudaGetLastError();
     timing_end(KK_STATE_FWD, s);
     return e;

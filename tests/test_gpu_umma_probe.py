@@ -1,6 +1,6 @@
 """UMMA building blocks on the GPU: one-tile GEMMs through the library's
-descriptor helpers, for every operand major-ness and M in {64, 128}, compared
-with torch.matmul.  A wrong descriptor field shows up here as a numerical
+descriptor helpers, for every operand major-ness and M in {64, 128}, and with
+the A operand read from tensor memory, compared with torch.matmul.  A wrong descriptor field shows up here as a numerical
 mismatch before it can confuse a full kernel."""
 import ctypes
 import os
@@ -21,7 +21,7 @@ def probe(tmp_path_factory):
                            os.path.join(HERE, "cuda", "umma_probe.cu"), "-o", out])
     lib = ctypes.CDLL(out)
     lib.umma_probe.restype = ctypes.c_int
-    lib.umma_probe.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 8 + [ctypes.c_void_p] * 2
+    lib.umma_probe.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 9 + [ctypes.c_void_p] * 2
     return lib
 
 
@@ -44,14 +44,23 @@ def test_m64_lane_offset_and_tmem_store(probe, lane16, restore, a_mn, b_mn):
     run_probe(probe, 64, 128, 128, a_mn, b_mn, 0, lane16, restore)
 
 
-def run_probe(probe, M, N, K, a_mn, b_mn, neg_a, lane16, restore):
+@pytest.mark.parametrize("N", [64, 128])
+@pytest.mark.parametrize("K", [64, 128])
+@pytest.mark.parametrize("b_mn", [0, 1])
+@pytest.mark.parametrize("restore", [0, 1])
+def test_umma_a_from_tmem(probe, N, K, b_mn, restore):
+    """A (M = 128) held in tensor memory, two bf16 per column, lower K index low."""
+    run_probe(probe, 128, N, K, 0, b_mn, 0, 0, restore, a_tmem=1)
+
+
+def run_probe(probe, M, N, K, a_mn, b_mn, neg_a, lane16, restore, a_tmem=0):
     g = torch.Generator(device="cuda").manual_seed(M * 7 + N * 3 + K + 2 * a_mn + b_mn)
     A = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
     B = torch.randn(K, N, device="cuda", generator=g).to(torch.bfloat16)
     C = torch.full((M, N), float("nan"), device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     rc = probe.umma_probe(A.data_ptr(), B.data_ptr(), C.data_ptr(), M, N, K, a_mn, b_mn, neg_a,
-                          lane16, restore, err.data_ptr(), torch.cuda.current_stream().cuda_stream)
+                          lane16, restore, a_tmem, err.data_ptr(), torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
     assert rc == 0 and int(err.item()) == 0
     ref = (A.float() @ B.float()) * (-1.0 if neg_a else 1.0) * (3.0 if restore else 1.0)
