@@ -79,11 +79,14 @@ struct IntraSmem {
     static constexpr int V = QK + QKBytes;                    // [dvblk][64][64]
     static constexpr int X1 = V + kTile;                      // A_o, then N^2, then T diag(beta gamma)
     static constexpr int X2 = X1 + kHalf;                     // D, then E, then T diag(beta) (I without beta)
-    static constexpr int X3 = X2 + kHalf;                     // N, then T (kP)
-    static constexpr int Pst = X3 + kHalf;                    // P staging (kP)
-    static constexpr int Adf = Pst + (kP ? kHalf : 0);        // fp32 [4][16][kDS]: diagonal blocks of A
-    static constexpr int Dfp = Adf + 4 * 16 * kDS * 4;        // fp32 [4][16][kDS]: their inverses
-    static constexpr int Gs = Dfp + 4 * 16 * kDS * 4;         // G
+    static constexpr int X3 = X2 + kHalf;                     // kP: P staging, then N, then T
+    static constexpr int Pst = X3;                            // (P is stored before N is written)
+    // fp32 [4][16][kDS] diagonal blocks of A and their inverses; with P they live in
+    // Q's two d_k blocks (dead after [Q; K] K^T), so that three CTAs fit on an SM
+    static constexpr int ADBytes = 4 * 16 * kDS * 4;
+    static constexpr int Adf = kP ? QK : X3 + kHalf;
+    static constexpr int Dfp = kP ? QK + kTile : Adf + ADBytes;
+    static constexpr int Gs = X3 + kHalf + (kP ? 0 : 2 * ADBytes);  // G
     static constexpr int Bs = Gs + 256;                       // beta
     static constexpr int BGs = Bs + 256;                      // beta gamma
     static constexpr int Bar = BGs + 256;
@@ -335,6 +338,7 @@ __global__ void __launch_bounds__(kIntraThreads)
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(c64, sdesc(x2 + ks * 32, 16, 1024), sdesc(x1 + ks * 2048, kHalf, 1024), id, ks > 0);
             mma_wait();
+            if (kP) bulk_wait_read<0>();  // the P store has read X3, where N goes next
         }
         mph ^= 1;
         __syncthreads();
@@ -767,7 +771,13 @@ teardown:
 
 template <typename K>
 cudaError_t set_smem(K kern, size_t smem) {
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // all of the SM's unified L1 / shared memory as shared memory, so that as many
+    // CTAs as their shared memory allows are resident
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+    return e;
 }
 
 }  // namespace
