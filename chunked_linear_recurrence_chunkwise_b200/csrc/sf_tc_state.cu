@@ -352,15 +352,14 @@ constexpr int kBStages = 2;
 struct BwdSmem {
     static constexpr int Kt = 0;                          // [stage] K   [2][64 r][64 d_k]
     static constexpr int dO = Kt + kBStages * kTile;      // [stage] dO  [2][64 r][64 d_v]
-    static constexpr int Q = dO + kBStages * kTile;       // [stage] Q   [2][64 r][64 d_k]
+    static constexpr int Q = dO + kBStages * kTile;       // [stage] Q   [2][64 r][64 d_k], scaled in place
     static constexpr int Wt = Q + kBStages * kTile;       // [stage] W^T [d_k][64 r]
     static constexpr int P = Wt + kBStages * kTile;       // [stage] P   [64 i][64 r]
-    static constexpr int St = P + kBStages * 8192;        // dS^T operand [2 kblk][d_v][64]
-    static constexpr int Dop = St + 2 * kTile;            // dDelta^T [d_v][64 r] (operand + store)
-    static constexpr int Dv = Dop + kTile;                // dv staging [2][64 r][64 d_v] (no beta)
-    static constexpr int Ed = Dv + kTile;                 // [stage][128] fp32 decay table
-    static constexpr int Bar = Ed + kBStages * 512;
-    static constexpr int Misc = Bar + (kBStages + 1) * 8;
+    static constexpr int St = P + kBStages * 8192;        // dS'^T staging for its store [2 kblk][d_v][64]
+    static constexpr int Dst = St + 2 * kTile;            // dDelta^T [d_v][64 r] (or dv [2][64 r][64 d_v]) staging
+    static constexpr int Ed = Dst + kTile;                // [stage][128] fp32 decay table
+    static constexpr int Bar = Ed + kBStages * 512;       // barriers, see the kernel
+    static constexpr int Misc = Bar + 16 * 8;             // TMEM base, abort flag
     static constexpr int Size = Misc + 16;
 };
 
@@ -370,8 +369,23 @@ struct BwdSmem {
 // (the transpose of dS = gamma_C dS' + (diag(gamma) Q)^T dO - W^T dDelta with
 // dDelta = P^T dO + Ktil dS').  Stores dS'^T of every chunk and dDelta^T (or
 // dv = dDelta directly for linear attention).
+//
+// As in the forward pass, the two products on the dependent chain take their
+// A operand from TMEM (dS'^T, and -dDelta^T in bf16 pairs), a seventeenth warp
+// issues every copy, UMMA and store, and the bf16 copies for global memory are
+// staged off the chain.  The products that do not involve the carried state
+// leave the chain: dO^T P of the next chunk is issued as soon as its tiles have
+// landed, and dO^T (diag(gamma) Q) right behind dS'^T K^T, while the
+// element-wise warps form dDelta^T.  Hand-overs (one arrival per warp):
+//   bar_s    dS'^T of chunk c in TMEM        bar_y  dS'^T K^T (and dO^T P) done
+//   bar_q    Q of chunk c scaled by gamma     bar_z  dS^T update product done
+//   bar_d    -dDelta^T in TMEM (dO^T P read)  bar_sfree / bar_dfree  stores have read
+//   bar_sst  dS'^T staged for its store                                their tiles
+//   bar_dst  dDelta^T (or dv) staged for its store
+// TMEM (512 columns): dS'^T K^T [0, 64), dO^T P [64, 128), the dS^T update
+// [128, 256), dS'^T operand [256, 320), -dDelta^T operand [320, 352).
 template <bool kDelta>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     state_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_do,
                         const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_wt,
                         const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_dsc,
@@ -381,8 +395,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     float* Eds = (float*)(sm + L::Ed);
-    uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);
-    uint64_t* bar_mma = bar_ld + kBStages;
+    uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);  // [kBStages], count 1
+    uint64_t* bar_y = bar_ld + kBStages;          // count 1 (commits and the issuer)
+    uint64_t* bar_z = bar_y + 1;
+    uint64_t* bar_sfree = bar_y + 2;
+    uint64_t* bar_dfree = bar_y + 3;
+    uint64_t* bar_fin = bar_y + 4;
+    uint64_t* bar_s = bar_y + 5;                  // count 16 (one arrival per element-wise warp)
+    uint64_t* bar_q = bar_y + 6;
+    uint64_t* bar_d = bar_y + 7;
+    uint64_t* bar_sst = bar_y + 8;
+    uint64_t* bar_dst = bar_y + 9;
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
     volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
 
@@ -392,104 +415,220 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
     const int NC = a.NC;
 
-    if (tid == 0) {
-        for (int s = 0; s < kBStages; ++s) mbar_init(&bar_ld[s], 1);
-        mbar_init(bar_mma, 1);
+    if (tid == kFwdIss) {
+        for (int i = 0; i < kBStages + 10; ++i) mbar_init(bar_ld + i, i >= kBStages + 5 ? 16 : 1);
         *s_abort = 0;
         fence_barrier_init();
     }
-    if (warp == 0) tmem_alloc(s_tmem, 256);
+    if (warp == 0) tmem_alloc(s_tmem, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    const uint32_t tY1 = tmem, tY2 = tmem + 64, tZ = tmem + 128;
+    const uint32_t tY1 = tmem, tY2 = tmem + 64, tZ = tmem + 128, tS = tmem + 256, tD = tmem + 320;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
 
-    // n-th load (n = 0, 1, ...) is chunk NC - 1 - n, stage n % 2
-    auto issue_load = [&](int n) {
-        const int c = NC - 1 - n, s = n % kBStages;
-        const uint32_t bytes = 3 * kTile + 8192 + (kDelta ? kTile : 0) + 512;
-        mbar_expect_tx(&bar_ld[s], bytes);
-        tma_load_4d(sm + L::Kt + s * kTile, &tm_k, 0, h, c * kChunk, b, &bar_ld[s]);
-        tma_load_4d(sm + L::Kt + s * kTile + 8192, &tm_k, 64, h, c * kChunk, b, &bar_ld[s]);
-        tma_load_4d(sm + L::dO + s * kTile, &tm_do, 0, h, c * kChunk, b, &bar_ld[s]);
-        tma_load_4d(sm + L::dO + s * kTile + 8192, &tm_do, 64, h, c * kChunk, b, &bar_ld[s]);
-        tma_load_4d(sm + L::Q + s * kTile, &tm_q, 0, h, c * kChunk, b, &bar_ld[s]);
-        tma_load_4d(sm + L::Q + s * kTile + 8192, &tm_q, 64, h, c * kChunk, b, &bar_ld[s]);
-        if (kDelta) tma_load_2d(sm + L::Wt + s * kTile, &tm_wt, 0, (bh * NC + c) * kD, &bar_ld[s]);
-        tma_load_2d(sm + L::P + s * 8192, &tm_p, 0, (bh * NC + c) * kChunk, &bar_ld[s]);
-        bulk_load(Eds + s * 128, a.Ed + ((size_t)bh * NC + c) * 128, 512, &bar_ld[s]);
-    };
-    int issued = 0;
-    if (tid == 0)
+    if (tid == kFwdIss) {
+        // ---------------- the issuer; the n-th iteration is chunk NC - 1 - n, stage n % 2
+        auto issue_load = [&](int n) {
+            const int c = NC - 1 - n, s = n % kBStages;
+            const uint32_t bytes = 3 * kTile + 8192 + (kDelta ? kTile : 0) + 512;
+            mbar_expect_tx(&bar_ld[s], bytes);
+            tma_load_4d(sm + L::Kt + s * kTile, &tm_k, 0, h, c * kChunk, b, &bar_ld[s]);
+            tma_load_4d(sm + L::Kt + s * kTile + 8192, &tm_k, 64, h, c * kChunk, b, &bar_ld[s]);
+            tma_load_4d(sm + L::dO + s * kTile, &tm_do, 0, h, c * kChunk, b, &bar_ld[s]);
+            tma_load_4d(sm + L::dO + s * kTile + 8192, &tm_do, 64, h, c * kChunk, b, &bar_ld[s]);
+            tma_load_4d(sm + L::Q + s * kTile, &tm_q, 0, h, c * kChunk, b, &bar_ld[s]);
+            tma_load_4d(sm + L::Q + s * kTile + 8192, &tm_q, 64, h, c * kChunk, b, &bar_ld[s]);
+            if (kDelta) tma_load_2d(sm + L::Wt + s * kTile, &tm_wt, 0, (bh * NC + c) * kD, &bar_ld[s]);
+            tma_load_2d(sm + L::P + s * 8192, &tm_p, 0, (bh * NC + c) * kChunk, &bar_ld[s]);
+            bulk_load(Eds + s * 128, a.Ed + ((size_t)bh * NC + c) * 128, 512, &bar_ld[s]);
+        };
+        // dO^T P of iteration n into its accumulator (its tiles have landed)
+        auto issue_y2 = [&](int n) {
+            const int s = n % kBStages;
+            const uint32_t dob = smem_u32(sm + L::dO + s * kTile), pb = smem_u32(sm + L::P + s * 8192);
+            constexpr uint32_t id = idesc_bf16(128, 64, true, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tY2, sdesc(dob + ks * 2048, 8192, 1024), sdesc(pb + ks * 2048, 8192, 1024), id, ks > 0);
+        };
+        int issued = 0;
         for (; issued < min(kBStages, NC); ++issued) issue_load(issued);
-
-    // dS^T row j, state columns i in [32 part, 32 part + 32): S[q] = dS_{i, j}
-    float S[32];
-#pragma unroll
-    for (int q = 0; q < 32; ++q)
-        S[q] = a.dS_out ? a.dS_out[((size_t)bh * kD + part * 32 + q) * kD + j] : 0.f;
-    uint8_t* St = sm + L::St + (part >> 1) * kTile;
-    const int sq0 = (part & 1) * 4;
-    put_row32(St, j, sq0, S);
-    fence_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-        tma_store_2d(&tm_dsc, sm + L::St, 0, (bh * NC + NC - 1) * kD);
-        tma_store_2d(&tm_dsc, sm + L::St + kTile, 64, (bh * NC + NC - 1) * kD);
-        bulk_commit();
-    }
-
-    uint32_t mma_phase = 0;
-    bool mma_pending = false;
-    bool aborted = false;
-    int n = 0;
-    for (; n < NC; ++n) {
-        const int c = NC - 1 - n, s = n % kBStages;
-        if (tid == 0) {
-            if (!mbar_wait(&bar_ld[s], (n / kBStages) & 1)) {
+        bool ok = true, y2_early = false;
+        int err = 0;
+        auto wait = [&](uint64_t* bar, uint32_t parity, int e) {
+            if (ok && !mbar_wait_or_abort(bar, parity, s_abort)) {
+                ok = false;
+                err = e;
                 *s_abort = 1;
-                atomicExch(a.err, kErrTimeoutTma);
-            } else {
+            }
+        };
+        for (int n = 0; n < NC; ++n) {
+            const int c = NC - 1 - n, s = n % kBStages;
+            const uint32_t par = n & 1;
+            wait(bar_s, par, kErrTimeoutMma);  // dS'^T of chunk c is in TMEM
+            // the stage of iteration n-1 is free: its products are done and the element-wise
+            // warps have handed over dS'^T of this iteration, after their last read of it
+            if (ok && n >= 1 && issued < NC) {
+                issue_load(issued);
+                ++issued;
+            }
+            wait(&bar_ld[s], (n / kBStages) & 1, kErrTimeoutTma);
+            if (ok) {
                 tc_fence_after();
-                const uint32_t st = smem_u32(sm + L::St), kt = smem_u32(sm + L::Kt + s * kTile);
-                const uint32_t dob = smem_u32(sm + L::dO + s * kTile), pb = smem_u32(sm + L::P + s * 8192);
-                constexpr uint32_t id1 = idesc_bf16(128, 64, false, false);
-                constexpr uint32_t id2 = idesc_bf16(128, 64, true, true);
+                if (!y2_early) issue_y2(n);
+                const uint32_t kt = smem_u32(sm + L::Kt + s * kTile);
+                constexpr uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_bf16(tY1, sdesc(st + (ks >> 2) * kTile + (ks & 3) * 32, 16, 1024),
-                             sdesc(kt + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id1, ks > 0);
+                for (int ks = 0; ks < 8; ++ks)  // dS'^T K^T
+                    mma_bf16_ts(tY1, tS + 8 * ks, sdesc(kt + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id,
+                                ks > 0);
+            }
+            mma_commit(bar_y);
+            wait(bar_q, par, kErrTimeoutMma);  // Q of chunk c scaled by gamma
+            if (ok) {
+                tc_fence_after();
+                const uint32_t dob = smem_u32(sm + L::dO + s * kTile), qb = smem_u32(sm + L::Q + s * kTile);
+                constexpr uint32_t id = idesc_bf16(128, 128, true, true);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tY2, sdesc(dob + ks * 2048, 8192, 1024), sdesc(pb + ks * 2048, 8192, 1024),
-                             id2, ks > 0);
-                mma_commit(bar_mma);
-                bulk_wait_read<1>();  // the dDelta^T / dv store of chunk c+1 has been read
-                if (!mbar_wait(bar_mma, mma_phase)) {
-                    *s_abort = 1;
-                    mma_pending = true;
-                    atomicExch(a.err, kErrTimeoutMma);
+                for (int ks = 0; ks < 4; ++ks)  // dO^T (diag(gamma) Q)
+                    mma_bf16(tZ, sdesc(dob + ks * 2048, 8192, 1024), sdesc(qb + ks * 2048, 8192, 1024), id, ks > 0);
+            }
+            // dS'^T of chunk c to global memory, staged while the products run
+            wait(bar_sst, par, kErrTimeoutMma);
+            if (ok) {
+                tma_store_2d(&tm_dsc, sm + L::St, 0, (bh * NC + c) * kD);
+                tma_store_2d(&tm_dsc, sm + L::St + kTile, 64, (bh * NC + c) * kD);
+            }
+            bulk_commit();
+            bulk_wait_read<1>();  // the dDelta^T (dv) store of iteration n-1 has read its tile
+            if (n > 0) mbar_arrive(bar_dfree);
+            wait(bar_d, par, kErrTimeoutMma);  // -dDelta^T in TMEM; dO^T P has been read
+            if (ok && kDelta) {
+                tc_fence_after();
+                const uint32_t wt = smem_u32(sm + L::Wt + s * kTile);
+                constexpr uint32_t id = idesc_bf16(128, 128, false, false);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)  // - dDelta^T W
+                    mma_bf16_ts(tZ, tD + 8 * ks, sdesc(wt + ks * 32, 16, 1024), id, 1);
+            }
+            mma_commit(bar_z);
+            // dO^T P of the next iteration, if its tiles have already landed
+            y2_early = false;
+            if (ok && n + 1 < NC && mbar_try_wait(&bar_ld[(n + 1) % kBStages], ((n + 1) / kBStages) & 1)) {
+                tc_fence_after();
+                issue_y2(n + 1);
+                y2_early = true;
+            }
+            wait(bar_dst, par, kErrTimeoutMma);
+            if (ok) {
+                if (kDelta) {
+                    tma_store_2d(&tm_ddt, sm + L::Dst, 0, (bh * NC + c) * kD);
+                } else {
+                    tma_store_4d(&tm_dv, sm + L::Dst, 0, h, c * kChunk, b);
+                    tma_store_4d(&tm_dv, sm + L::Dst + 8192, 64, h, c * kChunk, b);
                 }
             }
+            bulk_commit();
+            bulk_wait_read<1>();  // the dS'^T store of iteration n has read its tile
+            mbar_arrive(bar_sfree);
         }
-        mma_phase ^= 1;
-        __syncthreads();
+        if (!ok) atomicExch(a.err, err);
+        // teardown: copies still in flight land, every UMMA issued has finished and
+        // the stores have read shared memory before the CTA exits
         if (*s_abort) {
-            aborted = true;
-            break;
+            for (int m = 0; m < issued; ++m) mbar_wait(&bar_ld[m % kBStages], (m / kBStages) & 1);
+            mma_commit(bar_fin);
+            mbar_wait(bar_fin, 0);
         }
-        tc_fence_after();
-        const float* E = Eds + s * 128;
-        {
-            float y1[16], y2[16];
-            tmem_ld16(tY1 + lane_base + part * 16, y1);
-            tmem_ld16(tY2 + lane_base + part * 16, y2);
-            tmem_ld_wait();
-            float d[16];
+        bulk_wait_read<0>();
+    } else if (warp < 16) {
+        // ---------------- the element-wise warps (`bad` warp-uniform, as in the forward pass)
+        bool bad = false;
+        auto wait = [&](uint64_t* bar, uint32_t parity, int e) {
+            if (!bad && !mbar_wait_or_abort(bar, parity, s_abort)) {
+                bad = true;
+                if (!*s_abort) atomicExch(a.err, e);
+                *s_abort = 1;
+            }
+            bad = __any_sync(0xffffffffu, bad);
+        };
+        auto hand_over_tmem = [&](uint64_t* bar) {
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar);
+        };
+        auto hand_over_smem = [&](uint64_t* bar) {
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar);
+        };
+        // dS^T row j, state columns i in [32 part, 32 part + 32): S[q] = dS_{i, j}
+        float S[32];
 #pragma unroll
-            for (int q = 0; q < 16; ++q) d[q] = E[part * 16 + q] * y1[q] + y2[q];
+        for (int q = 0; q < 32; ++q)
+            S[q] = a.dS_out ? a.dS_out[((size_t)bh * kD + part * 32 + q) * kD + j] : 0.f;
+        uint8_t* St = sm + L::St + (part >> 1) * kTile;
+        const int sq0 = (part & 1) * 4;
+        for (int n = 0; n < NC && !bad; ++n) {
+            const int s = n % kBStages;
+            const uint32_t par = n & 1;
+            // (1) dS'^T as bf16 pairs into TMEM: the A operand of dS'^T K^T
+            {
+                uint32_t w[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) w[q] = pack_bf16(S[2 * q], S[2 * q + 1]);
+                tmem_st16u(tS + lane_base + 16 * part, w);
+            }
+            hand_over_tmem(bar_s);
+            // (2) diag(gamma) Q in place, 32 bytes of a 128-byte line per thread
+            wait(&bar_ld[s], (n / kBStages) & 1, kErrTimeoutTma);
+            const float* E = Eds + s * 128;
+            {
+                const int line = tid >> 2, r = line & 63, blk = line >> 6;
+                uint8_t* ln = sm + L::Q + s * kTile + blk * 8192 + r * 128 + (tid & 3) * 32;
+                const float f = E[64 + r];
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {
+                    uint4 u = *(uint4*)(ln + qq * 16);
+                    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const float2 x = unpack_bf16(w[p]);
+                        w[p] = pack_bf16(x.x * f, x.y * f);
+                    }
+                    *(uint4*)(ln + qq * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            hand_over_smem(bar_q);
+            // (3) dS'^T staged for its store, once the last one has read the tile
+            if (n > 0) wait(bar_sfree, (n - 1) & 1, kErrTimeoutTma);
+            put_row32(St, j, sq0, S);
+            hand_over_smem(bar_sst);
+            // (4) dDelta^T[j][r] = e^{G_C - G_r} (dS'^T K^T)[j][r] + (dO^T P)[j][r], r in
+            // [16 part, 16 part + 16); -dDelta^T into TMEM (A operand of - dDelta^T W)
+            wait(bar_y, par, kErrTimeoutMma);
+            tc_fence_after();
+            float d[16];
+            {
+                float y1[16], y2[16];
+                tmem_ld16(tY1 + lane_base + part * 16, y1);
+                tmem_ld16(tY2 + lane_base + part * 16, y2);
+                tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < 16; ++q) d[q] = E[part * 16 + q] * y1[q] + y2[q];
+            }
+            if (kDelta) {
+                uint32_t w[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) w[q] = pack_bf16(-d[2 * q], -d[2 * q + 1]);
+                tmem_st8u(tD + lane_base + 8 * part, w);
+            }
+            hand_over_tmem(bar_d);
+            // (5) dDelta^T (or dv = dDelta, token-major, for linear attention) staged for its store
+            if (n > 0) wait(bar_dfree, (n - 1) & 1, kErrTimeoutTma);
             if (kDelta) {
 #pragma unroll
                 for (int qq = 0; qq < 2; ++qq) {
@@ -498,78 +637,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     u.y = pack_bf16(d[qq * 8 + 2], d[qq * 8 + 3]);
                     u.z = pack_bf16(d[qq * 8 + 4], d[qq * 8 + 5]);
                     u.w = pack_bf16(d[qq * 8 + 6], d[qq * 8 + 7]);
-                    *(uint4*)(sm + L::Dop + sw128(j, part * 2 + qq)) = u;
+                    *(uint4*)(sm + L::Dst + sw128(j, part * 2 + qq)) = u;
                 }
             } else {
-                // linear attention: dv = dDelta, staged token-major for a TMA store
                 const uint32_t jb = (uint32_t)(j >> 6) * 8192, jq = (j & 63) >> 3, je = (j & 7) * 2;
 #pragma unroll
                 for (int q = 0; q < 16; ++q)
-                    *(__nv_bfloat16*)(sm + L::Dv + jb + sw128(part * 16 + q, jq) + je) =
-                        __float2bfloat16_rn(d[q]);
+                    *(__nv_bfloat16*)(sm + L::Dst + jb + sw128(part * 16 + q, jq) + je) = __float2bfloat16_rn(d[q]);
             }
-        }
-        if (tid < 256) {  // diag(gamma) Q in place, half a 128-byte line per thread
-            const int line = tid >> 1, r = line & 63, blk = line >> 6;
-            uint8_t* ln = sm + L::Q + s * kTile + blk * 8192 + r * 128 + (tid & 1) * 64;
-            const float f = E[64 + r];
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                const int q = (qq + (line >> 1)) & 3;  // lanes on distinct banks
-                uint4 u = *(uint4*)(ln + q * 16);
-                uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const float2 x = unpack_bf16(w[p]);
-                    w[p] = pack_bf16(x.x * f, x.y * f);
-                }
-                *(uint4*)(ln + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            if (kDelta) {
-                tma_store_2d(&tm_ddt, sm + L::Dop, 0, (bh * NC + c) * kD);
-            } else {
-                tma_store_4d(&tm_dv, sm + L::Dv, 0, h, c * kChunk, b);
-                tma_store_4d(&tm_dv, sm + L::Dv + 8192, 64, h, c * kChunk, b);
-            }
-            bulk_commit();
+            hand_over_smem(bar_dst);
+            // (6) dS^T <- gamma_C dS'^T + dO^T (diag(gamma) Q) - dDelta^T W
+            wait(bar_z, par, kErrTimeoutMma);
             tc_fence_after();
-            const uint32_t dob = smem_u32(sm + L::dO + s * kTile), qb = smem_u32(sm + L::Q + s * kTile);
-            constexpr uint32_t idA = idesc_bf16(128, 128, true, true);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tZ, sdesc(dob + ks * 2048, 8192, 1024), sdesc(qb + ks * 2048, 8192, 1024), idA,
-                         ks > 0);
-            if (kDelta) {
-                const uint32_t dop = smem_u32(sm + L::Dop), wt = smem_u32(sm + L::Wt + s * kTile);
-                constexpr uint32_t idB = idesc_bf16(128, 128, false, false, true);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tZ, sdesc(dop + ks * 32, 16, 1024), sdesc(wt + ks * 32, 16, 1024), idB, 1);
-            }
-            mma_commit(bar_mma);
-            bulk_wait_read<1>();  // the dS'^T store issued after chunk c+1 has been read
-            if (!mbar_wait(bar_mma, mma_phase)) {
-                *s_abort = 1;
-                mma_pending = true;
-                atomicExch(a.err, kErrTimeoutMma);
-            } else if (issued < NC) {
-                issue_load(issued);  // stage s is free again
-                ++issued;
-            }
-        }
-        mma_phase ^= 1;
-        __syncthreads();
-        if (*s_abort) {
-            aborted = true;
-            break;
-        }
-        tc_fence_after();
-        {
             float z[32];
             tmem_ld32(tZ + lane_base + part * 32, z);
             tmem_ld_wait();
@@ -577,34 +656,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int q = 0; q < 32; ++q) S[q] = gam * S[q] + z[q];
         }
-        if (c > 0) {
-            put_row32(St, j, sq0, S);
-            fence_async_smem();
-        }
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0 && c > 0) {
-            tma_store_2d(&tm_dsc, sm + L::St, 0, (bh * NC + c - 1) * kD);
-            tma_store_2d(&tm_dsc, sm + L::St + kTile, 64, (bh * NC + c - 1) * kD);
-            bulk_commit();
-        }
-    }
-    if (!aborted && a.dS_in) {
+        if (!bad && a.dS_in) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) a.dS_in[((size_t)bh * kD + part * 32 + q) * kD + j] = S[q];
-    }
-    if (tid == 0) {
-        if (aborted) {
-            for (int m = n; m < issued; ++m) mbar_wait(&bar_ld[m % kBStages], (m / kBStages) & 1);
-            if (mma_pending) mbar_wait(bar_mma, mma_phase ^ 1);
+            for (int q = 0; q < 32; ++q) a.dS_in[((size_t)bh * kD + part * 32 + q) * kD + j] = S[q];
         }
-        bulk_wait_read<0>();  // stores have read shared memory (their writes land before the grid completes)
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 }  // namespace
@@ -670,7 +731,7 @@ cudaError_t launch_state_bwd_tc(const Args& a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     timing_begin(KK_STATE_BWD, s);
-    kern<<<BH, kThreads, smem, s>>>(tm_k, tm_do, tm_q, tm_wt, tm_p, tm_dsc, tm_ddt, tm_dv, a);
+    kern<<<BH, kFwdThreads, smem, s>>>(tm_k, tm_do, tm_q, tm_wt, tm_p, tm_dsc, tm_ddt, tm_dv, a);
     e = cudaGetLastError();
     timing_end(KK_STATE_BWD, s);
     return e;
