@@ -359,7 +359,7 @@ struct BwdSmem {
     static constexpr int Dst = St + 2 * kTile;            // dDelta^T [d_v][64 r] (or dv [2][64 r][64 d_v]) staging
     static constexpr int Ed = Dst + kTile;                // [stage][128] fp32 decay table
     static constexpr int Bar = Ed + kBStages * 512;       // barriers, see the kernel
-    static constexpr int Misc = Bar + 16 * 8;             // TMEM base, abort flag
+    static constexpr int Misc = Bar + 16 * 8;             // TMEM base, abort flag (13 barriers)
     static constexpr int Size = Misc + 16;
 };
 
@@ -371,21 +371,24 @@ struct BwdSmem {
 // dv = dDelta directly for linear attention).
 //
 // As in the forward pass, the two products on the dependent chain take their
-// A operand from TMEM (dS'^T, and -dDelta^T in bf16 pairs), a seventeenth warp
-// issues every copy, UMMA and store, and the bf16 copies for global memory are
-// staged off the chain.  The products that do not involve the carried state
-// leave the chain: dO^T P of the next chunk is issued as soon as its tiles have
-// landed, and dO^T (diag(gamma) Q) right behind dS'^T K^T, while the
-// element-wise warps form dDelta^T.  Hand-overs (one arrival per warp):
-//   bar_s    dS'^T of chunk c in TMEM        bar_y  dS'^T K^T (and dO^T P) done
-//   bar_q    Q of chunk c scaled by gamma     bar_z  dS^T update product done
-//   bar_d    -dDelta^T in TMEM (dO^T P read)  bar_sfree / bar_dfree  stores have read
-//   bar_sst  dS'^T staged for its store                                their tiles
-//   bar_dst  dDelta^T (or dv) staged for its store
+// A operand from TMEM (dS'^T, and -dDelta^T in bf16 pairs) and the bf16 copies
+// for global memory are staged off the chain.  Two issuing threads, each the
+// first of its own warp: one issues the chain's UMMAs (dS'^T K^T, then
+// dO^T (diag(gamma) Q) behind it while the element-wise warps form dDelta^T,
+// then - dDelta^T W); the other every copy and store, and dO^T P of the next
+// chunk as soon as its tiles have landed, so that neither waits on the other's
+// slow issues.  Hand-overs (one arrival per element-wise warp):
+//   bar_s    dS'^T of chunk c in TMEM        bar_y   dS'^T K^T done (commit)
+//   bar_q    Q of chunk c scaled by gamma     bar_y2  dO^T P done (commit)
+//   bar_d    -dDelta^T in TMEM (dO^T P read)  bar_z   dS^T update product done
+//   bar_sst  dS'^T staged for its store       bar_sfree / bar_dfree  stores have
+//   bar_dst  dDelta^T (or dv) staged          read their tiles
 // TMEM (512 columns): dS'^T K^T [0, 64), dO^T P [64, 128), the dS^T update
 // [128, 256), dS'^T operand [256, 320), -dDelta^T operand [320, 352).
+constexpr int kBwdThreads = kThreads + 64;
+constexpr int kBwdChain = kThreads, kBwdCopy = kThreads + 32;
 template <bool kDelta>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     state_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_do,
                         const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_wt,
                         const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_dsc,
@@ -396,16 +399,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     float* Eds = (float*)(sm + L::Ed);
     uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);  // [kBStages], count 1
-    uint64_t* bar_y = bar_ld + kBStages;          // count 1 (commits and the issuer)
-    uint64_t* bar_z = bar_y + 1;
-    uint64_t* bar_sfree = bar_y + 2;
-    uint64_t* bar_dfree = bar_y + 3;
-    uint64_t* bar_fin = bar_y + 4;
-    uint64_t* bar_s = bar_y + 5;                  // count 16 (one arrival per element-wise warp)
-    uint64_t* bar_q = bar_y + 6;
-    uint64_t* bar_d = bar_y + 7;
-    uint64_t* bar_sst = bar_y + 8;
-    uint64_t* bar_dst = bar_y + 9;
+    uint64_t* bar_y = bar_ld + kBStages;          // count 1 (commits and the copy thread)
+    uint64_t* bar_y2 = bar_y + 1;
+    uint64_t* bar_z = bar_y + 2;
+    uint64_t* bar_sfree = bar_y + 3;
+    uint64_t* bar_dfree = bar_y + 4;
+    uint64_t* bar_fin = bar_y + 5;                // count 2 (both issuers)
+    uint64_t* bar_s = bar_y + 6;                  // count 16 (one arrival per element-wise warp)
+    uint64_t* bar_q = bar_y + 7;
+    uint64_t* bar_d = bar_y + 8;
+    uint64_t* bar_sst = bar_y + 9;
+    uint64_t* bar_dst = bar_y + 10;
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
     volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
 
@@ -415,8 +419,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
     const int NC = a.NC;
 
-    if (tid == kFwdIss) {
-        for (int i = 0; i < kBStages + 10; ++i) mbar_init(bar_ld + i, i >= kBStages + 5 ? 16 : 1);
+    if (tid == kBwdCopy) {
+        for (int i = 0; i < kBStages + 11; ++i) {
+            const int k = i - kBStages;
+            mbar_init(bar_ld + i, k < 5 ? 1 : (k == 5 ? 2 : 16));
+        }
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -428,8 +435,58 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t tY1 = tmem, tY2 = tmem + 64, tZ = tmem + 128, tS = tmem + 256, tD = tmem + 320;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
 
-    if (tid == kFwdIss) {
-        // ---------------- the issuer; the n-th iteration is chunk NC - 1 - n, stage n % 2
+    // the issuers' waits: a wait that gives up flags the abort; later waits are skipped
+    bool ok = true;
+    int err = 0;
+    auto iwait = [&](uint64_t* bar, uint32_t parity, int e) {
+        if (ok && !mbar_wait_or_abort(bar, parity, s_abort)) {
+            ok = false;
+            err = e;
+            *s_abort = 1;
+        }
+    };
+    if (tid == kBwdChain) {
+        // ---------------- the chain's UMMAs; the n-th iteration is chunk NC - 1 - n, stage n % 2
+        for (int n = 0; n < NC; ++n) {
+            const int s = n % kBStages;
+            const uint32_t par = n & 1;
+            iwait(bar_s, par, kErrTimeoutMma);  // dS'^T of chunk c is in TMEM
+            iwait(&bar_ld[s], (n / kBStages) & 1, kErrTimeoutTma);
+            if (ok) {
+                tc_fence_after();
+                const uint32_t kt = smem_u32(sm + L::Kt + s * kTile);
+                constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)  // dS'^T K^T
+                    mma_bf16_ts(tY1, tS + 8 * ks, sdesc(kt + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id,
+                                ks > 0);
+            }
+            mma_commit(bar_y);
+            iwait(bar_q, par, kErrTimeoutMma);  // Q of chunk c scaled by gamma
+            if (ok) {
+                tc_fence_after();
+                const uint32_t dob = smem_u32(sm + L::dO + s * kTile), qb = smem_u32(sm + L::Q + s * kTile);
+                constexpr uint32_t id = idesc_bf16(128, 128, true, true);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)  // dO^T (diag(gamma) Q)
+                    mma_bf16(tZ, sdesc(dob + ks * 2048, 8192, 1024), sdesc(qb + ks * 2048, 8192, 1024), id, ks > 0);
+            }
+            iwait(bar_d, par, kErrTimeoutMma);  // -dDelta^T in TMEM
+            if (ok && kDelta) {
+                tc_fence_after();
+                const uint32_t wt = smem_u32(sm + L::Wt + s * kTile);
+                constexpr uint32_t id = idesc_bf16(128, 128, false, false);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)  // - dDelta^T W
+                    mma_bf16_ts(tZ, tD + 8 * ks, sdesc(wt + ks * 32, 16, 1024), id, 1);
+            }
+            mma_commit(bar_z);
+        }
+        if (!ok) atomicExch(a.err, err);
+        mma_commit(bar_fin);  // every UMMA of this thread has finished before the TMEM is freed
+        mbar_wait(bar_fin, 0);
+    } else if (tid == kBwdCopy) {
+        // ---------------- copies, stores and dO^T P
         auto issue_load = [&](int n) {
             const int c = NC - 1 - n, s = n % kBStages;
             const uint32_t bytes = 3 * kTile + 8192 + (kDelta ? kTile : 0) + 512;
@@ -444,59 +501,35 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tma_load_2d(sm + L::P + s * 8192, &tm_p, 0, (bh * NC + c) * kChunk, &bar_ld[s]);
             bulk_load(Eds + s * 128, a.Ed + ((size_t)bh * NC + c) * 128, 512, &bar_ld[s]);
         };
-        // dO^T P of iteration n into its accumulator (its tiles have landed)
-        auto issue_y2 = [&](int n) {
+        auto issue_y2 = [&](int n) {  // dO^T P of iteration n, once its tiles have landed
             const int s = n % kBStages;
-            const uint32_t dob = smem_u32(sm + L::dO + s * kTile), pb = smem_u32(sm + L::P + s * 8192);
-            constexpr uint32_t id = idesc_bf16(128, 64, true, true);
+            iwait(&bar_ld[s], (n / kBStages) & 1, kErrTimeoutTma);
+            if (ok) {
+                tc_fence_after();
+                const uint32_t dob = smem_u32(sm + L::dO + s * kTile), pb = smem_u32(sm + L::P + s * 8192);
+                constexpr uint32_t id = idesc_bf16(128, 64, true, true);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tY2, sdesc(dob + ks * 2048, 8192, 1024), sdesc(pb + ks * 2048, 8192, 1024), id, ks > 0);
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tY2, sdesc(dob + ks * 2048, 8192, 1024), sdesc(pb + ks * 2048, 8192, 1024), id,
+                             ks > 0);
+            }
+            mma_commit(bar_y2);
         };
         int issued = 0;
         for (; issued < min(kBStages, NC); ++issued) issue_load(issued);
-        bool ok = true, y2_early = false;
-        int err = 0;
-        auto wait = [&](uint64_t* bar, uint32_t parity, int e) {
-            if (ok && !mbar_wait_or_abort(bar, parity, s_abort)) {
-                ok = false;
-                err = e;
-                *s_abort = 1;
-            }
-        };
+        issue_y2(0);
         for (int n = 0; n < NC; ++n) {
-            const int c = NC - 1 - n, s = n % kBStages;
+            const int c = NC - 1 - n;
             const uint32_t par = n & 1;
-            wait(bar_s, par, kErrTimeoutMma);  // dS'^T of chunk c is in TMEM
-            // the stage of iteration n-1 is free: its products are done and the element-wise
-            // warps have handed over dS'^T of this iteration, after their last read of it
+            // the stage of iteration n-1 is free once the element-wise warps have handed over
+            // dS'^T of this iteration: the products of n-1 are done and its tiles read
+            iwait(bar_s, par, kErrTimeoutMma);
             if (ok && n >= 1 && issued < NC) {
                 issue_load(issued);
                 ++issued;
             }
-            wait(&bar_ld[s], (n / kBStages) & 1, kErrTimeoutTma);
-            if (ok) {
-                tc_fence_after();
-                if (!y2_early) issue_y2(n);
-                const uint32_t kt = smem_u32(sm + L::Kt + s * kTile);
-                constexpr uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)  // dS'^T K^T
-                    mma_bf16_ts(tY1, tS + 8 * ks, sdesc(kt + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id,
-                                ks > 0);
-            }
-            mma_commit(bar_y);
-            wait(bar_q, par, kErrTimeoutMma);  // Q of chunk c scaled by gamma
-            if (ok) {
-                tc_fence_after();
-                const uint32_t dob = smem_u32(sm + L::dO + s * kTile), qb = smem_u32(sm + L::Q + s * kTile);
-                constexpr uint32_t id = idesc_bf16(128, 128, true, true);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)  // dO^T (diag(gamma) Q)
-                    mma_bf16(tZ, sdesc(dob + ks * 2048, 8192, 1024), sdesc(qb + ks * 2048, 8192, 1024), id, ks > 0);
-            }
-            // dS'^T of chunk c to global memory, staged while the products run
-            wait(bar_sst, par, kErrTimeoutMma);
+            // dS'^T of chunk c to global memory
+            iwait(bar_sst, par, kErrTimeoutMma);
             if (ok) {
                 tma_store_2d(&tm_dsc, sm + L::St, 0, (bh * NC + c) * kD);
                 tma_store_2d(&tm_dsc, sm + L::St + kTile, 64, (bh * NC + c) * kD);
@@ -504,24 +537,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             bulk_commit();
             bulk_wait_read<1>();  // the dDelta^T (dv) store of iteration n-1 has read its tile
             if (n > 0) mbar_arrive(bar_dfree);
-            wait(bar_d, par, kErrTimeoutMma);  // -dDelta^T in TMEM; dO^T P has been read
-            if (ok && kDelta) {
-                tc_fence_after();
-                const uint32_t wt = smem_u32(sm + L::Wt + s * kTile);
-                constexpr uint32_t id = idesc_bf16(128, 128, false, false);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)  // - dDelta^T W
-                    mma_bf16_ts(tZ, tD + 8 * ks, sdesc(wt + ks * 32, 16, 1024), id, 1);
-            }
-            mma_commit(bar_z);
-            // dO^T P of the next iteration, if its tiles have already landed
-            y2_early = false;
-            if (ok && n + 1 < NC && mbar_try_wait(&bar_ld[(n + 1) % kBStages], ((n + 1) / kBStages) & 1)) {
-                tc_fence_after();
-                issue_y2(n + 1);
-                y2_early = true;
-            }
-            wait(bar_dst, par, kErrTimeoutMma);
+            // dO^T P of the next iteration once this one's has been read
+            iwait(bar_d, par, kErrTimeoutMma);
+            if (n + 1 < NC) issue_y2(n + 1);
+            iwait(bar_dst, par, kErrTimeoutMma);
             if (ok) {
                 if (kDelta) {
                     tma_store_2d(&tm_ddt, sm + L::Dst, 0, (bh * NC + c) * kD);
@@ -535,13 +554,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_arrive(bar_sfree);
         }
         if (!ok) atomicExch(a.err, err);
-        // teardown: copies still in flight land, every UMMA issued has finished and
-        // the stores have read shared memory before the CTA exits
-        if (*s_abort) {
+        // teardown: copies still in flight land, every UMMA of this thread has finished
+        // and the stores have read shared memory before the CTA exits
+        if (*s_abort)
             for (int m = 0; m < issued; ++m) mbar_wait(&bar_ld[m % kBStages], (m / kBStages) & 1);
-            mma_commit(bar_fin);
-            mbar_wait(bar_fin, 0);
-        }
+        mma_commit(bar_fin);
+        mbar_wait(bar_fin, 0);
         bulk_wait_read<0>();
     } else if (warp < 16) {
         // ---------------- the element-wise warps (`bad` warp-uniform, as in the forward pass)
@@ -610,6 +628,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             // (4) dDelta^T[j][r] = e^{G_C - G_r} (dS'^T K^T)[j][r] + (dO^T P)[j][r], r in
             // [16 part, 16 part + 16); -dDelta^T into TMEM (A operand of - dDelta^T W)
             wait(bar_y, par, kErrTimeoutMma);
+            wait(bar_y2, par, kErrTimeoutMma);
             tc_fence_after();
             float d[16];
             {
@@ -731,7 +750,7 @@ cudaError_t launch_state_bwd_tc(const Args& a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     timing_begin(KK_STATE_BWD, s);
-    kern<<<BH, kFwdThreads, smem, s>>>(tm_k, tm_do, tm_q, tm_wt, tm_p, tm_dsc, tm_ddt, tm_dv, a);
+    kern<<<BH, kBwdThreads, smem, s>>>(tm_k, tm_do, tm_q, tm_wt, tm_p, tm_dsc, tm_ddt, tm_dv, a);
     e = cudaGetLastError();
     timing_end(KK_STATE_BWD, s);
     return e;
