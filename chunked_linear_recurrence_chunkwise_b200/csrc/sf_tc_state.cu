@@ -70,10 +70,11 @@ constexpr int kStages = 3;
 // quarter p = w >> 2 of every per-row tile (16 of 64 token columns, 32 of 128
 // state columns), so each step's elementwise work is split four ways per row.
 constexpr int kThreads = 512;
-// The forward pass adds a seventeenth warp whose first thread issues the
-// copies, the UMMAs and the stores.
-constexpr int kFwdThreads = kThreads + 32;
-constexpr int kFwdIss = kThreads;
+// Both passes add two warps whose first threads issue: one the UMMAs of the
+// dependent chain, the other the copies and stores (and, in the reverse pass,
+// the products off the chain), so that neither waits on the other's issues.
+constexpr int kFwdThreads = kThreads + 64;
+constexpr int kFwdChain = kThreads, kFwdCopy = kThreads + 32;
 
 // Shared-memory carve-up (byte offsets from a 1024-byte aligned base).
 struct FwdSmem {
@@ -107,7 +108,8 @@ __device__ __forceinline__ void put_row32(uint8_t* tile, int row, int q0, const 
 // dependent chain of a chunk is therefore UMMA -> TMEM -> registers -> TMEM ->
 // UMMA; the bf16 copies of S^T and Delta^T that go to global memory are staged
 // in shared memory and stored by TMA off that chain, while the next product
-// runs.  The warps hand over through mbarriers (one arrival per warp):
+// runs, by the other issuing thread.  The warps hand over through mbarriers
+// (one arrival per element-wise warp):
 //   bar_s    S^T of chunk c in TMEM            bar_x  X^T of chunk c done (commit)
 //   bar_d    scaled Delta^T in TMEM            bar_p  P^T of chunk c done (commit)
 //   bar_sst  S^T staged for its store          bar_sfree  that store has read the tile
@@ -134,7 +136,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint64_t* bar_dst = bar_x + 5;
     uint64_t* bar_sfree = bar_x + 6;              // count 1 (the issuer)
     uint64_t* bar_dfree = bar_x + 7;
-    uint64_t* bar_fin = bar_x + 8;
+    uint64_t* bar_fin = bar_x + 8;                // count 2 (both issuers)
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
     volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
 
@@ -144,10 +146,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
     const int NC = a.NC;
 
-    if (tid == kFwdIss) {
+    if (tid == kFwdCopy) {
         for (int i = 0; i < kStages + 9; ++i) {
-            const int k = i - kStages;  // 2..5: the element-wise hand-overs
-            mbar_init(bar_ld + i, (k >= 2 && k <= 5) ? 16 : 1);
+            const int k = i - kStages;  // 2..5: the element-wise hand-overs; 8: both issuers
+            mbar_init(bar_ld + i, (k >= 2 && k <= 5) ? 16 : (k == 8 ? 2 : 1));
         }
         *s_abort = 0;
         fence_barrier_init();
@@ -160,8 +162,48 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t tX = tmem, tP = tmem + 64, tS = tmem + 192, tD = tmem + 256;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
 
-    if (tid == kFwdIss) {
-        // ---------------- the issuer
+    // the issuers' waits: a wait that gives up flags the abort; later waits are skipped
+    bool ok = true;
+    int err = 0;
+    auto iwait = [&](uint64_t* bar, uint32_t parity, int e) {
+        if (ok && !mbar_wait_or_abort(bar, parity, s_abort)) {
+            ok = false;
+            err = e;
+            *s_abort = 1;
+        }
+    };
+    if (tid == kFwdChain) {
+        // ---------------- the chain's UMMAs
+        for (int c = 0; c < NC; ++c) {
+            const int s = c % kStages;
+            const uint32_t par = c & 1;
+            iwait(&bar_ld[s], (c / kStages) & 1, kErrTimeoutTma);
+            iwait(bar_s, par, kErrTimeoutMma);  // S^T entering chunk c is in TMEM
+            if (ok && kDelta) {
+                tc_fence_after();
+                const uint32_t b0 = smem_u32(sm + L::Wt + s * kTile);
+                constexpr uint32_t id = idesc_bf16(128, 64, false, true);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_bf16_ts(tX, tS + 8 * ks, sdesc(b0 + ks * 2048, 8192, 1024), id, ks > 0);
+            }
+            mma_commit(bar_x);
+            iwait(bar_d, par, kErrTimeoutMma);  // (e^{G_C - G} Delta)^T is in TMEM
+            if (ok) {
+                tc_fence_after();
+                const uint32_t b0 = smem_u32(sm + L::Kt + s * kTile);
+                constexpr uint32_t id = idesc_bf16(128, 128, false, true);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ts(tP, tD + 8 * ks, sdesc(b0 + ks * 2048, 8192, 1024), id, ks > 0);
+            }
+            mma_commit(bar_p);
+        }
+        if (!ok) atomicExch(a.err, err);
+        mma_commit(bar_fin);  // every UMMA issued has finished before the TMEM is freed
+        mbar_wait(bar_fin, 0);
+    } else if (tid == kFwdCopy) {
+        // ---------------- copies and stores
         auto issue_load = [&](int c) {
             const int s = c % kStages;
             const uint32_t bytes = (kDelta ? kTile : 0) + 2 * kTile + 512;
@@ -174,31 +216,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         };
         int issued = 0;
         for (; issued < min(kStages, NC); ++issued) issue_load(issued);
-        bool ok = true;
-        int err = 0;
-        auto wait = [&](uint64_t* bar, uint32_t parity, int e) {
-            if (ok && !mbar_wait_or_abort(bar, parity, s_abort)) {
-                ok = false;
-                err = e;
-                *s_abort = 1;
-            }
-        };
         for (int c = 0; c < NC; ++c) {
-            const int s = c % kStages;
             const uint32_t par = c & 1;
-            wait(&bar_ld[s], (c / kStages) & 1, kErrTimeoutTma);
-            wait(bar_s, par, kErrTimeoutMma);  // S^T entering chunk c is in TMEM
-            if (ok && kDelta) {
-                tc_fence_after();
-                const uint32_t b0 = smem_u32(sm + L::Wt + s * kTile);
-                constexpr uint32_t id = idesc_bf16(128, 64, false, true);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_bf16_ts(tX, tS + 8 * ks, sdesc(b0 + ks * 2048, 8192, 1024), id, ks > 0);
+            // the stage of chunk c-1 is free once S^T of chunk c is handed over: the products
+            // of c-1 are done and the element-wise warps have read its tiles (waited before
+            // bar_dfree below lets them reach the next hand-over of S^T)
+            iwait(bar_s, par, kErrTimeoutMma);
+            if (ok && c >= 1 && issued < NC) {
+                issue_load(issued);
+                ++issued;
             }
-            mma_commit(bar_x);
             // the chunk state entering c to global memory, staged while X^T is computed
-            wait(bar_sst, par, kErrTimeoutMma);
+            iwait(bar_sst, par, kErrTimeoutMma);
             if (ok) {
                 tma_store_2d(&tm_sc, sm + L::St, 0, (bh * NC + c) * kD);
                 tma_store_2d(&tm_sc, sm + L::St + kTile, 64, (bh * NC + c) * kD);
@@ -206,36 +235,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             bulk_commit();
             bulk_wait_read<1>();  // the Delta^T store of chunk c-1 has read its tile
             if (c > 0) mbar_arrive(bar_dfree);
-            // the stage of chunk c-1 is free: its products are done and the element-wise
-            // warps have handed over S^T of chunk c, after their last read of it
-            if (ok && c >= 1 && issued < NC) {
-                issue_load(issued);
-                ++issued;
-            }
-            wait(bar_d, par, kErrTimeoutMma);  // (e^{G_C - G} Delta)^T is in TMEM
-            if (ok) {
-                tc_fence_after();
-                const uint32_t b0 = smem_u32(sm + L::Kt + s * kTile);
-                constexpr uint32_t id = idesc_bf16(128, 128, false, true);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tP, tD + 8 * ks, sdesc(b0 + ks * 2048, 8192, 1024), id, ks > 0);
-            }
-            mma_commit(bar_p);
-            wait(bar_dst, par, kErrTimeoutMma);
+            iwait(bar_dst, par, kErrTimeoutMma);
             if (ok) tma_store_2d(&tm_dt, sm + L::Dst, 0, (bh * NC + c) * kD);
             bulk_commit();
             bulk_wait_read<1>();  // the S^T store of chunk c has read its tile
             mbar_arrive(bar_sfree);
         }
         if (!ok) atomicExch(a.err, err);
-        // teardown: copies still in flight land, every UMMA issued has finished and
-        // the stores have read shared memory before the CTA exits
-        if (*s_abort) {
+        // teardown: copies still in flight land and the stores have read shared memory
+        // before the CTA exits
+        if (*s_abort)
             for (int cc = 0; cc < issued; ++cc) mbar_wait(&bar_ld[cc % kStages], (cc / kStages) & 1);
-            mma_commit(bar_fin);
-            mbar_wait(bar_fin, 0);
-        }
+        mma_commit(bar_fin);
+        mbar_wait(bar_fin, 0);
         bulk_wait_read<0>();
     } else if (warp < 16) {
         // ---------------- the element-wise warps
@@ -385,8 +397,8 @@ struct BwdSmem {
 //   bar_dst  dDelta^T (or dv) staged          read their tiles
 // TMEM (512 columns): dS'^T K^T [0, 64), dO^T P [64, 128), the dS^T update
 // [128, 256), dS'^T operand [256, 320), -dDelta^T operand [320, 352).
-constexpr int kBwdThreads = kThreads + 64;
-constexpr int kBwdChain = kThreads, kBwdCopy = kThreads + 32;
+constexpr int kBwdThreads = kFwdThreads;
+constexpr int kBwdChain = kFwdChain, kBwdCopy = kFwdCopy;
 template <bool kDelta>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     state_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_do,
