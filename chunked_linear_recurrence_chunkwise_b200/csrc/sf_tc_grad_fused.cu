@@ -344,6 +344,11 @@ __global__ void __launch_bounds__(kBlock, 1)
             }
         }
         mma_commit(&bar_c[1]);
+        if (sok) {  // dq, staged in the dW tile (rows past the piece's end are clipped)
+            tma_store_4d(&tm_dq, sm + L::Dt, 0, h, t0, b);
+            tma_store_4d(&tm_dq, sm + L::Dt + kHalf, 64, h, t0, b);
+            bulk_commit();
+        }
         // dKp = diag(beta gamma) dKhat + (E + E^T) K once E + E^T is written
         sok = sok && mbar_wait(&bar_s[3], 0);
         if (sok) {
@@ -360,6 +365,28 @@ __global__ void __launch_bounds__(kBlock, 1)
         }
     } else if (warp < 16) {
         // ---------------- the element-wise warps
+        // <S, dS'> over the two identically laid out tiles (a dG term of the last row),
+        // while the first products run
+        wait_flag(&bar_ld[2], kErrTimeoutTma);
+        wait_flag(&bar_ld[3], kErrTimeoutTma);
+        {
+            float acc = 0.f;
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+                const int off = (qq * kThreads + tid) * 16;
+                const uint4 u = *(const uint4*)(sm + L::St + off);
+                const uint4 w = *(const uint4*)(sm + L::dSt + off);
+                const uint32_t uu[4] = {u.x, u.y, u.z, u.w}, ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const float2 a2 = unpack_bf16(uu[p]), b2 = unpack_bf16(ww[p]);
+                    acc += a2.x * b2.x + a2.y * b2.y;
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            if (lane == 0) red[warp] = acc;
+        }
         wait_flag(&bar_ld[0], kErrTimeoutTma);  // G, Q, K are read below
         wait_flag(&bar_a[0], kErrTimeoutMma);
         tc_fence_after();
@@ -446,33 +473,11 @@ __global__ void __launch_bounds__(kBlock, 1)
                 P(P_VD)[r] = vd;
                 put_row(sm + L::dDt + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);  // K-major A of dA
             }
-        }        // (d) <S, dS'> over the two identically laid out tiles; last-row sum
-        wait_flag(&bar_ld[2], kErrTimeoutTma);
-        wait_flag(&bar_ld[3], kErrTimeoutTma);
-        {
-            float acc = 0.f;
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                const int off = (qq * kThreads + tid) * 16;
-                const uint4 u = *(const uint4*)(sm + L::St + off);
-                const uint4 w = *(const uint4*)(sm + L::dSt + off);
-                const uint32_t uu[4] = {u.x, u.y, u.z, u.w}, ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const float2 a2 = unpack_bf16(uu[p]), b2 = unpack_bf16(ww[p]);
-                    acc += a2.x * b2.x + a2.y * b2.y;
-                }
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                acc += __shfl_xor_sync(0xffffffffu, acc, off);
-                lastpart += __shfl_xor_sync(0xffffffffu, lastpart, off);
-            }
-            if (lane == 0) {
-                red[warp] = acc;
-                red[16 + warp] = lastpart;
-            }
         }
+        // (d) the last-row sum of e^{G_C - G_r} <K_r, (Delta dS'^T)_r>
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) lastpart += __shfl_xor_sync(0xffffffffu, lastpart, off);
+        if (lane == 0) red[16 + warp] = lastpart;
         hand_over(&bar_s[1]);
         // dKhat: dG and dbeta terms, the K-major A operand of dKhat W^T, and
         // diag(beta gamma) dKhat as the start of dKp
@@ -492,6 +497,14 @@ __global__ void __launch_bounds__(kBlock, 1)
                 for (int q = 0; q < 32; ++q) x[q] *= br * gam;
             }
             tmem_st32(c256 + lane_base + cq * 32, x);
+        }
+        {
+            // dq (lanes 0-15 of the dQ accumulator) is final: its rows into the dead dW
+            // tile for an early store
+            float x[32];
+            tmem_ld32(c128 + lane_base + cq * 32, x);
+            tmem_ld_wait();
+            if (!hi) put_row(sm + L::Dt + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);
         }
         hand_over(&bar_s[2]);
         wait_flag(&bar_c[1], kErrTimeoutMma);
@@ -548,10 +561,8 @@ __global__ void __launch_bounds__(kBlock, 1)
             csp[g * 64 + col] = s;
         }
         hand_over(&bar_s[3]);
-        wait_flag(&bar_c[2], kErrTimeoutMma);
-        tc_fence_after();
-        named_sync(1, kThreads);  // the per-row partial sums of every warp
-        // ---------------- epilogue
+        named_sync(1, kThreads);  // the per-row partial sums and column sums of every warp
+        // ---------------- epilogue: dg and dbeta while (E + E^T) K runs, then dk
         if (warp == 0) {  // dG and dg = reverse in-chunk cumsum
             float sdot = 0.f, last = 0.f;
 #pragma unroll
@@ -590,26 +601,23 @@ __global__ void __launch_bounds__(kBlock, 1)
                 a.dbeta[tok_index(a, b, t0 + rr, h)] = db;
             }
         }
-        if (warp < 16) {
-            // dq (lanes 0-15) and dk = dK + dKp (lanes 16-31), columns [32 cq, 32 cq + 32)
+        wait_flag(&bar_c[2], kErrTimeoutMma);
+        tc_fence_after();
+        {
+            // dk = dK (lanes 16-31 of the dQ / dK accumulator) + dKp (lanes 0-15), columns
+            // [32 cq, 32 cq + 32), into the U^T tile (read by now)
             float x[32], y[32];
             tmem_ld32(c128 + lane_base + cq * 32, x);
             tmem_ld32(c256 + lane_base + cq * 32, y);  // lanes 0-15: dKp
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const float kp = __shfl_xor_sync(0xffffffffu, y[q], 16);
-                if (hi) x[q] += kp;
-            }
-            // dq rows into the W^T tile, dk rows into the U^T tile (both read by now)
-            put_row(sm + (hi ? L::Ut : L::Wt) + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);
+            for (int q = 0; q < 32; ++q) x[q] += __shfl_xor_sync(0xffffffffu, y[q], 16);
+            if (hi) put_row(sm + L::Ut + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);
         }
         fence_async_smem();
     }
     __syncthreads();
     if (tid == kIss && !*s_abort) {  // rows past the piece's end are clipped by the stores
-        tma_store_4d(&tm_dq, sm + L::Wt, 0, h, t0, b);
-        tma_store_4d(&tm_dq, sm + L::Wt + kHalf, 64, h, t0, b);
         tma_store_4d(&tm_dk, sm + L::Ut, 0, h, t0, b);
         tma_store_4d(&tm_dk, sm + L::Ut + kHalf, 64, h, t0, b);
         bulk_commit();
