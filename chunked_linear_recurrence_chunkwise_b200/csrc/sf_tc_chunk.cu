@@ -155,6 +155,9 @@ __global__ void __launch_bounds__(kIntraThreads)
         const int r0 = 2 * lane, r1 = r0 + 1;
         const float g0 = (a.g && r0 < Lr) ? a.g[tok_index(a, b, t0 + r0, h)] : 0.f;
         const float g1 = (a.g && r1 < Lr) ? a.g[tok_index(a, b, t0 + r1, h)] : 0.f;
+        // beta is read here too, so that both loads are in flight together
+        const float b0 = (kDelta && r0 < Lr) ? a.beta[tok_index(a, b, t0 + r0, h)] : 0.f;
+        const float b1 = (kDelta && r1 < Lr) ? a.beta[tok_index(a, b, t0 + r1, h)] : 0.f;
         float incl = g0 + g1;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -173,8 +176,6 @@ __global__ void __launch_bounds__(kIntraThreads)
         ed[r1] = __expf(gC - G1);
         ed[64 + r0] = e0;
         ed[64 + r1] = e1;
-        const float b0 = (kDelta && r0 < Lr) ? a.beta[tok_index(a, b, t0 + r0, h)] : 0.f;
-        const float b1 = (kDelta && r1 < Lr) ? a.beta[tok_index(a, b, t0 + r1, h)] : 0.f;
         Bs[r0] = b0;
         Bs[r1] = b1;
         BGs[r0] = b0 * e0;

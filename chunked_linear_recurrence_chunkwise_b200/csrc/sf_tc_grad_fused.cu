@@ -248,7 +248,6 @@ __global__ void __launch_bounds__(kBlock, 1)
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
                 mma_bf16(c0, sdesc(q + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);  // Q K^T
-                mma_bf16(c64, sdesc(k + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);  // K K^T
             }
             ok = mbar_wait(&bar_ld[1], 0);
         }
@@ -294,6 +293,13 @@ __global__ void __launch_bounds__(kBlock, 1)
                          idMK2, ks > 0);  // T^T dDelta
         }
         mma_commit(&bar_a[2]);
+        if (ok) {  // K K^T, first read after dA: behind every product the element-wise stages wait on
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
+                mma_bf16(c64, sdesc(k + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);
+            }
+        }
         // F K and F^T Q accumulate onto the rescaled dO S^T / Delta dS'^T once the
         // element-wise warps have written F and rescaled those ((a), (b))
         bool sok = ok && mbar_wait(&bar_s[0], 0);
