@@ -169,10 +169,11 @@ def kernel_units(name: str, w, mode: str = "keep") -> dict:
 # workload (2048 chunk-heads), from the committed ncu captures of the current kernels
 # (profiles/<kernel>_gdn_bf16_h32.md); per launch they scale with the chunk-heads covered.
 NCU_TRAFFIC_2048 = {
-    "grad_fused": 504.110e6,
-    "state_bwd": 222.702e6,
-    "state_fwd": 162.303e6,
-    "intra_bwd": 158.974e6,
+    # refreshed from the committed captures whenever a kernel changes; None until then
+    "grad_fused": None,
+    "state_bwd": None,
+    "state_fwd": None,
+    "intra_bwd": None,
     "output": 167.309e6,  # output_p_tc_kernel (the keep form)
 }
 
@@ -205,7 +206,7 @@ def roofline(timing: dict, w, steps: int, peaks: dict, peaks_src: str, clocks: d
     obj = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
            "frac": round(gbs / hbm, 4),
            "traffic": (round(NCU_TRAFFIC_2048[name] * units_per_launch / 2048)
-                       if (tc_path(w) and mode == "keep" and name in NCU_TRAFFIC_2048) else None),
+                       if (tc_path(w) and mode == "keep" and NCU_TRAFFIC_2048.get(name)) else None),
            "kernel": name, "launches": launches, "avg_launch_ms": round(ms / launches, 4),
            "bytes_per_launch": int(u["bytes"] * units_per_launch),
            "tensor_tflops": round(tfs, 2), "tensor_frac": round(tfs / bf16, 4),
@@ -351,20 +352,24 @@ def run_sf(args, w, rank, world, local_rank):
     dS_in = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
     keep = torch.empty(sf.sf_keep_bytes(sh, lens), dtype=torch.uint8, device=dev)
 
-    def step(src, serial=False, mode=None):
+    outs_main = {"o": o, "dq": dq, "dk": dk, "dv": dv, "S_out": S_out, "dS_in": dS_in, "dg": dg,
+                 "dbeta": db}
+
+    def step(src, serial=False, mode=None, out=None):
         sa = main if serial else aux
+        r = out or outs_main
         if (mode or args.mode) == "keep":
-            sf.sf_fwd_seq_keep(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], None, o,
-                               S_out, keep, ws_f, stream_main=main, stream_aux=sa)
+            sf.sf_fwd_seq_keep(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], None, r["o"],
+                               r["S_out"], keep, ws_f, stream_main=main, stream_aux=sa)
             sf.sf_bwd_seq_keep(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], keep,
-                               src["dO"], None, dq, dk, dv, dg, db, dS_in, ws_b, stream_main=main,
-                               stream_aux=sa)
+                               src["dO"], None, r["dq"], r["dk"], r["dv"], r["dg"], r["dbeta"], r["dS_in"],
+                               ws_b, stream_main=main, stream_aux=sa)
             return
-        sf.sf_fwd_seq(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], None, o, S_out,
-                      S_saved, ws_f, stream_main=main, stream_aux=sa)
+        sf.sf_fwd_seq(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], None, r["o"],
+                      r["S_out"], S_saved, ws_f, stream_main=main, stream_aux=sa)
         sf.sf_bwd_seq(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], S_saved,
-                      src["dO"], None, dq, dk, dv, dg, db, dS_in, ws_b, stream_main=main,
-                      stream_aux=sa)
+                      src["dO"], None, r["dq"], r["dk"], r["dv"], r["dg"], r["dbeta"], r["dS_in"], ws_b,
+                      stream_main=main, stream_aux=sa)
 
     def barrier():
         if world > 1:
@@ -425,30 +430,53 @@ def run_sf(args, w, rank, world, local_rank):
     timing = sf.sf_timing_read()
     launches = sum(v[0] for v in timing.values()) // max(1, args.steps)
 
-    # ---- end to end: pinned host inputs -> device -> fwd+bwd -> results back to host
+    # ---- end to end: pinned host inputs -> device -> fwd+bwd -> results back to host.
+    # Every step copies its inputs in and its results out inside the timed region; the
+    # copies run on their own streams with two device buffer sets, so that the inputs of
+    # step k+1 cross PCIe while the results of step k travel the other way (the two
+    # directions of the link and the two copy engines work at once), as a host-fed
+    # training loop would pipeline them.
     e2e = None
     if not args.no_e2e:
-        outs_h = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-                  for n, t in [("o", o), ("dq", dq), ("dk", dk), ("dv", dv), ("S_out", S_out),
-                               ("dS_in", dS_in)] + ([("dg", dg)] if dg is not None else [])
-                  + ([("dbeta", db)] if db is not None else [])}
-        outs_d = {"o": o, "dq": dq, "dk": dk, "dv": dv, "S_out": S_out, "dS_in": dS_in, "dg": dg,
-                  "dbeta": db}
+        names_out = ["o", "dq", "dk", "dv", "S_out", "dS_in"] + (["dg"] if dg is not None else []) \
+            + (["dbeta"] if db is not None else [])
+        outs_h = {n: torch.empty(outs_main[n].shape, dtype=outs_main[n].dtype, pin_memory=True)
+                  for n in names_out}
+        xs = [x, {n: (None if t is None else torch.empty_like(t)) for n, t in x.items()}]
+        outs = [outs_main, {n: (None if t is None else torch.empty_like(t)) for n, t in outs_main.items()}]
         h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
         d2h = sum(t.numel() * t.element_size() for t in outs_h.values())
-        e2e_steps = max(1, min(args.steps, 5))
+        e2e_steps = max(2, args.steps)
+        copy_in = torch.cuda.Stream(device=dev)
+        copy_out = torch.cuda.Stream(device=dev)
+        ev = lambda: torch.cuda.Event()
+        ev_in, ev_comp, ev_out = [ev(), ev()], [ev(), ev()], [ev(), ev()]
         barrier()
         torch.cuda.synchronize()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(main)
-        with torch.cuda.stream(main):
-            for _ in range(e2e_steps):
+        copy_in.wait_event(f0)
+        copy_out.wait_event(f0)
+        for k_ in range(e2e_steps):
+            b_ = k_ % 2
+            if k_ >= 2:
+                copy_in.wait_event(ev_comp[b_])  # step k-2 has finished reading this input set
+                main.wait_event(ev_out[b_])      # and its results in this set have left
+            with torch.cuda.stream(copy_in):
                 for n_, t in host.items():
                     if t is not None:
-                        x[n_].copy_(t, non_blocking=True)
-                step(x)
-                for n_, t in outs_h.items():
-                    t.copy_(outs_d[n_], non_blocking=True)
+                        xs[b_][n_].copy_(t, non_blocking=True)
+            ev_in[b_].record(copy_in)
+            main.wait_event(ev_in[b_])
+            step(xs[b_], out=outs[b_])
+            ev_comp[b_].record(main)
+            copy_out.wait_event(ev_comp[b_])
+            with torch.cuda.stream(copy_out):
+                for n_ in names_out:
+                    outs_h[n_].copy_(outs[b_][n_], non_blocking=True)
+            ev_out[b_].record(copy_out)
+        main.wait_event(ev_out[(e2e_steps - 1) % 2])
+        main.wait_event(ev_out[e2e_steps % 2])
         f1.record(main)
         torch.cuda.synchronize()
         barrier()
