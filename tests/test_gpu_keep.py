@@ -28,6 +28,9 @@ CASES = [
     ("bf16", 128, 128, [64, 100, 45]),
     ("bf16", 128, 128, [1, 64, 128, 16]),
     ("bf16", 128, 128, [64] * 9 + [100]),  # more pieces than workspace slots
+    # long pieces (dozens of chunks per state pass), a ragged last chunk; one piece
+    ("bf16", 128, 128, [64, 2048 + 17]),
+    ("bf16", 128, 128, [4096 + 3 * 64]),
     ("bf16", 64, 64, [130, 70]),
     ("f32", 64, 64, [64, 100, 45]),
     ("f32", 128, 128, [200]),
