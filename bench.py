@@ -169,11 +169,10 @@ def kernel_units(name: str, w, mode: str = "keep") -> dict:
 # workload (2048 chunk-heads), from the committed ncu captures of the current kernels
 # (profiles/<kernel>_gdn_bf16_h32.md); per launch they scale with the chunk-heads covered.
 NCU_TRAFFIC_2048 = {
-    # refreshed from the committed captures whenever a kernel changes; None until then
-    "grad_fused": None,
-    "state_bwd": None,
-    "state_fwd": None,
-    "intra_bwd": None,
+    "grad_fused": 504.724e6,
+    "state_bwd": 225.645e6,
+    "state_fwd": 162.909e6,
+    "intra_bwd": 154.866e6,
     "output": 167.309e6,  # output_p_tc_kernel (the keep form)
 }
 
