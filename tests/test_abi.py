@@ -138,3 +138,22 @@ def test_product_path_does_not_reference_the_oracle():
                 text = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in text and "from oracle" not in text, fn
                 assert "sf_oracle" not in text and "sfo_" not in text, fn
+
+
+def test_sequence_accumulation_memory_is_flat_in_T(sf):
+    """The memory property of Sequence Accumulation (atlas.scime.ai page, Key
+    results: device memory stays constant as the context grows) at the layer: with
+    pieces of a fixed length, the recompute drivers' workspace does not grow with
+    T, while the buffer of the drivers that keep the intermediates grows in
+    proportion to T."""
+    for dtype, d in ((sf.SF_BF16, 128), (sf.SF_F32, 64)):
+        ws, keep = {}, {}
+        for n in (4, 16, 64):
+            sh = sf.shape(1, 4096 * n, 32, d, d, dtype)
+            lens = [4096] * n
+            ws[n] = (sf.sf_seq_workspace_bytes(sh, lens, sf.SF_OP_FWD),
+                     sf.sf_seq_workspace_bytes(sh, lens, sf.SF_OP_BWD))
+            keep[n] = sf.sf_keep_bytes(sh, lens)
+        assert ws[4] == ws[16] == ws[64]
+        assert keep[16] == 4 * keep[4] and keep[64] == 16 * keep[4]
+        assert ws[64][1] < keep[64] / 8
