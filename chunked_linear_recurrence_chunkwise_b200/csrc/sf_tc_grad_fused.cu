@@ -19,15 +19,16 @@
 // The UMMAs are all M = 64, their accumulators paired at TMEM lane offsets 0
 // and 16 (rows 16 w + l of the lane-0 tile sit in lanes 32 w + l, those of the
 // lane-16 tile in lanes 32 w + 16 + l):
-//   cols [0, 64):    Q K^T          | dO Delta^T, later dA
-//   cols [64, 128):  K K^T          | -
+//   cols [0, 64):    Q K^T          | dA
+//   cols [64, 128):  dO Delta^T     | -      (with [128, 256) lanes 0-15: one N = 192 product)
 //   cols [128, 256): dQ             | dK
 //   cols [256, 384): dW, dKhat, dKp | dVhat
+//   cols [384, 448): K K^T          | -
 // Shared memory of operands that die early is reused for the later tiles and
 // scratch (about 218 KB in all, one CTA per SM).
 //
 // One thread of a seventeenth warp issues the copies and every UMMA, each as
-// soon as its operands are in place: the products of loaded tiles as their six
+// soon as its operands are in place: the products of loaded tiles as their five
 // copy groups land (committed in three groups), F K and F^T Q once F is
 // written, T^T dW and dVhat U^T once dW and dVhat are, dKhat W^T once dKhat
 // is, (E + E^T) K once E is.  Sixteen warps share the element-wise work (warp
@@ -53,7 +54,7 @@ constexpr int kHalf = 8192;
 constexpr int kThreads = 512;          // element-wise warps 0-15
 constexpr int kBlock = kThreads + 32;  // + the issuing warp
 constexpr int kIss = kThreads;         // the thread that issues copies and UMMAs
-constexpr int kLoads = 6;              // operand groups, in the order they are needed
+constexpr int kLoads = 5;              // operand groups, in the order they are needed
 
 // Per-row partial sums, each kept per column quarter: [term][quarter][64 rows].
 enum PartTerm {
@@ -76,9 +77,10 @@ struct FusedSmem {
     static constexpr int Ut = Wt + kTile;         // U^T [128 j][64 r]
     static constexpr int Tb = Ut + kTile;         // T [r'][64 r]
     static constexpr int F = Tb + kHalf;          // F = dP .* Gamma [r][64 t]; later E + E^T
-    static constexpr int Dt = F + kHalf;          // Delta^T [128 j][64 t]; later dW (bf16 [iblk][r][64])
-    static constexpr int dDt = Dt + kTile;        // dDelta^T [128 j][64 r]; later dVhat (bf16)
-    static constexpr int St = dDt + kTile;        // S^T [2][128 j][64 i]; later dKhat (bf16)
+    static constexpr int dDt = F + kHalf;         // dDelta^T [128 j][64 r]; later dVhat (bf16)
+    static constexpr int Dt = dDt + kTile;        // Delta^T [128 j][64 t]; later dW (bf16 [iblk][r][64])
+    static constexpr int St = Dt + kTile;         // S^T [2][128 j][64 i] (right behind Delta^T: one
+                                                  // N = 192 operand [Delta^T | S^T]); later dKhat
     static constexpr int dSt = St + 2 * kTile;    // dS'^T [2][128 j][64 i]; later E (fp32 [64][65])
     static constexpr int PD = dSt + 2 * kTile;    // fp32 [64][65]: dP .* P, then + dB .* B
     static constexpr int Gs = PD + 64 * 65 * 4;   // 64 fp32
@@ -171,27 +173,25 @@ __global__ void __launch_bounds__(kBlock, 1)
         tma_load_4d(sm + L::K, &tm_k, 0, h, t0, b, &bar_ld[0]);
         tma_load_4d(sm + L::K + kHalf, &tm_k, 64, h, t0, b, &bar_ld[0]);
         bulk_load(Gs, a.G + (size_t)bh * TP + t0, 256, &bar_ld[0]);
-        // 1: dO, Delta^T (dO Delta^T)
-        mbar_expect_tx(&bar_ld[1], 2 * kHalf + kTile);
+        // 1: dO, Delta^T, S^T (dO [Delta^T | S^T])
+        mbar_expect_tx(&bar_ld[1], 2 * kHalf + 3 * kTile);
         tma_load_4d(sm + L::dO, &tm_do, 0, h, t0, b, &bar_ld[1]);
         tma_load_4d(sm + L::dO + kHalf, &tm_do, 64, h, t0, b, &bar_ld[1]);
         tma_load_2d(sm + L::Dt, &tm_dt, 0, rowD, &bar_ld[1]);
-        // 2: S^T (dO S^T)
+        tma_load_2d(sm + L::St, &tm_sc, 0, rowD, &bar_ld[1]);
+        tma_load_2d(sm + L::St + kTile, &tm_sc, 64, rowD, &bar_ld[1]);
+        // 2: dS'^T (Delta dS'^T)
         mbar_expect_tx(&bar_ld[2], 2 * kTile);
-        tma_load_2d(sm + L::St, &tm_sc, 0, rowD, &bar_ld[2]);
-        tma_load_2d(sm + L::St + kTile, &tm_sc, 64, rowD, &bar_ld[2]);
-        // 3: dS'^T (Delta dS'^T)
-        mbar_expect_tx(&bar_ld[3], 2 * kTile);
-        tma_load_2d(sm + L::dSt, &tm_dsc, 0, rowD, &bar_ld[3]);
-        tma_load_2d(sm + L::dSt + kTile, &tm_dsc, 64, rowD, &bar_ld[3]);
-        // 4: dDelta^T, T (dDelta S^T, T^T dDelta)
-        mbar_expect_tx(&bar_ld[4], kTile + kHalf);
-        tma_load_2d(sm + L::dDt, &tm_ddt, 0, rowD, &bar_ld[4]);
-        tma_load_2d(sm + L::Tb, &tm_t, 0, rowC, &bar_ld[4]);
-        // 5: W^T, U^T (dVhat U^T, dKhat W^T)
-        mbar_expect_tx(&bar_ld[5], 2 * kTile);
-        tma_load_2d(sm + L::Wt, &tm_wt, 0, rowD, &bar_ld[5]);
-        tma_load_2d(sm + L::Ut, &tm_ut, 0, rowD, &bar_ld[5]);
+        tma_load_2d(sm + L::dSt, &tm_dsc, 0, rowD, &bar_ld[2]);
+        tma_load_2d(sm + L::dSt + kTile, &tm_dsc, 64, rowD, &bar_ld[2]);
+        // 3: dDelta^T, T (dDelta S^T, T^T dDelta)
+        mbar_expect_tx(&bar_ld[3], kTile + kHalf);
+        tma_load_2d(sm + L::dDt, &tm_ddt, 0, rowD, &bar_ld[3]);
+        tma_load_2d(sm + L::Tb, &tm_t, 0, rowC, &bar_ld[3]);
+        // 4: W^T, U^T (dVhat U^T, dKhat W^T)
+        mbar_expect_tx(&bar_ld[4], 2 * kTile);
+        tma_load_2d(sm + L::Wt, &tm_wt, 0, rowD, &bar_ld[4]);
+        tma_load_2d(sm + L::Ut, &tm_ut, 0, rowD, &bar_ld[4]);
     }
     if (warp == 0) tmem_alloc(s_tmem, 512);
     if (tid < 64) Bs[tid] = (tid < Lr) ? a.beta[tok_index(a, b, t0 + tid, h)] : 0.f;
@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(kBlock, 1)
     const uint32_t tmem = *s_tmem;
     const uint32_t l16 = 16u << 16;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    const uint32_t c0 = tmem, c64 = tmem + 64, c128 = tmem + 128, c256 = tmem + 256;
+    const uint32_t c0 = tmem, c64 = tmem + 64, c128 = tmem + 128, c256 = tmem + 256, c384 = tmem + 384;
 
     // Element-wise warps: a wait that gives up flags the abort (checked before the
     // final stores); every warp passes every barrier whatever happened, so that no
@@ -252,26 +252,18 @@ __global__ void __launch_bounds__(kBlock, 1)
             ok = mbar_wait(&bar_ld[1], 0);
         }
         if (ok) {
+            // dO [Delta^T | S^T]: one N = 192 product, dO Delta^T into columns [64, 128) and
+            // dO S^T into [128, 256) of lanes 0-15 (Delta^T and S^T lie 16 KB apart in smem)
             tc_fence_after();
+            constexpr uint32_t idKM3 = idesc_bf16(64, 192, false, true);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
-                mma_bf16(c0 + l16, sdesc(dob + o, 16, 1024), sdesc(dt + ks * 2048, kHalf, 1024), idKM,
-                         ks > 0);  // dO Delta^T
+                mma_bf16(c64, sdesc(dob + o, 16, 1024), sdesc(dt + ks * 2048, kTile, 1024), idKM3, ks > 0);
             }
         }
         mma_commit(&bar_a[0]);
         if (ok) ok = mbar_wait(&bar_ld[2], 0);
-        if (ok) {
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
-                mma_bf16(c128, sdesc(dob + o, 16, 1024), sdesc(st + ks * 2048, kTile, 1024), idKM2,
-                         ks > 0);  // dO S^T
-            }
-            ok = mbar_wait(&bar_ld[3], 0);
-        }
         if (ok) {
             tc_fence_after();
 #pragma unroll
@@ -280,7 +272,7 @@ __global__ void __launch_bounds__(kBlock, 1)
                          idMM2, ks > 0);  // Delta dS'^T
         }
         mma_commit(&bar_a[1]);
-        if (ok) ok = mbar_wait(&bar_ld[4], 0);
+        if (ok) ok = mbar_wait(&bar_ld[3], 0);
         if (ok) {
             tc_fence_after();
 #pragma unroll
@@ -297,7 +289,7 @@ __global__ void __launch_bounds__(kBlock, 1)
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
-                mma_bf16(c64, sdesc(k + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);
+                mma_bf16(c384, sdesc(k + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);
             }
         }
         // F K and F^T Q accumulate onto the rescaled dO S^T / Delta dS'^T once the
@@ -327,7 +319,7 @@ __global__ void __launch_bounds__(kBlock, 1)
         }
         mma_commit(&bar_c[0]);
         const bool sok_pre5 = sok;
-        const bool ok5 = sok && mbar_wait(&bar_ld[5], 0);  // W^T, U^T
+        const bool ok5 = sok && mbar_wait(&bar_ld[4], 0);  // W^T, U^T
         if (ok5) {
             tc_fence_after();
             const uint32_t ut = smem_u32(sm + L::Ut);
@@ -373,8 +365,8 @@ __global__ void __launch_bounds__(kBlock, 1)
         // ---------------- the element-wise warps
         // <S, dS'> over the two identically laid out tiles (a dG term of the last row),
         // while the first products run
+        wait_flag(&bar_ld[1], kErrTimeoutTma);
         wait_flag(&bar_ld[2], kErrTimeoutTma);
-        wait_flag(&bar_ld[3], kErrTimeoutTma);
         {
             float acc = 0.f;
 #pragma unroll
@@ -398,21 +390,23 @@ __global__ void __launch_bounds__(kBlock, 1)
         tc_fence_after();
         const float Gr = Gs[r];
         float rowpart;
-        // (a) P, dP, F on columns [16 cq, 16 cq + 16): lane l < 16 holds (Q K^T)[r], lane
-        // l + 16 (dO Delta^T)[r]; after one exchange each finishes 8 columns (the low
-        // lane the first 8, the high lane the last 8)
+        // (a) P, dP, F on columns [16 cq, 16 cq + 16): lane l < 16 holds (Q K^T)[r] and
+        // (dO Delta^T)[r]; it finishes the first 8 columns and hands the last 8 to
+        // lane l + 16
         {
-            float v[16];
-            tmem_ld16(c0 + lane_base + cq * 16, v);
+            float v[16], u[16];
+            tmem_ld16(c0 + lane_base + cq * 16, v);   // lanes 0-15: Q K^T
+            tmem_ld16(c64 + lane_base + cq * 16, u);  // lanes 0-15: dO Delta^T
             tmem_ld_wait();
             const int tb = 16 * cq + (hi ? 8 : 0);
             float rowsum = 0.f;
             float f[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                const float recv = __shfl_xor_sync(0xffffffffu, hi ? v[q] : v[8 + q], 16);
-                const float qk = hi ? recv : v[q];
-                const float dp = hi ? v[8 + q] : recv;
+                const float rq = __shfl_xor_sync(0xffffffffu, v[8 + q], 16);
+                const float rd = __shfl_xor_sync(0xffffffffu, u[8 + q], 16);
+                const float qk = hi ? rq : v[q];
+                const float dp = hi ? rd : u[q];
                 const int t = tb + q;
                 const float gam = (t <= r) ? __expf(Gr - Gs[t]) : 0.f;
                 const float pd = gam * qk * dp;
@@ -520,7 +514,7 @@ __global__ void __launch_bounds__(kBlock, 1)
             // holds (K K^T)[r], lane l + 16 dA[r]; each finishes 8 columns as in (a)
             float va[16], vb[16];
             tmem_ld16(c0 + lane_base + cq * 16, va);   // lanes 16-31: dA (before the sign)
-            tmem_ld16(c64 + lane_base + cq * 16, vb);  // lanes 0-15: K K^T
+            tmem_ld16(c384 + lane_base + cq * 16, vb);  // lanes 0-15: K K^T
             tmem_ld_wait();
             const int tb = 16 * cq + (hi ? 8 : 0);
             const float Gr = Gs[r], br = Bs[r];

@@ -126,8 +126,8 @@ __global__ void __launch_bounds__(128, 1)
 extern "C" int umma_probe(const void* A, const void* B, void* C, int M, int N, int K, int a_mn,
                           int b_mn, int neg_a, int lane16, int restore, int a_tmem, void* err,
                           void* stream) {
-    if (!(M == 64 || M == 128) || N % 32 || N > 128 || K % 64 || K > 128 || (lane16 && M != 64) ||
-        (a_tmem && M != 128))
+    if (!(M == 64 || M == 128) || N % 32 || N > 256 || K % 64 || K > 128 || (lane16 && M != 64) ||
+        (a_tmem && M != 128) || K * N * 2 > 32768)
         return 1;
     const int smem = 65536 + 64 + 1024;
     cudaFuncSetAttribute(umma_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -44,6 +44,13 @@ def test_m64_lane_offset_and_tmem_store(probe, lane16, restore, a_mn, b_mn):
     run_probe(probe, 64, 128, 128, a_mn, b_mn, 0, lane16, restore)
 
 
+@pytest.mark.parametrize("M", [64, 128])
+@pytest.mark.parametrize("b_mn", [0, 1])
+def test_umma_n192(probe, M, b_mn):
+    """N = 192: three 64-column blocks of B (MN-major: at a uniform block stride)."""
+    run_probe(probe, M, 192, 64, 0, b_mn, 0, 0, 0)
+
+
 @pytest.mark.parametrize("N", [64, 128])
 @pytest.mark.parametrize("K", [64, 128])
 @pytest.mark.parametrize("b_mn", [0, 1])
