@@ -502,8 +502,9 @@ struct OutSmem {
     static constexpr int St = K + kTile;       // S^T [kblk][128 j][64]
     static constexpr int Dt = St + 2 * kTile;  // Delta^T [128 j][64 r]
     static constexpr int Pb = Dt + kTile;      // P, K-major [r][64 i]
-    static constexpr int Gs = Pb + kHalf;
-    static constexpr int Bar = Gs + 256;
+    static constexpr int Gs = Pb + kHalf;      // G
+    static constexpr int Eg = Gs + 256;        // e^{G_r}, from the chunk's decay table
+    static constexpr int Bar = Eg + 256;
     static constexpr int Misc = Bar + 16;
     static constexpr int Size = Misc + 16;
 };
@@ -516,6 +517,7 @@ __global__ void __launch_bounds__(128)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     float* Gs = (float*)(sm + L::Gs);
+    const float* Eg = (const float*)(sm + L::Eg);
     uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);
     uint64_t* bar_mma = bar_ld + 1;
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
@@ -531,7 +533,7 @@ __global__ void __launch_bounds__(128)
         mbar_init(bar_mma, 1);
         *s_abort = 0;
         fence_barrier_init();
-        mbar_expect_tx(bar_ld, 2 * kTile + 2 * kTile + kTile + 256);
+        mbar_expect_tx(bar_ld, 2 * kTile + 2 * kTile + kTile + 512);
         tma_load_4d(sm + L::Q, &tm_q, 0, h, t0, b, bar_ld);
         tma_load_4d(sm + L::Q + kHalf, &tm_q, 64, h, t0, b, bar_ld);
         tma_load_4d(sm + L::K, &tm_k, 0, h, t0, b, bar_ld);
@@ -540,6 +542,7 @@ __global__ void __launch_bounds__(128)
         tma_load_2d(sm + L::St + kTile, &tm_sc, 64, (bh * NC + c) * kD, bar_ld);
         tma_load_2d(sm + L::Dt, &tm_dt, 0, (bh * NC + c) * kD, bar_ld);
         bulk_load(Gs, a.G + (size_t)bh * TP + t0, 256, bar_ld);
+        bulk_load(sm + L::Eg, a.Ed + ((size_t)bh * NC + c) * 128 + 64, 256, bar_ld);
     }
     if (warp == 0) tmem_alloc(s_tmem, 256);
     tc_fence_before();
@@ -625,7 +628,7 @@ __global__ void __launch_bounds__(128)
         const uint32_t jb = (uint32_t)(j >> 6) * kHalf, jq = (j & 63) >> 3, je = (j & 7) * 2;
 #pragma unroll
         for (int r = 0; r < 64; ++r) {
-            const float o = __expf(Gs[r]) * x2[r] + x3[r];
+            const float o = Eg[r] * x2[r] + x3[r];
             *(__nv_bfloat16*)(ost + jb + sw128(r, jq) + je) = __float2bfloat16_rn(o);
         }
     }
@@ -659,8 +662,8 @@ struct OutPSmem {
     static constexpr int St = Q + kTile;       // S^T [kblk][128 j][64]
     static constexpr int Dt = St + 2 * kTile;  // Delta^T [128 j][64 r]
     static constexpr int Pb = Dt + kTile;      // P, K-major [r][64 i]
-    static constexpr int Gs = Pb + kHalf;
-    static constexpr int Bar = Gs + 256;
+    static constexpr int Eg = Pb + kHalf;      // e^{G_r}, from the chunk's decay table
+    static constexpr int Bar = Eg + 256;
     static constexpr int Misc = Bar + 16;
     static constexpr int Size = Misc + 16;
 };
@@ -672,14 +675,14 @@ __global__ void __launch_bounds__(128)
     using L = OutPSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    float* Gs = (float*)(sm + L::Gs);
+    const float* Eg = (const float*)(sm + L::Eg);
     uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);
     uint64_t* bar_mma = bar_ld + 1;
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
     volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
 
     const int c = blockIdx.x, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
-    const int NC = a.NC, TP = NC * kChunk;
+    const int NC = a.NC;
     const int t0 = c * kChunk;
     const int tid = threadIdx.x, warp = tid >> 5;
 
@@ -695,7 +698,7 @@ __global__ void __launch_bounds__(128)
         tma_load_2d(sm + L::St + kTile, &tm_sc, 64, (bh * NC + c) * kD, bar_ld);
         tma_load_2d(sm + L::Dt, &tm_dt, 0, (bh * NC + c) * kD, bar_ld);
         tma_load_2d(sm + L::Pb, &tm_p, 0, (bh * NC + c) * kChunk, bar_ld);
-        bulk_load(Gs, a.G + (size_t)bh * TP + t0, 256, bar_ld);
+        bulk_load(sm + L::Eg, a.Ed + ((size_t)bh * NC + c) * 128 + 64, 256, bar_ld);
     }
     if (warp == 0) tmem_alloc(s_tmem, 128);
     tc_fence_before();
@@ -744,7 +747,7 @@ __global__ void __launch_bounds__(128)
         const uint32_t jb = (uint32_t)(j >> 6) * kHalf, jq = (j & 63) >> 3, je = (j & 7) * 2;
 #pragma unroll
         for (int r = 0; r < 64; ++r) {
-            const float o = __expf(Gs[r]) * x2[r] + x3[r];
+            const float o = Eg[r] * x2[r] + x3[r];
             *(__nv_bfloat16*)(ost + jb + sw128(r, jq) + je) = __float2bfloat16_rn(o);
         }
     }
