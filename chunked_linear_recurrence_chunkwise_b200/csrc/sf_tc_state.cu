@@ -14,11 +14,13 @@
 // which is S' = gamma_C S + Ktil^T Delta with the decay moved from K onto
 // Delta (Ktil^T Delta = K^T diag(e^{G_C - G}) Delta), so K feeds the tensor
 // core straight from its TMA tile.  S^T is rounded to bf16 only as an MMA
-// operand (and for the stored chunk states); the carried state stays fp32.
+// operand, which the element-wise warps write into TMEM (and for the stored
+// chunk states); the carried state stays fp32 in registers.
 //
-// Per chunk c the kernel stores S^T entering c and Delta^T (both bf16) for
-// the output and gradient kernels.  W^T, U^T, K and the cumulative log-decay
-// of chunk c+1.. are prefetched by TMA into a 3-stage ring while chunk c runs.
+// Per chunk c the forward pass stores S^T entering c and Delta^T (both bf16)
+// for the output and gradient kernels; W^T, U^T, K and the decay table of the
+// chunks ahead are prefetched by TMA into a 3-stage ring.  The reverse pass
+// (further down) mirrors it with a 2-stage ring.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -76,7 +78,7 @@ constexpr int kThreads = 512;
 constexpr int kFwdThreads = kThreads + 64;
 constexpr int kFwdChain = kThreads, kFwdCopy = kThreads + 32;
 
-// Shared-memory carve-up (byte offsets from a 1024-byte aligned base).
+// Shared-memory carve-up of the forward pass (byte offsets from a 1024-byte aligned base).
 struct FwdSmem {
     static constexpr int Wt = 0;                          // [stage] W^T  [d_k][64 r]
     static constexpr int Kt = Wt + kStages * kTile;       // [stage] K    [2][64 r][64 d_k]
