@@ -177,6 +177,29 @@ NCU_TRAFFIC_2048 = {
 }
 
 
+def kernel_rooflines(timing: dict, w, steps: int, peaks: dict, mode: str = "keep") -> dict:
+    """Every kernel of the serialized pass: launches and time per step, and per launch
+    its algorithmic bandwidth and tensor throughput with their fractions of the
+    measured peaks (HBM copy bandwidth; sustained bf16 GEMM rate)."""
+    chunk_heads = w.B * w.H * ((w.T + 63) // 64)
+    units_per_launch = chunk_heads / w.n_sub
+    hbm = float(peaks["hbm_gbs"])
+    bf16 = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1590.0)))
+    out = {}
+    for name, (launches, ms) in timing.items():
+        if launches <= 0:
+            continue
+        u = kernel_units(name, w, mode)
+        per_launch_s = ms / 1e3 / launches
+        gbs = u["bytes"] * units_per_launch / per_launch_s / 1e9
+        tfs = u["flops"] * units_per_launch / per_launch_s / 1e12
+        out[name] = {"launches": launches // max(1, steps), "ms_per_step": round(ms / steps, 4),
+                     "us_per_launch": round(per_launch_s * 1e6, 1), "gbs": round(gbs, 1),
+                     "hbm_frac": round(gbs / hbm, 4), "tflops": round(tfs, 2),
+                     "tensor_frac": round(tfs / bf16, 4)}
+    return out
+
+
 def roofline(timing: dict, w, steps: int, peaks: dict, peaks_src: str, clocks: dict,
              mode: str = "keep"):
     """Roofline object of the kernel with the largest total time (serialized pass).
@@ -511,9 +534,7 @@ def run_sf(args, w, rank, world, local_rank):
             "gpu_launches": launches,
             "e2e": e2e,
             "roofline": roofline(timing, w, args.steps, peaks, src, clocks, args.mode),
-            "kernels": {k_: {"launches": v[0] // max(1, args.steps),
-                             "ms_per_step": round(v[1] / args.steps, 4)} for k_, v in timing.items()
-                        if v[0] > 0},
+            "kernels": kernel_rooflines(timing, w, args.steps, peaks, args.mode),
             "kernel_timing": "serialized pass (driver streams merged), CUDA events per launch",
             "cpu_baseline": cpu,
         }
