@@ -123,7 +123,9 @@ __global__ void __launch_bounds__(kIntraThreads)
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
     volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
 
-    const int c = blockIdx.x, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+    int c, bh;
+    cta_chunk_head<kP>(c, bh);  // batch-heads fastest in the form that keeps P: measured faster
+    const int b = bh / a.H, h = bh % a.H;
     const int NC = a.NC, TP = NC * kChunk;
     const int t0 = c * kChunk, Lr = min(kChunk, a.T - t0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;

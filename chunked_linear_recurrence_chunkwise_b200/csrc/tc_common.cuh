@@ -241,6 +241,23 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
         : "memory");
 }
 
+// (chunk, batch-head) of this CTA in a (chunks, batch-heads) grid.  With
+// kHeadFastest the CTAs are numbered in launch order with the batch-head fastest:
+// the CTAs resident at once then cover every head of a few chunks, and their
+// token-major loads ([B, T, H, d]) take whole token rows instead of one head's
+// 256 bytes from many rows.  Otherwise the chunk is fastest.
+template <bool kHeadFastest>
+__device__ __forceinline__ void cta_chunk_head(int& c, int& bh) {
+    if (kHeadFastest) {
+        const int BH = (int)gridDim.y, n = (int)(blockIdx.y * gridDim.x + blockIdx.x);
+        c = n / BH;
+        bh = n - c * BH;
+    } else {
+        c = (int)blockIdx.x;
+        bh = (int)blockIdx.y;
+    }
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
                                             uint64_t* bar) {
