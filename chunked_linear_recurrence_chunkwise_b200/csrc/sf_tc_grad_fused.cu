@@ -84,8 +84,7 @@ struct FusedSmem {
     static constexpr int dSt = St + 2 * kTile;    // dS'^T [2][128 j][64 i]; later E (fp32 [64][65])
     static constexpr int PD = dSt + 2 * kTile;    // fp32 [64][65]: dP .* P, then + dB .* B
     static constexpr int Gs = PD + 64 * 65 * 4;   // 64 fp32
-    static constexpr int Bs = Gs + 256;           // 64 fp32
-    static constexpr int csp = Bs + 256;          // fp32 [8][64]: column sums of PD over 8-row groups
+    static constexpr int csp = Gs + 256;          // fp32 [8][64]: column sums of PD over 8-row groups
     static constexpr int part = csp + 8 * 256;    // fp32 [P_COUNT][4][64]
     static constexpr int red = part + P_COUNT * 4 * 256;  // fp32 [32]: per-warp <S, dS'>, last-row sums
     static constexpr int Bar = red + 128;         // kLoads + 11 mbarriers
@@ -138,7 +137,6 @@ __global__ void __launch_bounds__(kBlock, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     float* Gs = (float*)(sm + L::Gs);
-    float* Bs = (float*)(sm + L::Bs);
     float* csp = (float*)(sm + L::csp);
     float* PD = (float*)(sm + L::PD);
     float* Ef = (float*)(sm + L::dSt);
@@ -194,7 +192,9 @@ __global__ void __launch_bounds__(kBlock, 1)
         tma_load_2d(sm + L::Ut, &tm_ut, 0, rowD, &bar_ld[4]);
     }
     if (warp == 0) tmem_alloc(s_tmem, 512);
-    if (tid < 64) Bs[tid] = (tid < Lr) ? a.beta[tok_index(a, b, t0 + tid, h)] : 0.f;
+    // beta of this thread's row, held in a register: a load consumed before the
+    // block-wide barrier below would hold the issuer's first products back
+    const float bpre = (warp < 16 && r < Lr) ? a.beta[tok_index(a, b, t0 + r, h)] : 0.f;
     // this thread's quarter of V's row r (lanes 16-31), read while the tiles load
     uint4 vpre[4] = {};
     if (warp < 16 && hi && r < Lr) {
@@ -452,7 +452,7 @@ __global__ void __launch_bounds__(kBlock, 1)
                 for (int q = 0; q < 32; ++q) x[q] = -x[q];
                 put_row(sm + L::Dt + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);  // MN-major B of T^T dW
             } else {
-                const float br = Bs[r];
+                const float br = bpre;
                 float vd = 0.f;
                 uint4 ov[4];
 #pragma unroll
@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(kBlock, 1)
             tmem_ld32(c256 + lane_base + cq * 32, x);  // lanes 0-15: dKhat
             tmem_ld_wait();
             if (!hi) {
-                const float gam = __expf(Gs[r]), br = Bs[r];
+                const float gam = __expf(Gs[r]), br = bpre;
                 const float kd = dot_row32(sm + L::K + (cq >> 1) * kHalf, r, (cq & 1) * 4, x);
                 P(P_GK)[r] = gam * kd;
                 P(P_BGK)[r] = br * gam * kd;
@@ -517,7 +517,7 @@ __global__ void __launch_bounds__(kBlock, 1)
             tmem_ld16(c384 + lane_base + cq * 16, vb);  // lanes 0-15: K K^T
             tmem_ld_wait();
             const int tb = 16 * cq + (hi ? 8 : 0);
-            const float Gr = Gs[r], br = Bs[r];
+            const float Gr = Gs[r], br = bpre;
             float sab = 0.f, sbb = 0.f;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
