@@ -169,10 +169,10 @@ def kernel_units(name: str, w, mode: str = "keep") -> dict:
 # workload (2048 chunk-heads), from the committed ncu captures of the current kernels
 # (profiles/<kernel>_gdn_bf16_h32.md); per launch they scale with the chunk-heads covered.
 NCU_TRAFFIC_2048 = {
-    "grad_fused": 504.866e6,
+    "grad_fused": 505.206e6,
     "state_bwd": 225.645e6,
     "state_fwd": 162.909e6,
-    "intra_bwd": 154.866e6,
+    "intra_bwd": 156.399e6,
     "output": 168.811e6,  # output_p_tc_kernel (the keep form)
 }
 
