@@ -392,8 +392,19 @@ __global__ void __launch_bounds__(kBlock, 1)
         float rowpart;
         // (a) P, dP, F on columns [16 cq, 16 cq + 16): lane l < 16 holds (Q K^T)[r] and
         // (dO Delta^T)[r]; it finishes the first 8 columns and hands the last 8 to
-        // lane l + 16
-        {
+        // lane l + 16.  A warp whose columns all lie past its rows (cq > quad) writes
+        // the zeros without reading the products.
+        if (cq > quad) {
+            const int tb = 16 * cq + (hi ? 8 : 0);
+            float f[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                PD[r * 65 + tb + q] = 0.f;
+                f[q] = 0.f;
+            }
+            put_row(sm + L::F, r, tb >> 3, f, 8);
+            rowpart = 0.f;
+        } else {
             float v[16], u[16];
             tmem_ld16(c0 + lane_base + cq * 16, v);   // lanes 0-15: Q K^T
             tmem_ld16(c64 + lane_base + cq * 16, u);  // lanes 0-15: dO Delta^T
@@ -511,35 +522,46 @@ __global__ void __launch_bounds__(kBlock, 1)
         tc_fence_after();
         {
             // B, dA, dB .* B (added onto PD), E on columns [16 cq, 16 cq + 16): lane l < 16
-            // holds (K K^T)[r], lane l + 16 dA[r]; each finishes 8 columns as in (a)
-            float va[16], vb[16];
-            tmem_ld16(c0 + lane_base + cq * 16, va);   // lanes 16-31: dA (before the sign)
-            tmem_ld16(c384 + lane_base + cq * 16, vb);  // lanes 0-15: K K^T
-            tmem_ld_wait();
-            const int tb = 16 * cq + (hi ? 8 : 0);
-            const float Gr = Gs[r], br = bpre;
-            float sab = 0.f, sbb = 0.f;
+            // holds (K K^T)[r], lane l + 16 dA[r]; each finishes 8 columns as in (a).  A
+            // warp whose columns all lie past its rows has B = dA = 0 there: E = 0, PD as is.
+            if (cq > quad) {
+                const int tb = 16 * cq + (hi ? 8 : 0);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float recv = __shfl_xor_sync(0xffffffffu, hi ? va[q] : vb[8 + q], 16);
-                const float kk = hi ? recv : vb[q];
-                const float dar = hi ? va[8 + q] : recv;
-                const int t = tb + q;
-                const bool lower = t < r;
-                const float gam = lower ? __expf(Gr - Gs[t]) : 0.f;
-                const float bv = gam * kk;
-                const float da = lower ? -dar : 0.f;
-                sab += da * bv;
-                const float dbb = br * da * bv;
-                sbb += dbb;
-                PD[r * 65 + t] += dbb;  // the same thread wrote dP .* P here in (a)
-                Ef[r * 65 + t] = br * da * gam;
-            }
-            sab += __shfl_xor_sync(0xffffffffu, sab, 16);
-            sbb += __shfl_xor_sync(0xffffffffu, sbb, 16);
-            if (!hi) {
-                P(P_SAB)[r] = sab;
-                P(P_SBB)[r] = sbb;
+                for (int q = 0; q < 8; ++q) Ef[r * 65 + tb + q] = 0.f;
+                if (!hi) {
+                    P(P_SAB)[r] = 0.f;
+                    P(P_SBB)[r] = 0.f;
+                }
+            } else {
+                float va[16], vb[16];
+                tmem_ld16(c0 + lane_base + cq * 16, va);   // lanes 16-31: dA (before the sign)
+                tmem_ld16(c384 + lane_base + cq * 16, vb);  // lanes 0-15: K K^T
+                tmem_ld_wait();
+                const int tb = 16 * cq + (hi ? 8 : 0);
+                const float Gr = Gs[r], br = bpre;
+                float sab = 0.f, sbb = 0.f;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float recv = __shfl_xor_sync(0xffffffffu, hi ? va[q] : vb[8 + q], 16);
+                    const float kk = hi ? recv : vb[q];
+                    const float dar = hi ? va[8 + q] : recv;
+                    const int t = tb + q;
+                    const bool lower = t < r;
+                    const float gam = lower ? __expf(Gr - Gs[t]) : 0.f;
+                    const float bv = gam * kk;
+                    const float da = lower ? -dar : 0.f;
+                    sab += da * bv;
+                    const float dbb = br * da * bv;
+                    sbb += dbb;
+                    PD[r * 65 + t] += dbb;  // the same thread wrote dP .* P here in (a)
+                    Ef[r * 65 + t] = br * da * gam;
+                }
+                sab += __shfl_xor_sync(0xffffffffu, sab, 16);
+                sbb += __shfl_xor_sync(0xffffffffu, sbb, 16);
+                if (!hi) {
+                    P(P_SAB)[r] = sab;
+                    P(P_SBB)[r] = sbb;
+                }
             }
         }
         named_sync(1, kThreads);  // PD and E of every row
