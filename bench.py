@@ -169,7 +169,7 @@ def kernel_units(name: str, w, mode: str = "keep") -> dict:
 # workload (2048 chunk-heads), from the committed ncu captures of the current kernels
 # (profiles/<kernel>_gdn_bf16_h32.md); per launch they scale with the chunk-heads covered.
 NCU_TRAFFIC_2048 = {
-    "grad_fused": None,  # changed since its capture
+    "grad_fused": 507.538e6,
     "state_bwd": 225.645e6,
     "state_fwd": 162.909e6,
     "intra_bwd": 156.399e6,
