@@ -23,6 +23,12 @@ class sf_shape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("B", "T", "H", "dk", "dv", "chunk", "dtype", "ld_t")]
 
 
+class sf_chunk_costs(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_double) for n in ("intra_us", "output_us", "grad_us", "state_fwd_us",
+                                               "state_bwd_us")] + [("sms", ctypes.c_int),
+                                                                   ("min_chunks", ctypes.c_int)]
+
+
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libsf.so is not built ({LIB_PATH}); run "
                       "`python -m chunked_linear_recurrence_chunkwise_b200.build`")
@@ -53,6 +59,8 @@ _SIGS = {
                             ctypes.POINTER(ctypes.c_double)]),
     "sf_timing_trace": (_I, [_I, _IP, _IP, ctypes.POINTER(ctypes.c_double),
                              ctypes.POINTER(ctypes.c_double)]),
+    "sf_model_seq_us": (ctypes.c_double, [_SP, _I, _IP, ctypes.POINTER(sf_chunk_costs)]),
+    "sf_plan_cut": (_I, [_SP, _I, ctypes.POINTER(sf_chunk_costs), _IP]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -222,3 +230,23 @@ def sf_timing_trace(cap: int = 4096) -> list:
 def raw_call(name: str, *args):
     """Calls a C entry point with already-marshalled arguments (tests of the error paths)."""
     return getattr(_lib, name)(*args)
+
+
+def chunk_costs(intra_us, output_us, grad_us, state_fwd_us, state_bwd_us, sms,
+                min_chunks=0) -> sf_chunk_costs:
+    """Per-chunk kernel costs (microseconds for one 64-token chunk of all heads) for the planner."""
+    return sf_chunk_costs(float(intra_us), float(output_us), float(grad_us), float(state_fwd_us),
+                          float(state_bwd_us), int(sms), int(min_chunks))
+
+
+def sf_model_seq_us(sh: sf_shape, lens, costs: sf_chunk_costs) -> float:
+    us = float(_lib.sf_model_seq_us(ctypes.byref(sh), len(lens), _lens(lens), ctypes.byref(costs)))
+    if us < 0:
+        raise SfError(SF_ERR_INVALID, "sf_model_seq_us")
+    return us
+
+
+def sf_plan_cut(sh: sf_shape, n_sub: int, costs: sf_chunk_costs) -> list:
+    out = (ctypes.c_int * int(n_sub))()
+    _check(_lib.sf_plan_cut(ctypes.byref(sh), int(n_sub), ctypes.byref(costs), out), "sf_plan_cut")
+    return [int(x) for x in out]

@@ -206,6 +206,43 @@ int sf_timing_read(int cap, const char** names, int* launches, double* ms);
  * later sf_timing_read still totals them).  Returns the number written. */
 int sf_timing_trace(int cap, int* kinds, int* streams, double* start_ms, double* end_ms);
 
+/* Profile-guided cut into sub-sequences (host code; no GPU is touched).
+ *
+ * The StateFlow pages choose nonuniform block lengths from a profile of the
+ * kernels so that the sequential state passes and the parallel per-block work
+ * pipeline with fewer bubbles (StateFlow (newx.sg), Abstract; StateFlow
+ * (gptget.net), 术语表 and 方法详解).  sf_chunk_costs holds a profile: the
+ * microseconds one 64-token chunk of all B x H heads costs in each kernel of the
+ * drivers that keep the forward's intermediates, the parallel kernels measured
+ * on the whole GPU, the state passes with one CTA per batch-head, and the SM
+ * count.  Every field must be >= 0 and sms > 0.  The model counts work, not the
+ * tail of a launch's last wave of CTAs; min_chunks keeps the planner away from
+ * pieces so short that those tails dominate. */
+typedef struct {
+    double intra_us;      /* intra-chunk kernel (storing P and T), whole GPU */
+    double output_us;     /* output kernel, whole GPU */
+    double grad_us;       /* per-chunk gradient kernel(s), whole GPU */
+    double state_fwd_us;  /* forward state pass */
+    double state_bwd_us;  /* reverse (dS) pass */
+    int sms;              /* SMs of the GPU */
+    int min_chunks;       /* shortest piece sf_plan_cut may choose, in 64-token chunks (0: one) */
+} sf_chunk_costs;
+
+/* Modelled device time (microseconds) of sf_fwd_seq_keep followed by
+ * sf_bwd_seq_keep for the cut `lens` (host array of n_sub positive lengths
+ * summing to shape->T): the two streams of the drivers replayed with the
+ * state pass holding min(B*H, sms) SMs and the parallel kernels sharing the
+ * rest.  Returns -1 for invalid arguments. */
+double sf_model_seq_us(const sf_shape* shape, int n_sub, const int* lens, const sf_chunk_costs* costs);
+
+/* Writes to lens_out (host array of n_sub ints) a cut of shape->T tokens into
+ * n_sub pieces, each a multiple of 64 tokens except that a ragged last chunk
+ * shortens the last piece, chosen to minimise sf_model_seq_us: the even cut, or
+ * one whose last pieces ramp up geometrically from a short last piece (the
+ * backward starts with the last piece's reverse pass alone).  SF_ERR_INVALID
+ * for NULL pointers, invalid costs, T <= 0 or n_sub outside [1, ceil(T/64)]. */
+sf_status sf_plan_cut(const sf_shape* shape, int n_sub, const sf_chunk_costs* costs, int* lens_out);
+
 #ifdef __cplusplus
 }
 #endif

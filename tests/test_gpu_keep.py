@@ -98,3 +98,30 @@ def test_keep_backward_is_repeatable(layer):
     for key in ("dq", "dk", "dv", "dg", "dbeta", "dS_in"):
         assert torch.equal(g1[key], g2[key]), key
     assert np.isfinite(host(g1["dq"])).all()
+
+
+def test_planned_cut_gives_the_single_pass_result(layer):
+    """The profile-guided cut (sf_plan_cut) is a cut like any other: the keep
+    drivers on it give the single-pass result (fp32 state carry, chunk-aligned
+    cuts: to 1e-5 on the bf16 tensor-core path, as for any cut)."""
+    from chunked_linear_recurrence_chunkwise_b200 import sf
+    B, T, H = 1, 2560 + 17, 4
+    c = make_case(41, B, T, H, 128, 128, True, True, "bf16")
+    d = to_dev(c, "bf16")
+    sh = sf.shape_of(d["q"], d["v"])
+    costs = sf.chunk_costs(65.7 / 64, 38.5 / 64, 160.4 / 64, 106.9 / 64, 136.1 / 64, 148, 2)
+    plan = sf.sf_plan_cut(sh, 5, costs)
+    assert len(set(plan)) > 1 and sum(plan) == T
+    aux = torch.cuda.Stream()
+    res = []
+    for lens in ([T], plan):
+        o, S_out, kept = layer.forward_keep(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S_in"],
+                                            lens=lens, aux_stream=aux)
+        gr = layer.backward_keep(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], kept,
+                                 dS_out=d["dS_out"], lens=lens, aux_stream=aux)
+        torch.cuda.synchronize()
+        res.append({"o": host(o), "S_out": host(S_out), **{k_: host(gr[k_]) for k_ in
+                                                           ("dq", "dk", "dv", "dg", "dbeta", "dS_in")}})
+    errs = {k_: rel_l2(res[1][k_], res[0][k_]) for k_ in res[0]}
+    bad = {k_: e for k_, e in errs.items() if not e <= 1e-5}
+    assert not bad, f"planned cut vs single pass: {bad} (all {errs})"
