@@ -47,6 +47,9 @@ def parse_args(argv=None):
     p.add_argument("--no-other-mode", action="store_true",
                    help="do not time the other driver form beside the headline one")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--memory-study", default=None, metavar="T1,T2,...",
+                   help="instead of the bench line: the layer's device memory and step time for these "
+                        "sequence lengths at a fixed piece length of 4096 tokens (one JSON line)")
     p.add_argument("--no-plan", action="store_true",
                    help="skip timing the profile-guided cut (sf_plan_cut) beside the workload's own cut")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -349,6 +352,13 @@ def run_reference(args, w, rank, world):
 
 
 # ------------------------------------------------------------------ GPU arm
+def workspace(torch, nbytes: int, dev):
+    """A library workspace: its head (the device error word) starts zeroed."""
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    ws[:min(nbytes, 256)].zero_()
+    return ws
+
+
 def plan_costs(sf, timing: dict, steps: int, n_chunks: int, sms: int, bh: int):
     """Per-chunk costs (us for one 64-token chunk of all heads) from the serialized
     per-kernel timing of `steps` steps of the keep drivers over n_chunks chunks."""
@@ -372,8 +382,8 @@ def time_planned_cut(args, sf, torch, sh, lens, x, timing, dev, main, aux, outs)
                                   "grad": round(costs.grad_us, 4), "state_fwd": round(costs.state_fwd_us, 4),
                                   "state_bwd": round(costs.state_bwd_us, 4), "sms": sms,
                                   "min_chunks": costs.min_chunks}}
-    ws_f = torch.empty(sf.sf_seq_workspace_bytes(sh, plan, sf.SF_OP_FWD), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(sf.sf_seq_workspace_bytes(sh, plan, sf.SF_OP_BWD), dtype=torch.uint8, device=dev)
+    ws_f = workspace(torch, sf.sf_seq_workspace_bytes(sh, plan, sf.SF_OP_FWD), dev)
+    ws_b = workspace(torch, sf.sf_seq_workspace_bytes(sh, plan, sf.SF_OP_BWD), dev)
     keep = torch.empty(sf.sf_keep_bytes(sh, plan), dtype=torch.uint8, device=dev)
 
     def step():
@@ -415,8 +425,8 @@ def run_sf(args, w, rank, world, local_rank):
     torch.cuda.synchronize()
     B, T, H, d = wr.B, wr.T, wr.H, wr.d
     sh = sf.shape_of(x["q"], x["v"])
-    ws_f = torch.empty(sf.sf_seq_workspace_bytes(sh, lens, sf.SF_OP_FWD), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(sf.sf_seq_workspace_bytes(sh, lens, sf.SF_OP_BWD), dtype=torch.uint8, device=dev)
+    ws_f = workspace(torch, sf.sf_seq_workspace_bytes(sh, lens, sf.SF_OP_FWD), dev)
+    ws_b = workspace(torch, sf.sf_seq_workspace_bytes(sh, lens, sf.SF_OP_BWD), dev)
     main = torch.cuda.Stream(device=dev)
     aux = torch.cuda.Stream(device=dev)
     o = torch.empty_like(x["v"])
@@ -604,6 +614,87 @@ def run_sf(args, w, rank, world, local_rank):
     return 0
 
 
+def run_memory_study(args, w):
+    """Device memory the layer needs beside its inputs and outputs, against T at a fixed
+    piece length (Sequence Accumulation, Key results: memory flat in the sequence length).
+
+    For each T the workload's variant, heads and head size are kept and the sequence is
+    cut into pieces of 4096 tokens.  Per driver form: the bytes the caller allocates for
+    the layer (workspaces, plus the saved piece states of the recompute form or the kept
+    intermediates of the keep form), the change of free device memory across a
+    fwd+bwd call (the library allocates nothing itself), and the device time of one
+    fwd+bwd after a warm-up.  Inputs are drawn on the device with the workload's value
+    distributions (their values do not change the memory)."""
+    import torch
+    import torch.nn.functional as F
+    from chunked_linear_recurrence_chunkwise_b200 import sf
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    rows = []
+    for T in [int(x) for x in args.memory_study.split(",")]:
+        lens = [4096] * (T // 4096) + ([T % 4096] if T % 4096 else [])
+        gen = torch.Generator(device=dev).manual_seed(w.seed)
+        rn = lambda *shape: torch.randn(*shape, device=dev, generator=gen)
+        B, H, d = w.B, w.H, w.d
+        q, k = F.normalize(rn(B, T, H, d), dim=-1).to(dt), F.normalize(rn(B, T, H, d), dim=-1).to(dt)
+        v, dO = rn(B, T, H, d).to(dt), rn(B, T, H, d).to(dt)
+        g = (-0.1 * F.softplus(rn(B, T, H))) if w.has_g else None
+        beta = torch.sigmoid(rn(B, T, H)) if w.has_beta else None
+        o, dq, dk, dv = (torch.empty_like(v) for _ in range(4))
+        dg = None if g is None else torch.empty_like(g)
+        db = None if beta is None else torch.empty_like(beta)
+        S_out = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+        dS_in = torch.empty_like(S_out)
+        sh = sf.shape_of(q, v)
+        main_s, aux_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        row = {"T": T, "n_sub": len(lens)}
+        for form in ("recompute", "keep"):
+            ws_f = workspace(torch, sf.sf_seq_workspace_bytes(sh, lens, sf.SF_OP_FWD), dev)
+            ws_b = workspace(torch, sf.sf_seq_workspace_bytes(sh, lens, sf.SF_OP_BWD), dev)
+            if form == "keep":
+                extra = torch.empty(sf.sf_keep_bytes(sh, lens), dtype=torch.uint8, device=dev)
+            else:
+                extra = torch.empty((len(lens), B, H, d, d), dtype=torch.float32, device=dev)
+
+            def step():
+                if form == "keep":
+                    sf.sf_fwd_seq_keep(sh, lens, q, k, v, g, beta, None, o, S_out, extra, ws_f,
+                                       stream_main=main_s, stream_aux=aux_s)
+                    sf.sf_bwd_seq_keep(sh, lens, q, k, v, g, beta, extra, dO, None, dq, dk, dv, dg, db,
+                                       dS_in, ws_b, stream_main=main_s, stream_aux=aux_s)
+                else:
+                    sf.sf_fwd_seq(sh, lens, q, k, v, g, beta, None, o, S_out, extra, ws_f,
+                                  stream_main=main_s, stream_aux=aux_s)
+                    sf.sf_bwd_seq(sh, lens, q, k, v, g, beta, extra, dO, None, dq, dk, dv, dg, db,
+                                  dS_in, ws_b, stream_main=main_s, stream_aux=aux_s)
+
+            torch.cuda.synchronize()
+            free0 = torch.cuda.mem_get_info(dev)[0]
+            step()
+            torch.cuda.synchronize()
+            free1 = torch.cuda.mem_get_info(dev)[0]
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(main_s)
+            step()
+            e1.record(main_s)
+            torch.cuda.synchronize()
+            sf.sf_check(ws_f, main_s)
+            sf.sf_check(ws_b, main_s)
+            row[f"{form}_layer_bytes"] = ws_f.numel() + ws_b.numel() + extra.numel() * extra.element_size()
+            row[f"{form}_free_delta_bytes"] = free0 - free1
+            row[f"{form}_ms"] = round(e0.elapsed_time(e1), 3)
+            del ws_f, ws_b, extra
+        rows.append(row)
+        del q, k, v, dO, o, dq, dk, dv, g, beta, dg, db
+        torch.cuda.empty_cache()
+    print(json.dumps({"memory_study": {"workload": w.name, "variant": w.variant, "B": w.B, "H": w.H,
+                                       "d": w.d, "dtype": w.dtype, "piece_tokens": 4096, "rows": rows}}),
+          flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     rank, world, local_rank = dist_env()
@@ -613,6 +704,8 @@ def main(argv=None):
         w = w.scaled(T=T, H=args.heads or w.H, n_sub=max(1, min(w.n_sub, T // 4096)))
     if args.impl == "reference":
         return run_reference(args, w, rank, world)
+    if args.memory_study:
+        return run_memory_study(args, w) if rank == 0 else 0
     if world > 1:
         import datetime
         import torch

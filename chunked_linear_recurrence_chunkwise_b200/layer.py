@@ -16,7 +16,9 @@ from . import sf
 def _ws(nbytes: int, device) -> torch.Tensor:
     if nbytes <= 0:
         raise sf.SfError(sf.SF_ERR_INVALID, "workspace size")
-    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    ws[:min(nbytes, 256)].zero_()  # the device error word at its head starts clear
+    return ws
 
 
 def _check_inputs(*ts):
