@@ -176,8 +176,11 @@ extern "C" sf_status sf_plan_cut(const sf_shape* shape, int n_sub, const sf_chun
     std::vector<long> cut;
     const long even = total / n_sub;
     const long lo = std::max(1, costs->min_chunks);
+    // the last piece's length: every value up to 64 chunks, then steps of ~5%
+    std::vector<long> firsts;
+    for (long f = lo; f <= even; f = std::max(f + 1, (long)(f * 1.05))) firsts.push_back(f);
     for (int m = 1; m < n_sub; ++m)
-        for (long first = lo; first <= even; ++first)
+        for (long first : firsts)
             for (int r = 0; r <= 40; ++r) {
                 const double ratio = 1.0 + 0.05 * r;
                 if (!ramp_cut(total, n_sub, m, first, ratio, cut)) continue;
