@@ -40,8 +40,12 @@ def build(force: bool = False) -> str:
 def _load():
     global _lib
     if _lib is None:
-        build()
-        lib = ctypes.CDLL(_LIB)
+        # SF_ORACLE_LIB: a build of a deliberately altered sf_oracle.c, which the tests
+        # that plant a mistake load to check that the pins catch it
+        path = os.environ.get("SF_ORACLE_LIB")
+        if not path:
+            path = build()
+        lib = ctypes.CDLL(path)
         P = ctypes.c_void_p
         I = ctypes.c_int
         lib.sfo_fwd.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, I]
