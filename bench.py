@@ -359,22 +359,12 @@ def workspace(torch, nbytes: int, dev):
     return ws
 
 
-def plan_costs(sf, timing: dict, steps: int, n_chunks: int, sms: int, bh: int):
-    """Per-chunk costs (us for one 64-token chunk of all heads) from the serialized
-    per-kernel timing of `steps` steps of the keep drivers over n_chunks chunks."""
-    def us(prefix):
-        return sum(v[1] for k_, v in timing.items() if k_.startswith(prefix)) * 1e3 / steps / n_chunks
-    # the shortest piece fills the GPU with the three-CTAs-per-SM kernels in one wave
-    min_chunks = -(-3 * sms // bh)
-    return sf.chunk_costs(us("intra"), us("output"), us("grad") + us("dd_pre"), us("state_fwd"),
-                          us("state_bwd"), sms, min_chunks)
-
-
 def time_planned_cut(args, sf, torch, sh, lens, x, timing, dev, main, aux, outs):
     """Device time of the keep drivers on the cut sf_plan_cut picks from the measured costs."""
     n_chunks = sum(-(-n // 64) for n in lens)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    costs = plan_costs(sf, timing, args.steps, n_chunks, sms, sh.B * sh.H)
+    from chunked_linear_recurrence_chunkwise_b200 import layer
+    costs = layer.chunk_costs(timing, args.steps, n_chunks, sh.B * sh.H, sms)
     plan = sf.sf_plan_cut(sh, len(lens), costs)
     res = {"lens": plan, "model_ms": round(sf.sf_model_seq_us(sh, plan, costs) / 1e3, 4),
            "model_ms_own_cut": round(sf.sf_model_seq_us(sh, lens, costs) / 1e3, 4),

@@ -118,3 +118,26 @@ def backward_keep(q, k, v, g, beta, dO, keep, dS_out=None, lens=None, stream=Non
     sf.sf_bwd_seq_keep(sh, lens, q, k, v, g, beta, keep, dO, dS_out, dq, dk_, dv_, dg, db, dS_in, ws,
                        stream_main=stream, stream_aux=aux_stream)
     return {"dq": dq, "dk": dk_, "dv": dv_, "dg": dg, "dbeta": db, "dS_in": dS_in}
+
+
+def chunk_costs(timing: dict, steps: int, n_chunks: int, bh: int, sms: int, min_chunks=None):
+    """Per-chunk kernel costs for the planner from a timing profile of the keep drivers.
+
+    ``timing`` is ``sf.sf_timing_read()`` after ``steps`` fwd+bwd steps of the keep
+    drivers run with both driver streams merged onto one stream, so that every kernel
+    is timed alone.  The steps cover ``n_chunks`` 64-token chunks of ``bh`` heads
+    (batch rows x heads).  The result holds microseconds per chunk of all heads.
+    ``min_chunks`` defaults to the chunks whose kernels fill the GPU once at three
+    CTAs per SM."""
+    def us(prefix):
+        return sum(v[1] for k_, v in timing.items() if k_.startswith(prefix)) * 1e3 / steps / n_chunks
+    if min_chunks is None:
+        min_chunks = -(-3 * sms // bh)
+    return sf.chunk_costs(us("intra"), us("output"), us("grad") + us("dd_pre"), us("state_fwd"),
+                          us("state_bwd"), sms, min_chunks)
+
+
+def plan_cut(q, v, n_sub: int, costs) -> list:
+    """The cut of q's sequence into ``n_sub`` pieces that ``sf.sf_plan_cut`` chooses for
+    these costs (host computation; the tensors give the shape only)."""
+    return sf.sf_plan_cut(sf.shape_of(q, v), n_sub, costs)

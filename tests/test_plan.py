@@ -104,3 +104,19 @@ def test_plan_rejects_invalid_arguments(sf):
         sf.sf_plan_cut(sh, 2, costs(sf, sms=0))   # no SMs
     with pytest.raises(sf.SfError):
         sf.sf_plan_cut(sf.shape(1, 0, 2, 128, 128, sf.SF_BF16), 1, costs(sf))
+
+
+def test_costs_from_a_timing_profile_and_the_layer_helpers(sf):
+    import torch
+    from chunked_linear_recurrence_chunkwise_b200 import layer
+    # a serialized profile of 2 steps over 1024 chunks of 32 heads: kernel -> (launches, total ms)
+    timing = {"intra_bwd": (32, 2 * 1.05), "state_fwd": (32, 2 * 1.7), "output": (32, 2 * 0.62),
+              "state_bwd": (32, 2 * 2.18), "grad_fused": (32, 2 * 2.57), "intra_fwd": (0, 0.0)}
+    c = layer.chunk_costs(timing, steps=2, n_chunks=1024, bh=32, sms=148)
+    assert c.intra_us == pytest.approx(1.05e3 / 1024) and c.grad_us == pytest.approx(2.57e3 / 1024)
+    assert c.state_fwd_us == pytest.approx(1.7e3 / 1024) and c.state_bwd_us == pytest.approx(2.18e3 / 1024)
+    assert c.output_us == pytest.approx(0.62e3 / 1024)
+    assert c.sms == 148 and c.min_chunks == 14  # ceil(3 * 148 / 32)
+    q = torch.empty((1, 65536, 32, 128), dtype=torch.bfloat16)
+    plan = layer.plan_cut(q, q, 16, c)
+    assert sum(plan) == 65536 and len(plan) == 16 and plan[-1] < plan[0]
