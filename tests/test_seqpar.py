@@ -88,6 +88,7 @@ def _worker(rank, world, port, cuts, micro, q_out):
 
 
 @pytest.mark.parametrize("cuts,micro", [
+    ((0, 96), 2),               # one rank: no messages, the drivers' own result
     ((0, 40, 96), 1),           # two ranks, uneven slices, one micro-batch
     ((0, 40, 96), 2),           # two ranks, two micro-batches in flight
     ((0, 17, 64, 100), 3),      # three ranks, ragged slices, three micro-batches (of 2, 1, 1 rows)
