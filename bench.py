@@ -29,8 +29,6 @@ if ROOT not in sys.path:
 from chunked_linear_recurrence_chunkwise_b200 import inputs  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
-SM_COUNT = 148
-FP32_LANES_PER_SM = 128
 
 
 # ------------------------------------------------------------------ host logic
@@ -102,106 +100,182 @@ def tc_path(w) -> bool:
     return w.dtype == "bf16" and w.d == 128
 
 
-def kernel_units(name: str, w, mode: str = "keep") -> dict:
-    """Algorithmic bytes and flops of one chunk-head (64 tokens of one head) per kernel.
+# Per token-head, with C = 64 and d = d_k = d_v: u = 2 C d and v = 2 d^2 flops.  The
+# method's algorithmic work is counted triangle-aware (a product with a causal C x C
+# factor at half its square size), step by step of the chunkwise algorithm:
+#   forward:  A = K K^T, W, U (1.5 u); state pass W S and Ktil^T Delta (2 v);
+#             output P = Q K^T and P Delta (u), Q S (v)            -> 2.5 u + 3 v
+#   backward: reverse pass P^T dO (0.5 u), Ktil dS', Qtil^T dO, W^T dDelta (3 v);
+#             gradients dP, F K, F^T Q, dKhat, dVhat, dA (two), (E + E^T) K (4.5 u),
+#             dO S^T, dDelta S^T, Delta dS'^T (3 v)                 -> 5 u + 6 v
+# (linear attention drops the delta-rule terms).  These are the canonical counts of
+# the workload's headline TFLOP/s; what a kernel issues on full tiles is reported
+# beside them.
+def canonical_flops(name: str, w) -> float:
+    """Triangle-aware algorithmic flops of one chunk-head (64 tokens of one head)
+    that kernel `name` carries, from the per-token-head counts above."""
+    C, d = 64, w.d
+    u, v = 2.0 * C * d, 2.0 * d * d
+    delta = w.has_beta
+    per_token = {
+        "intra_fwd": 1.5 * u if delta else 0.0,
+        "intra_bwd": (1.5 * u if delta else 0.0) + 0.5 * u,   # also forms P
+        "state_fwd": 2 * v if delta else v,
+        "output": u + v,
+        "output_p": 0.5 * u + v,                               # P read, not formed
+        "state_bwd": 0.5 * u + (3 * v if delta else 2 * v),
+        "grad_fused": 4.5 * u + 3 * v,
+        "grad_attn": 1.5 * u + 2 * v,
+    }.get(name, 0.0)
+    return per_token * C
 
-    Bytes count each tensor the kernel must read or write once, at the
-    precision the path stores it: on the tensor-core path q, k, v, o and the
-    gradients are bf16, intermediates (W^T, U^T, chunk states, Delta, P) bf16,
-    g, beta, the cumulative decay and the delta-rule partial dk fp32.  Flops
-    are 2 x the multiply-adds of the chunk's dense products as the kernel
-    issues them on 64 x 64 / 64 x 128 / 128 x 128 tiles.
+
+def layer_io_bytes_per_token_head(w) -> dict:
+    """The layer's own I/O per token-head (the minimum traffic of an ideally fused
+    layer): forward reads q, k, v, g, beta and writes o; backward reads q, k, v, g,
+    beta, dO and writes dq, dk, dv, dg, dbeta."""
+    e = 2 if w.dtype == "bf16" else 4
+    dk = dv = w.d
+    gb = 4 * (int(w.has_g) + int(w.has_beta))
+    fwd = (2 * dk + dv) * e + gb + dv * e
+    bwd = (2 * dk + 2 * dv) * e + gb + (2 * dk + dv) * e + gb
+    return {"fwd": fwd, "bwd": bwd, "total": fwd + bwd}
+
+
+def kernel_units(name: str, w, mode: str = "keep") -> dict:
+    """Bytes and flops of one chunk-head (64 tokens of one head) per kernel.
+
+    io_bytes: the layer I/O tensors (q, k, v, g, beta, dO read; o, dq, dk, dv, dg,
+    dbeta written) that this kernel reads or writes, each once: the kernel's share
+    of the layer's minimum traffic.  design_bytes: every tensor the kernel must read
+    or write once at the precision the path stores it, intermediates included
+    (W^T, U^T, chunk states, Delta, P, T ... in bf16 on the tensor-core path; g,
+    beta, the cumulative decay fp32).  flops: the canonical triangle-aware count
+    (canonical_flops); flops_issued: 2 x the multiply-adds of the products as the
+    kernel issues them on full tiles.
     """
     C, d = 64, w.d
     f = 4
+    gb = C * f * (int(w.has_g) + int(w.has_beta))   # g and beta of one chunk-head
+    if tc_path(w) and name == "output" and mode == "keep":
+        name = "output_p"  # the forward that keeps P runs the output kernel that reads it
     if tc_path(w):
         e = 2                       # bf16 I/O and intermediates
         tile = C * d * e            # one 64 x 128 bf16 tile: 16 KB
         st = d * d * e              # one chunk state, bf16: 32 KB
         mm = lambda m, n, k: 2 * m * n * k
+        # (io_bytes, design_bytes, issued flops)
         tab = {
-            # read k, v (+ q), g, beta; write G, W^T, U^T (+ P)
-            "intra_fwd": (2 * tile + 2 * C * f + C * f + 2 * tile,
+            # read k, v, g, beta; write G, W^T, U^T
+            "intra_fwd": (2 * tile + gb, 2 * tile + 2 * C * f + C * f + 2 * tile,
                           mm(C, C, d) + 2 * mm(d, C, C)),
             # as intra_fwd, also reading q and writing P (and T for the delta rule)
-            "intra_bwd": (3 * tile + 2 * C * f + C * f + 2 * tile
+            "intra_bwd": (3 * tile + gb, 3 * tile + 2 * C * f + C * f + 2 * tile
                           + (2 if w.has_beta else 1) * C * C * e,
                           mm(2 * C, C, d) + 2 * mm(d, C, C)),
             # read W^T, U^T, k, decay table; write S^T, Delta^T
-            "state_fwd": (3 * tile + 2 * C * f + st + tile, mm(d, C, d) + mm(d, d, C)),
+            "state_fwd": (tile, 3 * tile + 2 * C * f + st + tile, mm(d, C, d) + mm(d, d, C)),
             # read q, k, S^T, Delta^T, G; write o (P recomputed on chip)
-            "output": (2 * tile + st + tile + C * f + tile,
+            "output": (3 * tile, 2 * tile + st + tile + C * f + tile,
                        mm(C, C, d) + mm(d, C, d) + mm(d, C, C)),
             # read q, S^T, Delta^T, the stored P, G; write o
-            "output_p": (tile + st + tile + C * C * e + C * f + tile, mm(d, C, d) + mm(d, C, C)),
+            "output_p": (2 * tile, tile + st + tile + C * C * e + C * f + tile,
+                         mm(d, C, d) + mm(d, C, C)),
             # read k, dO, q, W^T, P, G; write dS'^T, dDelta^T
-            "state_bwd": (4 * tile + C * C * e + C * f + st + tile,
+            "state_bwd": (3 * tile, 4 * tile + C * C * e + C * f + st + tile,
                           mm(d, C, d) + mm(d, C, C) + 2 * mm(d, d, C)),
-            # read k, v, dDelta^T, S^T, W^T, U^T, beta, G; write dv, dbeta, dKp (fp32), dGp
-            "grad_delta": (5 * tile + st + 2 * C * f + tile + C * d * f + 2 * C * f,
-                           mm(C, C, d) + mm(C, d, d) + 2 * mm(C, d, C) + 2 * mm(C, C, d)
-                           + mm(C, d, C)),
-            # read q, k, dO, Delta^T, S^T, dS'^T, G, dKp, dGp; write dq, dk, dg
-            "grad_attn": (4 * tile + 2 * st + C * f + C * d * f + C * f + 2 * tile + C * f,
+            # read q, k, dO, Delta^T (= V^T), S^T, dS'^T, G; write dq, dk, dg
+            "grad_attn": (4 * tile + C * f + 2 * tile + C * f,
+                          4 * tile + 2 * st + C * f + 2 * tile + C * f,
                           2 * mm(C, C, d) + 2 * mm(C, d, d) + 2 * mm(C, d, C)),
-            # read q, k, v, dO, W^T, U^T, T, Delta^T, dDelta^T, S^T, dS'^T, G, beta;
+            # read q, k, v, dO, T, Delta^T, dDelta^T, S^T, dS'^T, G, beta;
             # write dq, dk, dv, dg, dbeta
-            "grad_fused": (8 * tile + C * C * e + 2 * st + 2 * C * f + 3 * tile + 2 * C * f,
-                           5 * mm(C, C, d) + 3 * mm(C, d, d) + 5 * mm(C, d, C)),
+            "grad_fused": (4 * tile + gb + 3 * tile + gb,
+                           6 * tile + C * C * e + 2 * st + 2 * C * f + 3 * tile + 2 * C * f,
+                           4 * mm(C, C, d) + 3 * mm(C, d, d) + 4 * mm(C, d, C)),
         }
     else:
         e = 2 if w.dtype == "bf16" else 4
+        t1 = C * d * e
         tri_s = C * (C - 1) // 2
         tri_i = C * (C + 1) // 2
         tab = {
-            "intra_fwd": (2 * C * d * e + 3 * C * f + 2 * C * d * e, tri_s * 2 * d * 3),
-            "state_fwd": (3 * C * d * e + C * f + d * d * e + C * d * e, 4 * C * d * d),
-            "output": (3 * C * d * e + C * f + d * d * e + C * d * e, tri_i * 4 * d + 2 * C * d * d),
-            "dd_pre": (3 * C * d * e + C * f + C * d * e, tri_i * 4 * d),
-            "state_bwd": (5 * C * d * e + C * f + d * d * e + C * d * e, 6 * C * d * d),
-            "grad_delta": (6 * C * d * e + d * d * e + C * d * f + 3 * C * f,
+            "intra_fwd": (2 * t1 + gb, 2 * C * d * e + 3 * C * f + 2 * C * d * e, tri_s * 2 * d * 3),
+            "state_fwd": (t1, 3 * C * d * e + C * f + d * d * e + C * d * e, 4 * C * d * d),
+            "output": (2 * t1, 3 * C * d * e + C * f + d * d * e + C * d * e, tri_i * 4 * d + 2 * C * d * d),
+            "dd_pre": (2 * t1, 3 * C * d * e + C * f + C * d * e, tri_i * 4 * d),
+            "state_bwd": (3 * t1, 5 * C * d * e + C * f + d * d * e + C * d * e, 6 * C * d * d),
+            "grad_delta": (2 * t1 + gb + t1 + C * f, 6 * C * d * e + d * d * e + C * d * f + 3 * C * f,
                            tri_s * 12 * d + 2 * C * d * d),
-            "grad_attn": (5 * C * d * e + 2 * d * d * e + C * d * f + 2 * C * f,
+            "grad_attn": (3 * t1 + C * f + 2 * t1 + C * f, 5 * C * d * e + 2 * d * d * e + C * d * f + 2 * C * f,
                           tri_i * 8 * d + 4 * C * d * d),
         }
-    if tc_path(w) and name == "output" and mode == "keep":
-        name = "output_p"  # the forward that keeps P runs the output kernel that reads it
-    b, fl = tab.get(name, (0, 0))
-    return {"bytes": b, "flops": fl}
+    io, design, fl = tab.get(name, (0, 0, 0))
+    return {"io_bytes": io, "design_bytes": design, "flops": canonical_flops(name, w), "flops_issued": fl}
 
 
 # DRAM bytes (read + write) per launch of one 4096-token piece of the 32-head, d = 128
-# workload (2048 chunk-heads), from the committed ncu captures of the current kernels
-# (profiles/<kernel>_gdn_bf16_h32.md); per launch they scale with the chunk-heads covered.
+# workload (2048 chunk-heads) from an ncu capture, per kernel, with the sha256 (first 16
+# hex digits) of the source file the kernel was built from at the time of the capture.
+# A kernel whose source has changed since reports traffic null.
 NCU_TRAFFIC_2048 = {
-    "grad_fused": 507.538e6,
-    "state_bwd": 225.645e6,
-    "state_fwd": 162.909e6,
-    "intra_bwd": 156.399e6,
-    "output": 168.811e6,  # output_p_tc_kernel (the keep form)
+    # name: (bytes per 2048 chunk-heads, source file, sha256[:16])
 }
+KERNEL_SOURCE = {
+    "grad_fused": "sf_tc_grad_fused.cu", "state_fwd": "sf_tc_state.cu", "state_bwd": "sf_tc_state.cu",
+    "intra_bwd": "sf_tc_chunk.cu", "intra_fwd": "sf_tc_chunk.cu", "output": "sf_tc_chunk.cu",
+    "grad_attn": "sf_tc_grad.cu",
+}
+
+
+def source_sha(fname: str) -> str | None:
+    import hashlib
+    path = os.path.join(ROOT, "chunked_linear_recurrence_chunkwise_b200", "csrc", fname)
+    try:
+        with open(path, "rb") as f:
+            return hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+
+
+def measured_traffic(name: str, units_per_launch: float, w, mode: str):
+    """DRAM bytes per launch from the committed capture, or None when there is none for
+    this kernel on this path or the kernel's source has changed since it was taken."""
+    ent = NCU_TRAFFIC_2048.get(name)
+    if not ent or not tc_path(w) or mode != "keep":
+        return None
+    nbytes, fname, sha = ent
+    if source_sha(fname) != sha:
+        return None
+    return round(nbytes * units_per_launch / 2048)
 
 
 def kernel_rooflines(timing: dict, w, steps: int, peaks: dict, mode: str = "keep") -> dict:
     """Every kernel of the serialized pass: launches and time per step, and per launch
-    its algorithmic bandwidth and tensor throughput with their fractions of the
-    measured peaks (HBM copy bandwidth; sustained bf16 GEMM rate)."""
+    its bandwidth on the layer's own I/O (io) and on everything it moves (design), and
+    its canonical and issued tensor throughput, with fractions of the measured peaks
+    (HBM copy bandwidth; burst bf16 GEMM rate: the timed pass runs well under a second
+    at full clock)."""
     chunk_heads = w.B * w.H * ((w.T + 63) // 64)
     units_per_launch = chunk_heads / w.n_sub
     hbm = float(peaks["hbm_gbs"])
-    bf16 = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1590.0)))
+    bf16 = float(peaks.get("bf16_tflops", 1590.0))
     out = {}
     for name, (launches, ms) in timing.items():
         if launches <= 0:
             continue
         u = kernel_units(name, w, mode)
         per_launch_s = ms / 1e3 / launches
-        gbs = u["bytes"] * units_per_launch / per_launch_s / 1e9
+        io = u["io_bytes"] * units_per_launch / per_launch_s / 1e9
+        des = u["design_bytes"] * units_per_launch / per_launch_s / 1e9
         tfs = u["flops"] * units_per_launch / per_launch_s / 1e12
+        tfi = u["flops_issued"] * units_per_launch / per_launch_s / 1e12
         out[name] = {"launches": launches // max(1, steps), "ms_per_step": round(ms / steps, 4),
-                     "us_per_launch": round(per_launch_s * 1e6, 1), "gbs": round(gbs, 1),
-                     "hbm_frac": round(gbs / hbm, 4), "tflops": round(tfs, 2),
-                     "tensor_frac": round(tfs / bf16, 4)}
+                     "us_per_launch": round(per_launch_s * 1e6, 1),
+                     "io_gbs": round(io, 1), "io_frac": round(io / hbm, 4),
+                     "design_gbs": round(des, 1), "design_frac": round(des / hbm, 4),
+                     "tflops": round(tfs, 2), "tensor_frac": round(tfs / bf16, 4),
+                     "tflops_issued": round(tfi, 2)}
     return out
 
 
@@ -209,37 +283,58 @@ def roofline(timing: dict, w, steps: int, peaks: dict, peaks_src: str, clocks: d
              mode: str = "keep"):
     """Roofline object of the kernel with the largest total time (serialized pass).
 
-    Every kernel of this layer moves more bytes than its arithmetic can hide
-    (about 20-60 flop/byte against a ridge near 240 flop/byte), so the bound
-    is HBM bandwidth; the tensor-pipe fraction of the same kernel is reported
-    beside it.
+    achieved = the kernel's algorithmic bytes per launch (its share of the layer's
+    own I/O, kernel_units io_bytes, x the chunk-heads one launch covers) / the
+    average launch duration, against the measured HBM copy bandwidth.  The bytes
+    it moves with the split design's intermediates (design_bytes) and its canonical
+    tensor throughput against the burst bf16 peak are reported beside it.
     """
     if not timing:
         return None
     name, (launches, ms) = max(timing.items(), key=lambda kv: kv[1][1])
     if launches == 0 or ms <= 0:
         return None
-    per_step = launches / steps
     chunk_heads = w.B * w.H * ((w.T + 63) // 64)  # per step, over all pieces
-    # every launch processes one piece (all heads, batch rows); pieces of the workload
-    # are uniform, so a launch covers chunk_heads / n_sub chunk-heads
+    # every launch processes one piece (all heads, batch rows); a launch covers
+    # chunk_heads / n_sub chunk-heads on average
     units_per_launch = chunk_heads / w.n_sub
     u = kernel_units(name, w, mode)
     per_launch_s = ms / 1e3 / launches
-    gbs = u["bytes"] * units_per_launch / per_launch_s / 1e9
+    gbs = u["io_bytes"] * units_per_launch / per_launch_s / 1e9
+    des = u["design_bytes"] * units_per_launch / per_launch_s / 1e9
     tfs = u["flops"] * units_per_launch / per_launch_s / 1e12
     hbm = float(peaks["hbm_gbs"])
-    bf16 = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1590.0)))
+    bf16 = float(peaks.get("bf16_tflops", 1590.0))
     obj = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
            "frac": round(gbs / hbm, 4),
-           "traffic": (round(NCU_TRAFFIC_2048[name] * units_per_launch / 2048)
-                       if (tc_path(w) and mode == "keep" and NCU_TRAFFIC_2048.get(name)) else None),
+           "traffic": measured_traffic(name, units_per_launch, w, mode),
            "kernel": name, "launches": launches, "avg_launch_ms": round(ms / launches, 4),
-           "bytes_per_launch": int(u["bytes"] * units_per_launch),
-           "tensor_tflops": round(tfs, 2), "tensor_frac": round(tfs / bf16, 4),
-           "peak_source": peaks_src + " (hbm_gbs; bf16_tflops_sustained for tensor_frac)",
+           "chunk_heads_per_launch": units_per_launch,
+           "bytes_per_chunk_head": u["io_bytes"],
+           "bytes_per_launch": int(u["io_bytes"] * units_per_launch),
+           "design_bytes_per_launch": int(u["design_bytes"] * units_per_launch),
+           "design_gbs": round(des, 1), "design_frac": round(des / hbm, 4),
+           "tensor_tflops": round(tfs, 2), "tensor_peak": bf16, "tensor_frac": round(tfs / bf16, 4),
+           "peak_source": peaks_src + " (hbm_gbs for bytes; bf16_tflops, burst, for tensor_frac)",
            "share_of_kernel_time": round(ms / sum(v[1] for v in timing.values()), 4)}
     return obj
+
+
+def step_roofline(w, ms: float, peaks: dict) -> dict:
+    """Whole-step figures: canonical TFLOP/s of forward + backward and the fraction of
+    the layer's HBM floor (its own I/O at the measured bandwidth) the step reaches."""
+    C = 64
+    token_heads = w.B * w.T * w.H
+    fl = sum(canonical_flops(n, w) for n in ("intra_bwd", "state_fwd", "output_p", "state_bwd",
+                                              "grad_fused" if w.has_beta else "grad_attn")) / C
+    io = layer_io_bytes_per_token_head(w)["total"]
+    hbm = float(peaks["hbm_gbs"])
+    bf16 = float(peaks.get("bf16_tflops", 1590.0))
+    s = ms / 1e3
+    return {"flops_per_token_head": fl, "tflops": round(fl * token_heads / s / 1e12, 2),
+            "tensor_frac": round(fl * token_heads / s / 1e12 / bf16, 4),
+            "io_bytes_per_token_head": io, "hbm_floor_ms": round(io * token_heads / (hbm * 1e9) * 1e3, 4),
+            "hbm_floor_frac": round(io * token_heads / s / 1e9 / hbm, 4)}
 
 
 class ClockSampler:
@@ -304,10 +399,12 @@ def summarize_clocks(lines) -> dict:
 
 
 # ------------------------------------------------------------------ oracle timing
-def time_oracle(w, heads: int, tokens: int):
-    """fp64 oracle fwd + bwd on a bounded sample of workload w; returns (tokens/s, info)."""
+def time_oracle(w, heads: int, tokens: int, nthreads: int | None = None):
+    """fp64 oracle fwd + bwd on a bounded sample of workload w: the first `tokens`
+    tokens of the first `heads` heads.  Returns (layer tokens/s, info); a layer token
+    covers all H heads, so the sample's rate is scaled by heads / H."""
     import oracle
-    cores = oracle.max_threads()
+    cores = nthreads or oracle.max_threads()
     hs = list(range(min(heads, w.H)))
     x = inputs.generate(w, 0, tokens, heads=hs, with_grad=True)
     t0 = time.perf_counter()
@@ -316,34 +413,63 @@ def time_oracle(w, heads: int, tokens: int):
     dt = time.perf_counter() - t0
     layer_tokens = w.B * tokens * len(hs) / w.H  # a layer token covers all H heads
     return layer_tokens / dt, {
-        "cores": cores, "seconds": round(dt, 3),
+        "cores": cores, "seconds": round(dt, 3), "token_heads": w.B * tokens * len(hs),
         "sample": f"B={w.B} x {tokens} tokens x {len(hs)} of {w.H} heads, fwd+bwd, fp64 token loop; "
                   f"tokens/s counts a token as all {w.H} heads",
     }
 
 
+def cpu_baseline(w, tokens: int) -> dict:
+    """The oracle on every host core over a bounded sample of all heads, plus the same
+    oracle on one thread over a smaller sample (one head per 16 of the workload's heads)."""
+    val, info = time_oracle(w, heads=w.H, tokens=tokens)
+    h1 = max(1, w.H // 16)
+    v1, info1 = time_oracle(w, heads=h1, tokens=min(tokens, 4096), nthreads=1)
+    return {"value": round(val, 3), "unit": "tokens/s", "cores": info["cores"], "kind": "oracle",
+            "sample": info["sample"], "seconds": info["seconds"],
+            "one_thread": {"value": round(v1, 3), "unit": "tokens/s", "cores": 1,
+                           "sample": info1["sample"], "seconds": info1["seconds"]}}
+
+
+def bench_config(w, lens, world: int, mode: str) -> dict:
+    """The `config` object of a bench line (the reference arm uses the same one)."""
+    return {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d": w.d, "n_sub": len(lens),
+            "chunk": 64, "variant": w.variant, "l2": "inputs larger than L2, no flush",
+            "parallelism": f"replicas{world}", "mode": mode}
+
+
 def run_reference(args, w, rank, world):
+    """The reference arm: the fp64 oracle as it stands, on this host's cores.  Each step
+    is a bounded sample (4096 tokens of as many heads as there are cores), timed; the
+    line's value is the sample's rate in layer tokens/s, ms_per_step the sample's own
+    measured time per step.  What the whole layer would take at that rate is reported
+    as an extrapolation, not as a measured time."""
     if rank != 0:
         return 0
     import oracle
     cores = oracle.max_threads()
     heads = max(1, min(w.H, cores))
     tokens = min(w.T, 4096)
-    vals = []
+    vals, secs = [], []
     for i in range(args.warmup + args.steps):
         v, info = time_oracle(w, heads, tokens)
         if i >= args.warmup:
             vals.append(v)
+            secs.append(info["seconds"])
     val = statistics.median(vals)
+    sample_ms = statistics.median(secs) * 1e3
     line = {
         "impl": "reference", "metric": "fwd+bwd tokens/s per layer", "value": round(val, 3),
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(w.B * w.T / val * 1e3, 3), "higher_is_better": True,
+        "ms_per_step": round(sample_ms, 3),
+        "ms_per_step_is": "measured time of one step's bounded sample (see cpu_baseline.sample)",
+        "full_layer_ms_extrapolated": round(w.B * w.T / val * 1e3, 3),
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d": w.d,
-                   "n_sub": w.n_sub, "chunk": 64},
+        "config": bench_config(w, inputs.sub_lengths(w), world, args.mode),
         "cpu_baseline": {"value": round(val, 3), "unit": "tokens/s", "cores": info["cores"],
-                         "kind": "oracle", "sample": info["sample"] + "; each step one sample"},
+                         "kind": "oracle", "sample": info["sample"] + "; each step one sample",
+                         "seconds_per_sample": round(sample_ms / 1e3, 3)},
         "e2e": {"value": round(val, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -570,9 +696,7 @@ def run_sf(args, w, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        val, info = time_oracle(w, heads=w.H, tokens=min(w.T, args.cpu_sample_tokens))
-        cpu = {"value": round(val, 3), "unit": "tokens/s", "cores": info["cores"], "kind": "oracle",
-               "sample": info["sample"]}
+        cpu = cpu_baseline(w, min(w.T, args.cpu_sample_tokens))
 
     if rank == 0:
         peaks, src = load_peaks()
@@ -582,10 +706,7 @@ def run_sf(args, w, rank, world, local_rank):
             "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
             "data": "synthetic",
-            "config": {"workload": w.name, "B": B, "T": T, "H": H, "d": d, "n_sub": len(lens),
-                       "chunk": 64, "variant": w.variant, "l2": "inputs larger than L2, no flush",
-                       "parallelism": f"replicas{world}", "mode": args.mode,
-                       "keep_bytes": keep.numel()},
+            "config": bench_config(w, lens, world, args.mode),
             "modes": {args.mode: {"ms_per_step": round(ms_max, 4),
                                   "value": round(job_tokens_per_s(world, B, T, ms_max), 1)},
                       other: None if ms_other is None else
@@ -595,6 +716,8 @@ def run_sf(args, w, rank, world, local_rank):
             "gpu_launches": launches,
             "e2e": e2e,
             "roofline": roofline(timing, w, args.steps, peaks, src, clocks, args.mode),
+            "step": step_roofline(w, ms_max, peaks),
+            "keep_bytes": keep.numel(),
             "kernels": kernel_rooflines(timing, w, args.steps, peaks, args.mode),
             "kernel_timing": "serialized pass (driver streams merged), CUDA events per launch",
             "cpu_baseline": cpu,

@@ -90,10 +90,8 @@ cudaError_t launch_intra_tc(const Args& a, bool with_p, cudaStream_t s);
 cudaError_t launch_output_tc(const Args& a, cudaStream_t s);
 // reverse dS pass; consumes P from the backward intra kernel (no dDelta pre-pass)
 cudaError_t launch_state_bwd_tc(const Args& a, cudaStream_t s);
-// dq, dk, dg (adds dKp / dGp of the delta-rule gradient kernel when beta is given)
+// dq, dk, dv, dg of (gated) linear attention (no beta)
 cudaError_t launch_grad_attn_tc(const Args& a, cudaStream_t s);
-// dv, dbeta and the delta-rule parts dKp, dGp
-cudaError_t launch_grad_delta_tc(const Args& a, cudaStream_t s);
 // every per-chunk gradient of the gated delta rule in one kernel (dq, dk, dv, dg, dbeta)
 cudaError_t launch_grad_fused_tc(const Args& a, cudaStream_t s);
 

@@ -13,13 +13,12 @@
 // library, for as long as the process runs.  All calls share it, so two calls
 // whose work overlaps on the GPU (different streams, or different host
 // threads) race on it; calls that are ordered on one stream are safe.  The
-// array keeps whatever the previous call left in it; this call clears the one
-// word that must start at zero (the error word read by sf_check) and every
-// other byte it reads is written by an earlier kernel of the same call.
+// array keeps whatever the previous call left in it; each call clears the one
+// word that must start at zero (the error word that bounded device waits set)
+// and every other byte it reads is written by an earlier kernel of the same
+// call.  sf_check_noalloc reads that error word.
 
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "../../include/sf.h"
 #include "sf_internal.h"
@@ -31,24 +30,17 @@ constexpr size_t kScratchBytes = (size_t)32 << 20;  // 32 MiB
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_scratch on the current device (looked up once per device).
+// Device address of g_scratch in the current device's context.  In host code
+// g_scratch names a host-side stand-in, so kernels must be given this address.
+// It is looked up on every call (cheap once the module is loaded), so that a new
+// context after cudaDeviceReset, in which the module may land elsewhere, gets
+// its own address; the first lookup on a device may load the module, which is
+// why the first call should come before any stream capture.
 cudaError_t scratch_address(void** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    *out = p;
     return cudaSuccess;
 }
 
@@ -68,6 +60,12 @@ sf_status sf_fwd_noalloc(const sf_shape* s, const void* q, const void* k, const 
     if (sf::scratch_address(&ws) != cudaSuccess) return SF_ERR_CUDA;
     if (cudaMemsetAsync(ws, 0, sizeof(int), (cudaStream_t)stream) != cudaSuccess) return SF_ERR_CUDA;
     return sf_fwd(s, q, k, v, g, beta, S_in, o, S_out, ws, sf::kScratchBytes, stream);
+}
+
+sf_status sf_check_noalloc(void* stream) {
+    void* ws = nullptr;
+    if (sf::scratch_address(&ws) != cudaSuccess) return SF_ERR_CUDA;
+    return sf_check(ws, stream);
 }
 
 }  // extern "C"

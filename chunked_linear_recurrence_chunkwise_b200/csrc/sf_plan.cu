@@ -81,8 +81,9 @@ bool valid_costs(const sf_chunk_costs* c) {
 
 // Modelled device time of the forward and the backward of the keep drivers.
 double model_us(const sf_shape* s, int n_sub, const int* lens, const sf_chunk_costs* c) {
+    // the state passes' per-chunk costs are measured over all B x H heads, the extra
+    // waves of CTAs when the heads outnumber the SMs included
     const long bh = (long)s->B * s->H;
-    const long waves = (bh + c->sms - 1) / c->sms;
     const double free_frac = std::max(0.0, (double)(c->sms - std::min<long>(bh, c->sms)) / c->sms);
     std::vector<double> nc(n_sub);
     for (int i = 0; i < n_sub; ++i) nc[i] = std::ceil((double)lens[i] / kChunkTokens);
@@ -97,7 +98,7 @@ double model_us(const sf_shape* s, int n_sub, const int* lens, const sf_chunk_co
     };
     for (int j = 0; j < std::min(2, n_sub); ++j) intra[j] = add(f, 1, nc[j] * c->intra_us, {});
     for (int i = 0; i < n_sub; ++i) {
-        state[i] = add(f, 0, nc[i] * c->state_fwd_us * waves, {intra[i]});
+        state[i] = add(f, 0, nc[i] * c->state_fwd_us, {intra[i]});
         if (i + 2 < n_sub) intra[i + 2] = add(f, 1, nc[i + 2] * c->intra_us, {});
         add(f, 1, nc[i] * c->output_us, {state[i]});
     }
@@ -108,7 +109,7 @@ double model_us(const sf_shape* s, int n_sub, const int* lens, const sf_chunk_co
     for (int i = n_sub - 1; i >= 0; --i) {
         std::vector<int> deps;
         if (i + 3 < n_sub) deps.push_back(grads[i + 3]);
-        const int sb = add(b, 0, nc[i] * c->state_bwd_us * waves, deps);
+        const int sb = add(b, 0, nc[i] * c->state_bwd_us, deps);
         grads[i] = add(b, 1, nc[i] * c->grad_us, {sb});
     }
     return simulate(f, free_frac) + simulate(b, free_frac);

@@ -502,13 +502,20 @@ __global__ void __launch_bounds__(kThreads) grad_delta_kernel(Args a) {
         float acc = 0.f;
         for (int i = r; i < kChunk; ++i) acc += Ts[i * kChunk + r] * dDs[i * ldv + n];
         dVh[r * ldv + n] = acc;
-        if (r < L) {
-            const size_t ti = tok(a, b, t0 + r, h) * dv + n;
-            stf((TIO*)a.dv_ + ti, bs[r] * acc);
-            atomicAdd(&db1[r], ldf((const TIO*)a.v + ti) * acc);
-        }
+        if (r < L) stf((TIO*)a.dv_ + tok(a, b, t0 + r, h) * dv + n, bs[r] * acc);
     }
     __syncthreads();
+    // <V_r, dVhat_r>, summed in a fixed order (one thread per row) so that results
+    // do not depend on the scheduling of the threads
+    if (threadIdx.x < kChunk) {
+        const int r = threadIdx.x;
+        float acc = 0.f;
+        if (r < L) {
+            const TIO* vr = (const TIO*)a.v + tok(a, b, t0 + r, h) * dv;
+            for (int n = 0; n < dv; ++n) acc += ldf(vr + n) * dVh[r * ldv + n];
+        }
+        db1[r] = acc;
+    }
     for (int e = threadIdx.x; e < kChunk * kChunk; e += blockDim.x) {
         const int r = e >> 6, i = e & 63;
         float acc = 0.f;
@@ -549,9 +556,11 @@ __global__ void __launch_bounds__(kThreads) grad_delta_kernel(Args a) {
             for (int d = 0; d < dk; ++d) acc += dWs[r * ldk + d] * Wsm[i * ldk + d];
         dAs[e] = (i < r) ? -acc : 0.f;
     }
-    for (int e = threadIdx.x; e < kChunk * dk; e += blockDim.x) {
-        const int r = e / dk, i = e - r * dk;
-        atomicAdd(&red[r], Ks[r * ldk + i] * dWs[r * ldk + i]);  // <K_r, dKhat_r>
+    if (threadIdx.x < kChunk) {  // <K_r, dKhat_r>, one thread per row
+        const int r = threadIdx.x;
+        float acc = 0.f;
+        for (int i = 0; i < dk; ++i) acc += Ks[r * ldk + i] * dWs[r * ldk + i];
+        red[r] = acc;
     }
     __syncthreads();
     // dbeta and dG (delta part); E = dB .* Gamma into Ts.
@@ -595,8 +604,8 @@ __global__ void __launch_bounds__(kThreads) grad_attn_kernel(Args a) {
     extern __shared__ float sm[];
     float* Gs = sm;                      // 64
     float* dGs = Gs + kChunk;            // 64
-    float* scal = dGs + kChunk;          // 2 (+pad to 64)
-    float* Qs = scal + kChunk;           // [64][dk+1]
+    float* scal = dGs + kChunk;          // 128: <S, dS'>, -, per-warp partials, then per-row terms
+    float* Qs = scal + 2 * kChunk;       // [64][dk+1]
     float* Ks = Qs + kChunk * ldk;       // [64][dk+1]
     float* dOs = Ks + kChunk * ldk;      // [64][dv+1]
     float* Ds = dOs + kChunk * ldv;      // [64][dv+1]
@@ -610,6 +619,7 @@ __global__ void __launch_bounds__(kThreads) grad_attn_kernel(Args a) {
         Gs[threadIdx.x] = a.G[(size_t)bh * TP + t0 + threadIdx.x];
         dGs[threadIdx.x] = 0.f;
         scal[threadIdx.x] = 0.f;
+        scal[kChunk + threadIdx.x] = 0.f;
     }
     load_rows(a, (const TIO*)a.q, dk, b, h, t0, L, Qs, ldk);
     load_rows(a, (const TIO*)a.k, dk, b, h, t0, L, Ks, ldk);
@@ -673,10 +683,22 @@ __global__ void __launch_bounds__(kThreads) grad_attn_kernel(Args a) {
             const int r = e / dk, d = e - r * dk;
             float x = 0.f;
             for (int n = 0; n < dv; ++n) x += dOs[r * ldv + n] * Ss[d * ldv + n];
-            const float gam = __expf(Gs[r]);
-            dq[j] += gam * x;
-            atomicAdd(&dGs[r], gam * Qs[r * ldk + d] * x);
+            dq[j] += __expf(Gs[r]) * x;
         }
+    }
+    // gamma_r <Q_r, (dO S^T)_r> per row, one warp per row in a fixed order of summation
+    // (lanes over d, then a shuffle tree), so that results do not depend on scheduling
+    for (int r = threadIdx.x >> 5; r < kChunk; r += kThreads / 32) {
+        const int lane = threadIdx.x & 31;
+        float acc = 0.f;
+        for (int d = lane; d < dk; d += 32) {
+            float x = 0.f;
+            for (int n = 0; n < dv; ++n) x += dOs[r * ldv + n] * Ss[d * ldv + n];
+            acc += Qs[r * ldk + d] * x;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) dGs[r] += __expf(Gs[r]) * acc;
     }
     __syncthreads();
     float* dSp = R;  // [dk][dv+1], dS'[i][n]
@@ -687,10 +709,17 @@ __global__ void __launch_bounds__(kThreads) grad_attn_kernel(Args a) {
         dSp[i * ldv + n] = x;
         sdot += x * ldf(Scg + e);
     }
-    atomicAdd(&scal[0], sdot);
+    // <S, dS'>: per-warp shuffle trees, then warp 0's lanes in order
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sdot += __shfl_xor_sync(0xffffffffu, sdot, off);
+    if ((threadIdx.x & 31) == 0) scal[2 + (threadIdx.x >> 5)] = sdot;
     __syncthreads();
+    if (threadIdx.x == 0) {
+        float acc = 0.f;
+        for (int w = 0; w < kThreads / 32; ++w) acc += scal[2 + w];
+        scal[0] = acc;
+    }
     const float gC = Gs[kChunk - 1];
-    float lastsum = 0.f;
 #pragma unroll
     for (int j = 0; j < kMaxE; ++j) {
         const int e = threadIdx.x + j * kThreads;
@@ -698,17 +727,33 @@ __global__ void __launch_bounds__(kThreads) grad_attn_kernel(Args a) {
             const int r = e / dk, d = e - r * dk;
             float x = 0.f;
             for (int n = 0; n < dv; ++n) x += Ds[r * ldv + n] * dSp[d * ldv + n];
-            const float ec = __expf(gC - Gs[r]);
-            dkk[j] += ec * x;
-            const float t = ec * Ks[r * ldk + d] * x;
-            atomicAdd(&dGs[r], -t);
-            lastsum += t;
+            dkk[j] += __expf(gC - Gs[r]) * x;
         }
     }
-    atomicAdd(&scal[1], lastsum);
+    // e^{G_C - G_r} <K_r, (Delta dS'^T)_r> per row (one warp per row, fixed order), kept in
+    // red[r] for its last-row sum
+    float* red = scal + 2 + kThreads / 32;
+    for (int r = threadIdx.x >> 5; r < kChunk; r += kThreads / 32) {
+        const int lane = threadIdx.x & 31;
+        float acc = 0.f;
+        for (int d = lane; d < dk; d += 32) {
+            float x = 0.f;
+            for (int n = 0; n < dv; ++n) x += Ds[r * ldv + n] * dSp[d * ldv + n];
+            acc += Ks[r * ldk + d] * x;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) {
+            const float t = __expf(gC - Gs[r]) * acc;
+            dGs[r] -= t;
+            red[r] = t;
+        }
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
-        dGs[kChunk - 1] += scal[1] + __expf(gC) * scal[0];
+        float lastsum = 0.f;
+        for (int r = 0; r < kChunk; ++r) lastsum += red[r];
+        dGs[kChunk - 1] += lastsum + __expf(gC) * scal[0];
         float acc = 0.f;
         for (int r = kChunk - 1; r >= 0; --r) {
             acc += dGs[r] + (a.beta ? a.dGp[(size_t)bh * TP + t0 + r] : 0.f);
@@ -760,7 +805,7 @@ size_t smem_grad_delta(const Args& a) {
 size_t smem_grad_attn(const Args& a) {
     const int ldk = a.dk + 1, ldv = a.dv + 1;
     const int Rsize = std::max(2 * kChunk * kChunk, a.dk * ldv);
-    return sizeof(float) * (3 * kChunk + 2 * kChunk * ldk + 2 * kChunk * ldv + Rsize);
+    return sizeof(float) * (4 * kChunk + 2 * kChunk * ldk + 2 * kChunk * ldv + Rsize);
 }
 
 template <typename K>

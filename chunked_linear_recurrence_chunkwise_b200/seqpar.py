@@ -39,26 +39,59 @@ def micro_rows(B: int, micro: int) -> list:
 
 
 class KeepRunner:
-    """One rank's compute: the CUDA keep drivers on the rank's slice (the product path)."""
+    """One rank's compute: the CUDA keep drivers on the rank's slice (the product path).
 
-    def __init__(self, lens=None, aux_stream=None):
+    lens: the cut of the rank's slice into pieces (its lengths must sum to the
+    slice's length); or piece: cut the slice into pieces of at most `piece`
+    tokens; neither: the slice is one piece.  host_states: the boundary states
+    travel through host memory (pinned copies on both sides of a message), for a
+    transport that carries host tensors only, such as gloo; NCCL takes the device
+    tensors as they are."""
+
+    def __init__(self, lens=None, aux_stream=None, piece=None, host_states=False):
+        if lens is not None and piece is not None:
+            raise ValueError("give lens or piece, not both")
         self.lens = lens
+        self.piece = piece
         self.aux = aux_stream
+        self.host_states = host_states
+
+    def _cut(self, T: int):
+        if self.piece is not None:
+            return [min(self.piece, T - t) for t in range(0, T, self.piece)]
+        return self.lens
 
     def state_buffer(self, rows: int, H: int, dk: int, dv: int, like):
         import torch
+        if self.host_states:
+            return torch.empty((rows, H, dk, dv), dtype=torch.float32, pin_memory=True)
         return torch.empty((rows, H, dk, dv), dtype=torch.float32, device=like.device)
+
+    def _to_dev(self, s, like):
+        return None if s is None else s.to(like.device, non_blocking=True).contiguous()
+
+    def _to_msg(self, s):
+        if not self.host_states:
+            return s
+        import torch
+        h = torch.empty(s.shape, dtype=s.dtype, pin_memory=True)
+        h.copy_(s)  # synchronous: the message must hold the state before it is sent
+        return h
 
     def fwd(self, q, k, v, g, beta, S_in):
         from . import layer
-        o, S_out, kept = layer.forward_keep(q, k, v, g, beta, S_in, lens=self.lens, aux_stream=self.aux)
-        return o, S_out, (q, k, v, g, beta, kept)
+        lens = self._cut(q.shape[1])
+        o, S_out, kept = layer.forward_keep(q, k, v, g, beta, self._to_dev(S_in, q), lens=lens,
+                                            aux_stream=self.aux)
+        return o, self._to_msg(S_out), (q, k, v, g, beta, kept, lens)
 
     def bwd(self, ctx, dO, dS_out):
         from . import layer
-        q, k, v, g, beta, kept = ctx
-        return layer.backward_keep(q, k, v, g, beta, dO, kept, dS_out=dS_out, lens=self.lens,
-                                   aux_stream=self.aux)
+        q, k, v, g, beta, kept, lens = ctx
+        gr = layer.backward_keep(q, k, v, g, beta, dO, kept, dS_out=self._to_dev(dS_out, q), lens=lens,
+                                 aux_stream=self.aux)
+        gr["dS_in"] = self._to_msg(gr["dS_in"])
+        return gr
 
 
 @dataclass

@@ -51,6 +51,7 @@ _SIGS = {
     "sf_fwd_seq_keep": (_I, [_SP, _I, _IP] + [_P] * 8 + [_P, _S, _P, _S, _P, _P]),
     "sf_bwd_seq_keep": (_I, [_SP, _I, _IP] + [_P] * 5 + [_P, _S] + [_P] * 8 + [_P, _S, _P, _P]),
     "sf_fwd_noalloc": (_I, [_SP] + [_P] * 8 + [_P]),
+    "sf_check_noalloc": (_I, [_P]),
     "sf_check": (_I, [_P, _P]),
     "sf_status_string": (ctypes.c_char_p, [_I]),
     "sf_timing_enable": (None, [_I]),
@@ -193,6 +194,11 @@ def sf_fwd_noalloc(sh, q, k, v, g, beta, S_in, o, S_out, stream=None):
     """sf_fwd with the library's built-in scratch instead of a caller workspace."""
     _check(_lib.sf_fwd_noalloc(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
                                _ptr(S_in), _ptr(o), _ptr(S_out), _stream(stream)), "sf_fwd_noalloc")
+
+
+def sf_check_noalloc(stream=None):
+    """sf_check for sf_fwd_noalloc: the built-in scratch array's error word."""
+    _check(_lib.sf_check_noalloc(_stream(stream)), "sf_check_noalloc")
 
 
 def sf_check(ws, stream=None):

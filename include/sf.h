@@ -171,18 +171,25 @@ sf_status sf_bwd_seq_keep(const sf_shape* shape, int n_sub, const int* lens, con
  * memory by every GPU that loads the library until the process exits.  A shape
  * whose sf_workspace_bytes(shape, SF_OP_FWD) exceeds 32 MiB is rejected with
  * SF_ERR_WORKSPACE before anything is launched (bf16, d_k = d_v = 128 needs
- * about 1.3 KB per token and head).  The first call on a device looks up the
- * array's device address (once per device, with that device current); make
- * that first call before any stream capture.  All calls share the one array:
- * calls whose work may overlap on the GPU (other streams, other host threads)
- * race on it, calls ordered on one stream do not.  The array keeps the previous
- * call's contents; each call first clears the error word that bounded device
- * waits set (it lives in the array, so sf_check cannot read it for this entry
- * point).  Allocates nothing: no cudaMalloc, cudaFree or allocating library
+ * about 1.3 KB per token and head).  Each call looks up the array's device
+ * address in the current device's context; the first lookup on a device may
+ * load the library's device code, so make the first call on each device before
+ * any stream capture.  All calls share the one array: calls whose work may
+ * overlap on the GPU (other streams, other host threads) race on it, calls
+ * ordered on one stream do not.  The array keeps the previous call's contents;
+ * each call first clears the error word that bounded device waits set (it lives
+ * in the array), so read it with sf_check_noalloc after a call and before the
+ * next one.  Allocates nothing: no cudaMalloc, cudaFree or allocating library
  * routine is called. */
 sf_status sf_fwd_noalloc(const sf_shape* shape, const void* q, const void* k, const void* v,
                          const float* g, const float* beta, const float* S_in, void* o,
                          float* S_out, void* stream);
+
+/* sf_check for sf_fwd_noalloc: synchronises `stream`, then reads and clears the
+ * error word of the built-in scratch array on the current device.  Returns
+ * SF_ERR_TIMEOUT if a kernel of an sf_fwd_noalloc call gave up a bounded wait
+ * since the word was last cleared, SF_ERR_CUDA on a CUDA error, else SF_OK. */
+sf_status sf_check_noalloc(void* stream);
 
 /* Synchronises `stream`, then reads and clears the device error word kept at
  * the head of workspace `ws`.  Returns SF_ERR_TIMEOUT if a kernel gave up a

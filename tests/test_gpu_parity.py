@@ -4,6 +4,8 @@ Tolerances (relative L2 over each whole output tensor, ||x - ref|| / ||ref||):
 1e-4 for fp32 inputs and 2e-2 for bf16 inputs; chunking invariance on the GPU
 within 1e-5 in fp32.  bf16 cases feed the oracle the bf16-rounded inputs.
 """
+import zlib
+
 import numpy as np
 import pytest
 import torch
@@ -78,7 +80,8 @@ SHAPES = [
 @pytest.mark.parametrize("shape", SHAPES)
 def test_single_piece_matches_oracle(layer, dtype, has_g, has_beta, shape):
     B, T, H, dk, dv = shape
-    c = make_case(hash((shape, has_g, has_beta)) % 1000, B, T, H, dk, dv, has_g, has_beta, dtype)
+    seed = zlib.crc32(repr((shape, has_g, has_beta)).encode()) % 1000  # fixed across processes
+    c = make_case(seed, B, T, H, dk, dv, has_g, has_beta, dtype)
     d = to_dev(c, dtype)
     o, S_out, _ = layer.forward(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S_in"])
     gr = layer.backward(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], S_in=d["S_in"],

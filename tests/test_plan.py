@@ -49,11 +49,20 @@ def test_two_pieces_by_hand(sf):
     assert sf.sf_model_seq_us(sh, [64, 64], c) == pytest.approx(13.0)
 
 
-def test_state_passes_run_in_waves_when_heads_outnumber_sms(sf):
-    # 8 heads on 4 SMs: each state pass takes two waves and leaves no SM free
+def test_state_passes_hold_every_sm_when_heads_outnumber_sms(sf):
+    # 8 heads on 4 SMs: the state passes' costs, measured over all heads, already hold
+    # their two waves of CTAs (they are not counted twice), and no SM is left free for
+    # the parallel kernels beside them.  One piece: 1 + 3 + 1, then 5 + 1.
     sh = sf.shape(2, 64, 4, 128, 128, sf.SF_BF16)
     c = costs(sf, intra_us=1.0, output_us=1.0, grad_us=1.0, state_fwd_us=3.0, state_bwd_us=5.0, sms=4)
-    assert sf.sf_model_seq_us(sh, [64], c) == pytest.approx(1 + 6 + 1 + 10 + 1)
+    assert sf.sf_model_seq_us(sh, [64], c) == pytest.approx(1 + 3 + 1 + 5 + 1)
+    # two pieces, every cost 1: with no SM free, the parallel kernels advance only while
+    # no state pass runs.  forward: intra0 [0,1]; state0 [1,2] (intra1 stalled); intra1
+    # [2,3]; state1 [3,4] (output0 stalled); output0 [4,5]; output1 [5,6].  backward:
+    # reverse pass of piece 1 [0,1]; reverse pass of piece 0 [1,2] (gradients of piece 1
+    # stalled); gradients of piece 1 [2,3]; of piece 0 [3,4].  Total 6 + 4.
+    c2 = costs(sf, intra_us=1.0, output_us=1.0, grad_us=1.0, state_fwd_us=1.0, state_bwd_us=1.0, sms=4)
+    assert sf.sf_model_seq_us(sf.shape(2, 128, 4, 128, 128, sf.SF_BF16), [64, 64], c2) == pytest.approx(10.0)
 
 
 def test_model_rejects_invalid_cuts(sf):
