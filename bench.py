@@ -123,6 +123,7 @@ def canonical_flops(name: str, w) -> float:
         "state_fwd": 2 * v if delta else v,
         "output": u + v,
         "output_p": 0.5 * u + v,                               # P read, not formed
+        "state_out": (2 * v if delta else v) + 0.5 * u + v,    # state pass + output (P read)
         "state_bwd": 0.5 * u + (3 * v if delta else 2 * v),
         "grad_fused": 4.5 * u + 3 * v,
         "grad_attn": 1.5 * u + 2 * v,
@@ -181,6 +182,10 @@ def kernel_units(name: str, w, mode: str = "keep") -> dict:
             # read q, S^T, Delta^T, the stored P, G; write o
             "output_p": (2 * tile, tile + st + tile + C * C * e + C * f + tile,
                          mm(d, C, d) + mm(d, C, C)),
+            # the fused forward: read W^T, U^T, k, q, the stored P, decay table; write S^T,
+            # Delta^T, o
+            "state_out": (3 * tile, 4 * tile + C * C * e + 2 * C * f + st + 2 * tile,
+                          mm(d, C, d) + mm(d, d, C) + mm(d, C, d) + mm(d, C, C)),
             # read k, dO, q, W^T, P, G; write dS'^T, dDelta^T
             "state_bwd": (3 * tile, 4 * tile + C * C * e + C * f + st + tile,
                           mm(d, C, d) + mm(d, C, C) + 2 * mm(d, d, C)),
@@ -219,10 +224,14 @@ def kernel_units(name: str, w, mode: str = "keep") -> dict:
 # hex digits) of the source file the kernel was built from at the time of the capture.
 # A kernel whose source has changed since reports traffic null.
 NCU_TRAFFIC_2048 = {
-    # name: (bytes per 2048 chunk-heads, source file, sha256[:16])
+    # name: (bytes per 2048 chunk-heads, source file, sha256[:16]); profiles/<kernel>_*.md
+    "grad_fused": (437198336, "sf_tc_grad_fused.cu", "f75f206f17a7051b"),
+    "grad_attn": (321572096, "sf_tc_grad.cu", "5803a1b053b95f97"),
+    "state_fwd": (162895104, "sf_tc_state.cu", "c25118f738eb4316"),
 }
 KERNEL_SOURCE = {
     "grad_fused": "sf_tc_grad_fused.cu", "state_fwd": "sf_tc_state.cu", "state_bwd": "sf_tc_state.cu",
+    "state_out": "sf_tc_state.cu",
     "intra_bwd": "sf_tc_chunk.cu", "intra_fwd": "sf_tc_chunk.cu", "output": "sf_tc_chunk.cu",
     "grad_attn": "sf_tc_grad.cu",
 }
@@ -242,7 +251,7 @@ def measured_traffic(name: str, units_per_launch: float, w, mode: str):
     """DRAM bytes per launch from the committed capture, or None when there is none for
     this kernel on this path or the kernel's source has changed since it was taken."""
     ent = NCU_TRAFFIC_2048.get(name)
-    if not ent or not tc_path(w) or mode != "keep":
+    if not ent or not tc_path(w):
         return None
     nbytes, fname, sha = ent
     if source_sha(fname) != sha:

@@ -83,7 +83,8 @@ cudaError_t launch_grad_attn(const Args& a, cudaStream_t s);
 
 // Tensor-core kernels (sm_100a tcgen05/TMEM/TMA; bf16, d_k = d_v = 128).
 bool tc_eligible(const Args& a);
-cudaError_t launch_state_fwd_tc(const Args& a, cudaStream_t s);
+// with_output: the fused forward, which also writes o (reads the stored P from a.Pm)
+cudaError_t launch_state_fwd_tc(const Args& a, bool with_output, cudaStream_t s);
 // with_p: also store P (backward recompute)
 cudaError_t launch_intra_tc(const Args& a, bool with_p, cudaStream_t s);
 // reads P from a.Pm when it is set (the forward that keeps its intermediates)
@@ -106,6 +107,7 @@ enum KernelKind {
     KK_GRAD_ATTN,
     KK_INTRA_BWD,
     KK_GRAD_FUSED,
+    KK_STATE_OUT,
     KK_COUNT
 };
 const char* kernel_name(int kind);
