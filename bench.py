@@ -123,7 +123,6 @@ def canonical_flops(name: str, w) -> float:
         "state_fwd": 2 * v if delta else v,
         "output": u + v,
         "output_p": 0.5 * u + v,                               # P read, not formed
-        "state_out": (2 * v if delta else v) + 0.5 * u + v,    # state pass + output (P read)
         "state_bwd": 0.5 * u + (3 * v if delta else 2 * v),
         "grad_fused": 4.5 * u + 3 * v,
         "grad_attn": 1.5 * u + 2 * v,
@@ -182,10 +181,6 @@ def kernel_units(name: str, w, mode: str = "keep") -> dict:
             # read q, S^T, Delta^T, the stored P, G; write o
             "output_p": (2 * tile, tile + st + tile + C * C * e + C * f + tile,
                          mm(d, C, d) + mm(d, C, C)),
-            # the fused forward: read W^T, U^T, k, q, the stored P, decay table; write S^T,
-            # Delta^T, o
-            "state_out": (3 * tile, 4 * tile + C * C * e + 2 * C * f + st + 2 * tile,
-                          mm(d, C, d) + mm(d, d, C) + mm(d, C, d) + mm(d, C, C)),
             # read k, dO, q, W^T, P, G; write dS'^T, dDelta^T
             "state_bwd": (3 * tile, 4 * tile + C * C * e + C * f + st + tile,
                           mm(d, C, d) + mm(d, C, C) + 2 * mm(d, d, C)),
@@ -231,7 +226,6 @@ NCU_TRAFFIC_2048 = {
 }
 KERNEL_SOURCE = {
     "grad_fused": "sf_tc_grad_fused.cu", "state_fwd": "sf_tc_state.cu", "state_bwd": "sf_tc_state.cu",
-    "state_out": "sf_tc_state.cu",
     "intra_bwd": "sf_tc_chunk.cu", "intra_fwd": "sf_tc_chunk.cu", "output": "sf_tc_chunk.cu",
     "grad_attn": "sf_tc_grad.cu",
 }

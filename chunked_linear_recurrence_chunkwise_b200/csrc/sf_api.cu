@@ -105,6 +105,7 @@ void bind_slot(Args& a, void* ws, const WsLayout& L, int slot, bool bwd) {
     a.dKp = bwd ? (float*)(base + L.dKp) : nullptr;
     a.dGp = bwd ? (float*)(base + L.dGp) : nullptr;
     a.err = (int*)ws;
+    a.ticket = (unsigned*)((char*)ws + 8);
 }
 
 // ------------------------------------------------------------------ timing
@@ -134,8 +135,7 @@ cudaEvent_t pool_get() {
 
 const char* kernel_name(int kind) {
     static const char* names[KK_COUNT] = {"intra_fwd", "state_fwd", "output",    "dd_pre",    "state_bwd",
-                                          "grad_delta", "grad_attn", "intra_bwd", "grad_fused",
-                                          "state_out"};
+                                          "grad_delta", "grad_attn", "intra_bwd", "grad_fused"};
     return (kind >= 0 && kind < KK_COUNT) ? names[kind] : "?";
 }
 
@@ -211,7 +211,7 @@ cudaError_t copy_state(float* dst, const float* src, size_t n, cudaStream_t st) 
 // Kernel choice: the tensor-core kernels cover bf16 with d_k = d_v = 128; the
 // SIMT kernels cover everything else (and are the fp32 path).
 cudaError_t state_fwd(const Args& a, cudaStream_t st) {
-    return tc_eligible(a) ? launch_state_fwd_tc(a, false, st) : launch_state_fwd(a, st);
+    return tc_eligible(a) ? launch_state_fwd_tc(a, st) : launch_state_fwd(a, st);
 }
 
 cudaError_t intra(const Args& a, bool with_p, cudaStream_t st) {
@@ -539,24 +539,17 @@ sf_status fwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* q, 
         SF_TRY(run_intra_piece(piece(j)));
         SF_TRY(cudaEventRecord(ev_intra[j % NS], sa));
     }
-    // With keep on the tensor-core path the state pass also forms the output (the fused
-    // forward, reading the P the intra kernel kept); otherwise the output kernel follows the
-    // state pass on the aux stream.
-    const bool fused = false && keep != nullptr && tc_eligible(piece(0));
     for (int i = 0; i < n_sub; ++i) {
         const Args a = piece(i);
         SF_TRY(cudaStreamWaitEvent(sc, ev_intra[i % NS], 0));
-        if (fused)
-            SF_TRY(launch_state_fwd_tc(a, true, sc));
-        else
-            SF_TRY(run_state_output(a, sc, false));
+        SF_TRY(run_state_output(a, sc, false));
         SF_TRY(cudaEventRecord(ev_state[i % NS], sc));
         if (i + 2 < n_sub) {  // its slot's previous piece (i-1) finished its output
             SF_TRY(run_intra_piece(piece(i + 2)));
             SF_TRY(cudaEventRecord(ev_intra[(i + 2) % NS], sa));
         }
         SF_TRY(cudaStreamWaitEvent(sa, ev_state[i % NS], 0));
-        if (!fused) SF_TRY(output(a, sa));
+        SF_TRY(output(a, sa));
     }
     SF_TRY(cudaEventRecord(ev_aux_done, sa));
     SF_TRY(cudaEventRecord(ev_crit_done, sc));
@@ -667,7 +660,12 @@ sf_status bwd_seq(const sf_shape* s, int n_sub, const int* lens, const void* q, 
             SF_TRY(cudaEventRecord(ev_prep[(i - 2) % NS], sa));
         }
         SF_TRY(cudaStreamWaitEvent(sa, ev_state[i % NS], 0));
-        SF_TRY(run_bwd_chunk_grads(a, sa));
+        // the reverse pass of piece i-1 (one CTA per batch-head) runs beside these gradients:
+        // they keep off its SMs, or their resident CTAs, which take chunk-heads until none are
+        // left, would hold the SMs the next reverse pass needs
+        Args ag = a;
+        if (i > 0) ag.grad_sms = -(s->B * s->H);
+        SF_TRY(run_bwd_chunk_grads(ag, sa));
         if (keep) SF_TRY(cudaEventRecord(ev_prep[i % NS], sa));
     }
     SF_TRY(cudaEventRecord(ev_aux_done, sa));

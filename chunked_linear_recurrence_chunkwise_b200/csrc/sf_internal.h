@@ -49,6 +49,12 @@ struct Args {
     float* dKp;   // [BH][TP][dk]        fp32 delta-rule part of dk (SIMT gradient kernels)
     float* dGp;   // [BH][TP]            fp32 delta-rule part of dG (SIMT gradient kernels)
     int* err;     // device error word
+    // two work counters of the gradient kernel, zero between launches (the last CTA of a
+    // launch puts them back)
+    unsigned* ticket;
+    // SMs the gradient kernel may hold (0: all): the sub-sequence drivers leave those of a
+    // state pass that runs beside it free
+    int grad_sms;
 };
 
 // Workspace carve-up for a piece of at most T tokens.
@@ -83,8 +89,7 @@ cudaError_t launch_grad_attn(const Args& a, cudaStream_t s);
 
 // Tensor-core kernels (sm_100a tcgen05/TMEM/TMA; bf16, d_k = d_v = 128).
 bool tc_eligible(const Args& a);
-// with_output: the fused forward, which also writes o (reads the stored P from a.Pm)
-cudaError_t launch_state_fwd_tc(const Args& a, bool with_output, cudaStream_t s);
+cudaError_t launch_state_fwd_tc(const Args& a, cudaStream_t s);
 // with_p: also store P (backward recompute)
 cudaError_t launch_intra_tc(const Args& a, bool with_p, cudaStream_t s);
 // reads P from a.Pm when it is set (the forward that keeps its intermediates)
@@ -107,7 +112,6 @@ enum KernelKind {
     KK_GRAD_ATTN,
     KK_INTRA_BWD,
     KK_GRAD_FUSED,
-    KK_STATE_OUT,
     KK_COUNT
 };
 const char* kernel_name(int kind);

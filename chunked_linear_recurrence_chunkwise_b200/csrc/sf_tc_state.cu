@@ -78,23 +78,16 @@ constexpr int kThreads = 512;
 constexpr int kFwdThreads = kThreads + 64;
 constexpr int kFwdChain = kThreads, kFwdCopy = kThreads + 32;
 
-// Shared-memory carve-up of the forward pass (byte offsets from a 1024-byte aligned
-// base).  With the output (kOut) each stage also holds Q and the stored P of its
-// chunk, and the ring is two stages deep instead of three.
-template <bool kOut>
+// Shared-memory carve-up of the forward pass (byte offsets from a 1024-byte aligned base).
 struct FwdSmem {
-    static constexpr int kSt = kOut ? 2 : kStages;
     static constexpr int Wt = 0;                          // [stage] W^T  [d_k][64 r]
-    static constexpr int Kt = Wt + kSt * kTile;           // [stage] K    [2][64 r][64 d_k]
-    static constexpr int Ut = Kt + kSt * kTile;           // [stage] U^T  [d_v][64 r]
-    static constexpr int Qt = Ut + kSt * kTile;           // kOut: [stage] Q [2][64 r][64 d_k], scaled by gamma in place
-    static constexpr int Pt = Qt + (kOut ? kSt * kTile : 0);  // kOut: [stage] P [64 r][64 r']
-    static constexpr int St = Pt + (kOut ? kSt * 8192 : 0);   // S^T staging for its store [2 kblk][d_v][64]
+    static constexpr int Kt = Wt + kStages * kTile;       // [stage] K    [2][64 r][64 d_k]
+    static constexpr int Ut = Kt + kStages * kTile;       // [stage] U^T  [d_v][64 r]
+    static constexpr int St = Ut + kStages * kTile;       // S^T staging for its store [2 kblk][d_v][64]
     static constexpr int Dst = St + 2 * kTile;            // Delta^T staging for its store
-    static constexpr int Ost = Dst + kTile;               // kOut: O staging [2 d_v blk][64 r][64]
-    static constexpr int Ed = Ost + (kOut ? kTile : 0);   // [stage][128] fp32 decay table
-    static constexpr int Bar = Ed + kSt * 512;            // barriers, see the kernel
-    static constexpr int Misc = Bar + (2 * kSt + 14) * 8;  // TMEM base, abort flag
+    static constexpr int Ed = Dst + kTile;                // [stage][128] fp32 decay table
+    static constexpr int Bar = Ed + kStages * 512;        // barriers, see the kernel
+    static constexpr int Misc = Bar + (kStages + 10) * 8;  // TMEM base, abort flag
     static constexpr int Size = Misc + 16;
 };
 
@@ -125,56 +118,27 @@ __device__ __forceinline__ void put_row32(uint8_t* tile, int row, int q0, const 
 //   bar_dst  Delta^T staged for its store      bar_dfree  that store has read the tile
 // TMEM (512 columns): X^T [0, 64), P^T [64, 192), S^T operand [192, 256),
 // Delta^T operand [256, 288).
-//
-// With kOut the same CTA also forms the chunk's output, the fused forward: the
-// state pass and the output of the StateFlow summary's block kernel run as one
-// warp-specialised pass, so the chunk states and Delta are not read back from
-// global memory.  Per chunk, off the dependent chain,
-//   O^T = S^T (diag(gamma) Q)^T + Delta^T P^T     (M = 128 UMMAs into tO[c % 2])
-// with S^T the TMEM operand already in place, Q scaled by gamma in its tile,
-// Delta^T the staging tile of its store and P the tile the intra-chunk kernel
-// stored.  The chain thread issues S^T Qg^T behind X^T and Delta^T P^T behind
-// P^T; the element-wise warps write O (token-major bf16) for chunk c - 1 while
-// P^T of chunk c runs, and the copy thread stores it.  Each ring stage loads in
-// two parts: the chain's operands (W^T, U^T, K, the decay table) as soon as the
-// chain products of the stage's previous chunk are done, the output's (Q, P)
-// once its Delta^T P^T has run.  Further hand-overs:
-//   bar_q    Q of chunk c scaled by gamma      bar_o  Delta^T P^T of chunk c done (commit)
-//   bar_pfree  Delta^T P^T of chunk c - 1 seen done (Q and P of its stage may be reloaded)
-//   bar_ost  O staged for its store            bar_ofree  that store has read the tile
-//   bar_ldo[s]  Q and P of stage s landed
-// TMEM: tO[0] [288, 352), tO[1] [352, 416).
-template <bool kDelta, bool kOut>
+template <bool kDelta>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     state_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_wt,
                         const __grid_constant__ CUtensorMap tm_ut,
                         const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_sc,
-                        const __grid_constant__ CUtensorMap tm_dt,
-                        const __grid_constant__ CUtensorMap tm_q,
-                        const __grid_constant__ CUtensorMap tm_p,
-                        const __grid_constant__ CUtensorMap tm_o, const Args a) {
-    using L = FwdSmem<kOut>;
-    constexpr int kSt = L::kSt;
+                        const __grid_constant__ CUtensorMap tm_dt, const Args a) {
+    using L = FwdSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     float* Eds = (float*)(sm + L::Ed);
-    uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);  // [kSt], count 1
-    uint64_t* bar_x = bar_ld + kSt;               // count 1 (commits)
+    uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);  // [kStages], count 1
+    uint64_t* bar_x = bar_ld + kStages;           // count 1 (commits)
     uint64_t* bar_p = bar_x + 1;
     uint64_t* bar_s = bar_x + 2;                  // count 16 (one arrival per element-wise warp)
     uint64_t* bar_d = bar_x + 3;
     uint64_t* bar_sst = bar_x + 4;
     uint64_t* bar_dst = bar_x + 5;
-    uint64_t* bar_sfree = bar_x + 6;              // count 1 (the copy thread)
+    uint64_t* bar_sfree = bar_x + 6;              // count 1 (the issuer)
     uint64_t* bar_dfree = bar_x + 7;
     uint64_t* bar_fin = bar_x + 8;                // count 2 (both issuers)
-    uint64_t* bar_q = bar_x + 9;                  // kOut: count 16
-    uint64_t* bar_o = bar_x + 10;                 // kOut: count 1 (commit)
-    uint64_t* bar_pfree = bar_x + 11;             // kOut: count 16
-    uint64_t* bar_ost = bar_x + 12;               // kOut: count 16
-    uint64_t* bar_ofree = bar_x + 13;             // kOut: count 1 (the copy thread)
-    uint64_t* bar_ldo = bar_x + 14;               // kOut: [kSt] Q and P of a stage landed, count 1
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
     volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
 
@@ -185,10 +149,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int NC = a.NC;
 
     if (tid == kFwdCopy) {
-        for (int i = 0; i < 2 * kSt + 14; ++i) {
-            const int k = i - kSt;  // 2..5, 9, 11, 12: the element-wise hand-overs; 8: both issuers
-            const bool ew = (k >= 2 && k <= 5) || k == 9 || k == 11 || k == 12;
-            mbar_init(bar_ld + i, ew ? 16 : (k == 8 ? 2 : 1));
+        for (int i = 0; i < kStages + 9; ++i) {
+            const int k = i - kStages;  // 2..5: the element-wise hand-overs; 8: both issuers
+            mbar_init(bar_ld + i, (k >= 2 && k <= 5) ? 16 : (k == 8 ? 2 : 1));
         }
         *s_abort = 0;
         fence_barrier_init();
@@ -198,7 +161,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    const uint32_t tX = tmem, tP = tmem + 64, tS = tmem + 192, tD = tmem + 256, tO0 = tmem + 288;
+    const uint32_t tX = tmem, tP = tmem + 64, tS = tmem + 192, tD = tmem + 256;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
 
     // the issuers' waits: a wait that gives up flags the abort; later waits are skipped
@@ -212,11 +175,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
     };
     if (tid == kFwdChain) {
-        // ---------------- the chain's UMMAs (and, with kOut, the output's)
+        // ---------------- the chain's UMMAs
         for (int c = 0; c < NC; ++c) {
-            const int s = c % kSt;
+            const int s = c % kStages;
             const uint32_t par = c & 1;
-            iwait(&bar_ld[s], (c / kSt) & 1, kErrTimeoutTma);
+            iwait(&bar_ld[s], (c / kStages) & 1, kErrTimeoutTma);
             iwait(bar_s, par, kErrTimeoutMma);  // S^T entering chunk c is in TMEM
             if (ok && kDelta) {
                 tc_fence_after();
@@ -227,19 +190,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     mma_bf16_ts(tX, tS + 8 * ks, sdesc(b0 + ks * 2048, 8192, 1024), id, ks > 0);
             }
             mma_commit(bar_x);
-            if (kOut) {
-                iwait(&bar_ldo[s], (c / kSt) & 1, kErrTimeoutTma);
-                iwait(bar_q, par, kErrTimeoutMma);  // Q of chunk c scaled by gamma
-                if (ok) {
-                    tc_fence_after();
-                    const uint32_t qb = smem_u32(sm + L::Qt + s * kTile);
-                    constexpr uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)  // S^T (diag(gamma) Q)^T into tO[c % 2]
-                        mma_bf16_ts(tO0 + (c & 1) * 64, tS + 8 * ks,
-                                    sdesc(qb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id, ks > 0);
-                }
-            }
             iwait(bar_d, par, kErrTimeoutMma);  // (e^{G_C - G} Delta)^T is in TMEM
             if (ok) {
                 tc_fence_after();
@@ -250,27 +200,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     mma_bf16_ts(tP, tD + 8 * ks, sdesc(b0 + ks * 2048, 8192, 1024), id, ks > 0);
             }
             mma_commit(bar_p);
-            if (kOut) {
-                iwait(bar_dst, par, kErrTimeoutMma);  // Delta^T staged (its store's tile)
-                if (ok) {
-                    tc_fence_after();
-                    const uint32_t dsb = smem_u32(sm + L::Dst), pb = smem_u32(sm + L::Pt + s * 8192);
-                    constexpr uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)  // + Delta^T P^T
-                        mma_bf16(tO0 + (c & 1) * 64, sdesc(dsb + ks * 32, 16, 1024), sdesc(pb + ks * 32, 16, 1024),
-                                 id, 1);
-                }
-                mma_commit(bar_o);
-            }
         }
         if (!ok) atomicExch(a.err, err);
         mma_commit(bar_fin);  // every UMMA issued has finished before the TMEM is freed
         mbar_wait(bar_fin, 0);
     } else if (tid == kFwdCopy) {
         // ---------------- copies and stores
-        auto issue_load = [&](int c) {  // the chain's operands of chunk c
-            const int s = c % kSt;
+        auto issue_load = [&](int c) {
+            const int s = c % kStages;
             const uint32_t bytes = (kDelta ? kTile : 0) + 2 * kTile + 512;
             mbar_expect_tx(&bar_ld[s], bytes);
             if (kDelta) tma_load_2d(sm + L::Wt + s * kTile, &tm_wt, 0, (bh * NC + c) * kD, &bar_ld[s]);
@@ -279,34 +216,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tma_load_4d(sm + L::Kt + s * kTile + kTile / 2, &tm_k, 64, h, c * kChunk, b, &bar_ld[s]);
             bulk_load(Eds + s * 128, a.Ed + ((size_t)bh * NC + c) * 128, 512, &bar_ld[s]);
         };
-        auto issue_load_out = [&](int c) {  // kOut: the output's operands of chunk c
-            const int s = c % kSt;
-            mbar_expect_tx(&bar_ldo[s], kTile + 8192);
-            tma_load_4d(sm + L::Qt + s * kTile, &tm_q, 0, h, c * kChunk, b, &bar_ldo[s]);
-            tma_load_4d(sm + L::Qt + s * kTile + kTile / 2, &tm_q, 64, h, c * kChunk, b, &bar_ldo[s]);
-            tma_load_2d(sm + L::Pt + s * 8192, &tm_p, 0, (bh * NC + c) * kChunk, &bar_ldo[s]);
-        };
-        auto store_o = [&](int c) {  // O of chunk c, token-major (rows past the piece's end are clipped)
-            tma_store_4d(&tm_o, sm + L::Ost, 0, h, c * kChunk, b);
-            tma_store_4d(&tm_o, sm + L::Ost + kTile / 2, 64, h, c * kChunk, b);
-        };
         int issued = 0;
-        for (; issued < min(kSt, NC); ++issued) {
-            issue_load(issued);
-            if (kOut) issue_load_out(issued);
-        }
+        for (; issued < min(kStages, NC); ++issued) issue_load(issued);
         for (int c = 0; c < NC; ++c) {
             const uint32_t par = c & 1;
             // the stage of chunk c-1 is free once S^T of chunk c is handed over: the products
             // of c-1 are done and the element-wise warps have read its tiles (waited before
-            // bar_dfree below lets them reach the next hand-over of S^T); with the output, its
-            // Q and P once Delta^T P^T of c-1 has run (bar_pfree: the warps have seen its commit)
+            // bar_dfree below lets them reach the next hand-over of S^T)
             iwait(bar_s, par, kErrTimeoutMma);
-            const bool reload = c >= 1 && issued < NC;
-            if (ok && reload) issue_load(issued);
-            if (kOut && c >= 1) iwait(bar_pfree, (c - 1) & 1, kErrTimeoutMma);
-            if (kOut && ok && reload) issue_load_out(issued);
-            if (reload) ++issued;
+            if (ok && c >= 1 && issued < NC) {
+                issue_load(issued);
+                ++issued;
+            }
             // the chunk state entering c to global memory, staged while X^T is computed
             iwait(bar_sst, par, kErrTimeoutMma);
             if (ok) {
@@ -314,37 +235,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 tma_store_2d(&tm_sc, sm + L::St + kTile, 64, (bh * NC + c) * kD);
             }
             bulk_commit();
-            bulk_wait_read<1>();  // the Delta^T store of chunk c-1 (and O of c-2) have read their tiles
+            bulk_wait_read<1>();  // the Delta^T store of chunk c-1 has read its tile
             if (c > 0) mbar_arrive(bar_dfree);
-            if (kOut && c > 0) mbar_arrive(bar_ofree);
             iwait(bar_dst, par, kErrTimeoutMma);
             if (ok) tma_store_2d(&tm_dt, sm + L::Dst, 0, (bh * NC + c) * kD);
             bulk_commit();
-            if (kOut && c > 0) {
-                iwait(bar_ost, (c - 1) & 1, kErrTimeoutMma);  // O of chunk c-1 staged
-                if (ok) store_o(c - 1);
-                bulk_commit();
-                bulk_wait_read<2>();  // the S^T store of chunk c has read its tile
-            } else {
-                bulk_wait_read<1>();
-            }
+            bulk_wait_read<1>();  // the S^T store of chunk c has read its tile
             mbar_arrive(bar_sfree);
-        }
-        if (kOut && NC > 0) {  // O of the last chunk
-            bulk_wait_read<0>();
-            if (NC > 1) mbar_arrive(bar_ofree);  // O of chunk NC - 2 has been read
-            iwait(bar_ost, (NC - 1) & 1, kErrTimeoutMma);
-            if (ok) store_o(NC - 1);
-            bulk_commit();
         }
         if (!ok) atomicExch(a.err, err);
         // teardown: copies still in flight land and the stores have read shared memory
         // before the CTA exits
         if (*s_abort)
-            for (int cc = 0; cc < issued; ++cc) {
-                mbar_wait(&bar_ld[cc % kSt], (cc / kSt) & 1);
-                if (kOut) mbar_wait(&bar_ldo[cc % kSt], (cc / kSt) & 1);
-            }
+            for (int cc = 0; cc < issued; ++cc) mbar_wait(&bar_ld[cc % kStages], (cc / kStages) & 1);
         mma_commit(bar_fin);
         mbar_wait(bar_fin, 0);
         bulk_wait_read<0>();
@@ -372,25 +275,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar);
         };
-        // O of chunk cc (kOut): O[r][j] = (S^T Qg^T + Delta^T P^T)[j][r] for this thread's
-        // d_v row j and tokens r in [16 part, 16 part + 16), into the token-major staging
-        // tile once the store of the previous O has read it
-        auto emit_o = [&](int cc) {  // after bar_o of chunk cc has been seen
-            // the copy thread's k-th arrival (its iteration k + 1) certifies that O of chunk k - 1
-            // has been read: O of chunk cc - 1 is the cc-th
-            if (cc >= 1) wait(bar_ofree, cc & 1, kErrTimeoutTma);
-            if (bad) return;
-            tc_fence_after();
-            float x[16];
-            tmem_ld16(tO0 + (cc & 1) * 64 + lane_base + part * 16, x);
-            tmem_ld_wait();
-            uint8_t* ost = sm + L::Ost + (j >> 6) * (kTile / 2);
-            const uint32_t jq = (j & 63) >> 3, je = (j & 7) * 2;
-#pragma unroll
-            for (int q = 0; q < 16; ++q)
-                *(__nv_bfloat16*)(ost + sw128(part * 16 + q, jq) + je) = __float2bfloat16_rn(x[q]);
-            hand_over_smem(bar_ost);
-        };
         // S^T row j, state columns i in [32 part, 32 part + 32): S[q] = S_{i, j}
         float S[32];
 #pragma unroll
@@ -399,7 +283,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         uint8_t* St = sm + L::St + (part >> 1) * kTile;
         const int sq0 = (part & 1) * 4;  // first 16-byte chunk of this thread's 32 state columns
         for (int c = 0; c < NC && !bad; ++c) {
-            const int s = c % kSt;
+            const int s = c % kStages;
             const uint32_t par = c & 1;
             // (1) S^T as bf16 pairs into TMEM: the A operand of X^T = S^T W^T
             {
@@ -409,39 +293,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 tmem_st16u(tS + lane_base + 16 * part, w);
             }
             hand_over_tmem(bar_s);
-            const float* E = Eds + s * 128;
-            if (kOut) {
-                // (1a) Delta^T P^T of chunk c - 1 has run: Q and P of its stage may be reloaded
-                if (c > 0) {
-                    wait(bar_o, (c - 1) & 1, kErrTimeoutMma);
-                    if (lane == 0) mbar_arrive(bar_pfree);
-                }
-                // (1b) Q of chunk c scaled by gamma_r in place, 32 bytes of a 128-byte line per thread
-                wait(&bar_ld[s], (c / kSt) & 1, kErrTimeoutTma);
-                wait(&bar_ldo[s], (c / kSt) & 1, kErrTimeoutTma);
-                const int line = tid >> 2, r = line & 63, blk = line >> 6;
-                uint8_t* ln = sm + L::Qt + s * kTile + blk * 8192 + r * 128 + (tid & 3) * 32;
-                const float f = E[64 + r];
-#pragma unroll
-                for (int qq = 0; qq < 2; ++qq) {
-                    uint4 u = *(uint4*)(ln + qq * 16);
-                    uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        const float2 x = unpack_bf16(w[p]);
-                        w[p] = pack_bf16(x.x * f, x.y * f);
-                    }
-                    *(uint4*)(ln + qq * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-                hand_over_smem(bar_q);
-            }
             // (2) the same bf16 S^T staged for its store, once the last one has read the tile
             if (c > 0) wait(bar_sfree, (c - 1) & 1, kErrTimeoutTma);
             put_row32(St, j, sq0, S);
             hand_over_smem(bar_sst);
             // (3) Delta^T[j][r] = U^T[j][r] - X^T[j][r] for tokens r in [16 part, 16 part + 16);
             // e^{G_C - G_r} Delta^T into TMEM (A operand of P^T), Delta^T kept for its store
-            wait(&bar_ld[s], (c / kSt) & 1, kErrTimeoutTma);
+            wait(&bar_ld[s], (c / kStages) & 1, kErrTimeoutTma);
             float X[16];
             if (kDelta) {
                 wait(bar_x, par, kErrTimeoutMma);
@@ -452,6 +310,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
                 for (int q = 0; q < 16; ++q) X[q] = 0.f;
             }
+            const float* E = Eds + s * 128;
             const uint8_t* Ut = sm + L::Ut + s * kTile;
             uint32_t dw[8], tw[8];
 #pragma unroll
@@ -472,15 +331,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             tmem_st8u(tD + lane_base + 8 * part, tw);
             hand_over_tmem(bar_d);
-            // (4) Delta^T staged for its store (and, with kOut, as the A operand of Delta^T P^T)
+            // (4) Delta^T staged for its store
             if (c > 0) wait(bar_dfree, (c - 1) & 1, kErrTimeoutTma);
 #pragma unroll
             for (int qq = 0; qq < 2; ++qq)
                 *(uint4*)(sm + L::Dst + sw128(j, part * 2 + qq)) =
                     make_uint4(dw[qq * 4], dw[qq * 4 + 1], dw[qq * 4 + 2], dw[qq * 4 + 3]);
-            hand_over_smem(bar_dst);  // read by the store (and with kOut by Delta^T P^T)
-            // (4b) O of the previous chunk, while P^T of this one runs
-            if (kOut && c > 0) emit_o(c - 1);
+            hand_over_smem(bar_dst);
             // (5) S^T <- gamma_C S^T + P^T
             wait(bar_p, par, kErrTimeoutMma);
             tc_fence_after();
@@ -490,10 +347,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const float gam = E[64 + kChunk - 1];  // gamma_C
 #pragma unroll
             for (int q = 0; q < 32; ++q) S[q] = gam * S[q] + P[q];
-        }
-        if (kOut && NC > 0) {
-            wait(bar_o, (NC - 1) & 1, kErrTimeoutMma);
-            emit_o(NC - 1);
         }
         if (!bad && a.S_out) {
 #pragma unroll
@@ -872,28 +725,23 @@ bool tc_eligible(const Args& a) {
     return a.dtype == SF_BF16 && a.dk == kD && a.dv == kD;
 }
 
-cudaError_t launch_state_fwd_tc(const Args& a, bool with_output, cudaStream_t s) {
+cudaError_t launch_state_fwd_tc(const Args& a, cudaStream_t s) {
     const int BH = a.B * a.H;
     if (BH == 0 || a.NC == 0) return cudaSuccess;
     const uint64_t rows = (uint64_t)BH * a.NC * kD;
-    CUtensorMap tm_wt{}, tm_ut{}, tm_k{}, tm_sc{}, tm_dt{}, tm_q{}, tm_p{}, tm_o{};
+    CUtensorMap tm_wt{}, tm_ut{}, tm_k{}, tm_sc{}, tm_dt{};
     bool ok = tmap_2d(&tm_ut, a.Ut, 64, rows, 128) && tmap_tokens(&tm_k, a.k, a, kD) &&
               tmap_2d(&tm_sc, a.Sc, kD, rows, 128) && tmap_2d(&tm_dt, a.Dt, 64, rows, 128);
     if (a.beta) ok = ok && tmap_2d(&tm_wt, a.Wt, 64, rows, 128);
-    if (with_output)
-        ok = ok && a.Pm && tmap_tokens(&tm_q, a.q, a, kD) && tmap_tokens(&tm_o, a.o, a, kD) &&
-             tmap_2d(&tm_p, a.Pm, 64, (uint64_t)BH * a.NC * kChunk, 64);
     if (!ok) return cudaErrorInvalidValue;
-    const size_t smem = (with_output ? FwdSmem<true>::Size : FwdSmem<false>::Size) + 1024;
-    auto kern = with_output ? (a.beta ? state_fwd_tc_kernel<true, true> : state_fwd_tc_kernel<false, true>)
-                            : (a.beta ? state_fwd_tc_kernel<true, false> : state_fwd_tc_kernel<false, false>);
+    const size_t smem = FwdSmem::Size + 1024;
+    auto kern = a.beta ? state_fwd_tc_kernel<true> : state_fwd_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int kind = with_output ? KK_STATE_OUT : KK_STATE_FWD;
-    timing_begin(kind, s);
-    kern<<<BH, kFwdThreads, smem, s>>>(tm_wt, tm_ut, tm_k, tm_sc, tm_dt, tm_q, tm_p, tm_o, a);
+    timing_begin(KK_STATE_FWD, s);
+    kern<<<BH, kFwdThreads, smem, s>>>(tm_wt, tm_ut, tm_k, tm_sc, tm_dt, a);
     e = cudaGetLastError();
-    timing_end(kind, s);
+    timing_end(KK_STATE_FWD, s);
     return e;
 }
 

@@ -133,9 +133,8 @@ def chunk_costs(timing: dict, steps: int, n_chunks: int, bh: int, sms: int, min_
         return sum(v[1] for k_, v in timing.items() if k_.startswith(prefix)) * 1e3 / steps / n_chunks
     if min_chunks is None:
         min_chunks = -(-3 * sms // bh)
-    # the fused forward (state_out) carries the output inside the state pass
     return sf.chunk_costs(us("intra"), us("output"), us("grad") + us("dd_pre"),
-                          us("state_fwd") + us("state_out"), us("state_bwd"), sms, min_chunks)
+                          us("state_fwd"), us("state_bwd"), sms, min_chunks)
 
 
 def plan_cut(q, v, n_sub: int, costs) -> list:

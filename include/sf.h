@@ -70,11 +70,12 @@ typedef struct {
 /* Bytes of device workspace sf_fwd (op = SF_OP_FWD) or sf_bwd (SF_OP_BWD) needs
  * for this shape.  Returns 0 for an invalid shape.  The workspace is scratch:
  * its contents need not be preserved between calls, and two calls that may run
- * at the same time must not share one.  The exception is its first 4 bytes, the
- * device error word that bounded device waits set and sf_check reads and
- * clears.  They must be zero before the workspace's first call: allocate it
- * zeroed, or zero those bytes once.  This holds for every workspace the
- * sub-sequence drivers take as well. */
+ * at the same time must not share one.  The exception is its first 16 bytes:
+ * the device error word that bounded device waits set and sf_check reads and
+ * clears (bytes 0-3), and the work counters of the gradient kernel (bytes
+ * 8-15), which every launch leaves at zero.  They must be zero before the
+ * workspace's first call: allocate it zeroed, or zero those bytes once.  This
+ * holds for every workspace the sub-sequence drivers take as well. */
 size_t sf_workspace_bytes(const sf_shape* shape, int op);
 
 /* Forward over one sequence piece of T tokens:
