@@ -67,7 +67,8 @@ constexpr int kHalf = 8192;
 constexpr int kThreads = 512;          // element-wise warps 0-15
 constexpr int kBlock = kThreads + 32;  // + the issuing warp
 constexpr int kIss = kThreads;         // the thread that issues copies, stores and UMMAs
-constexpr int kLoads = 4;              // operand groups, in the order they are needed
+constexpr int kLoads = 5;              // operand groups: four in the order the products need
+                                       // them, and V (read by the element-wise warps)
 
 // Per-row partial sums, each kept per column quarter: [term][quarter][64 rows].
 // Lanes 0-15 and 16-31 of a warp own different terms, and each term is set in
@@ -83,9 +84,10 @@ constexpr int kDgTerms = P_DB_LO;  // terms [0, kDgTerms) go to dG, the rest to 
 
 // Barriers: kLoads copy groups; commits a0 (T^T dDelta), a1 (dO [Delta^T | S^T]),
 // a2 (Q K^T, K K^T), a3 (Delta dS'^T), c0 ([dA | dKhat]), c1 (F K, F^T Q),
-// c2 ((E + E^T) K); hand-overs s_c, s_ab, s_d, s_q and dk (16 arrivals); kfree
-// (the issuer: the item's stores have read their staging tiles); fin.
-constexpr int kNBar = kLoads + 4 + 3 + 5 + 1 + 1;
+// c2 ((E + E^T) K); hand-overs s_c, s_ab, s_d, s_q and dk (16 arrivals); pdfree
+// (the issuer: the dq store has read the PD region); pub (the issuer: the next
+// item is published); fin.
+constexpr int kNBar = kLoads + 4 + 3 + 5 + 1 + 1 + 1;
 
 struct FusedSmem {
     static constexpr int dDt = 0;                 // dDelta^T [128 j][64 r]; later dVhat, bf16 [jblk][64 r][64]
@@ -94,14 +96,15 @@ struct FusedSmem {
     static constexpr int Dt = dO + kTile;         // Delta^T [128 j][64 t]
     static constexpr int St = Dt + kTile;         // S^T [2][128 j][64 i], 16 KB behind Delta^T:
                                                   // [Delta^T | S^T] is one N = 192 operand
-    static constexpr int Q = St + 2 * kTile;      // [dkblk][64 r][64]; later the dq staging
-    static constexpr int K = Q + kTile;           // [dkblk][64 r][64]
+    static constexpr int Q = St + 2 * kTile;      // [dkblk][64 r][64]
+    static constexpr int K = Q + kTile;           // K of even items [dkblk][64 r][64]; then their dk staging
     static constexpr int dSt = K + kTile;         // dS'^T [2][128 j][64 i]; later E, fp32 [64][65]
     static constexpr int F = dSt + 2 * kTile;     // F = dP .* Gamma, bf16 [r][64 t]
     static constexpr int EE = F + kHalf;          // E + E^T, bf16 [r][64 t]
-    static constexpr int dVs = EE + kHalf;        // dv staging [dvblk][64 r][64]
-    static constexpr int dKs = dVs + kTile;       // dk staging [dkblk][64 r][64]
-    static constexpr int PD = dKs + kTile;        // fp32 [64][65]: dP .* P, then + dB .* B
+    static constexpr int dVs = EE + kHalf;        // V [dvblk][64 r][64], then the dv staging
+    static constexpr int K1 = dVs + kTile;        // K of odd items; then their dk staging
+    static constexpr int PD = K1 + kTile;         // fp32 [64][65]: dP .* P, then + dB .* B; then
+                                                  // the dq staging [dkblk][64 r][64]
     static constexpr int Gs = PD + 64 * 65 * 4;   // [item parity][64] fp32
     static constexpr int csp = Gs + 512;          // fp32 [8][64]: column sums of PD over 8-row groups
     static constexpr int part = csp + 8 * 256;    // fp32 [P_COUNT][4][64]
@@ -116,16 +119,9 @@ __device__ __forceinline__ size_t tok_index(const Args& a, int b, int t, int h) 
     return ((size_t)b * a.ld_t + t) * a.H + h;
 }
 
-// Global loads that stay where they are written (read-only data; an asm volatile
-// load is not moved to its first use), so that their latency overlaps the work
-// that follows.
-__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
-    uint4 r;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
+// A global load that stays where it is written (read-only data; an asm volatile
+// load is not moved to its first use), so that its latency overlaps the work that
+// follows.
 __device__ __forceinline__ float ldg_nc_f32(const float* p) {
     float r;
     asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(r) : "l"(p));
@@ -181,7 +177,8 @@ __global__ void __launch_bounds__(kBlock, 1)
                          const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_ddt,
                          const __grid_constant__ CUtensorMap tm_sc, const __grid_constant__ CUtensorMap tm_dsc,
                          const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
-                         const __grid_constant__ CUtensorMap tm_dv, const Args a) {
+                         const __grid_constant__ CUtensorMap tm_dv, const __grid_constant__ CUtensorMap tm_v,
+                         const Args a) {
     using L = FusedSmem;
     extern __shared__ uint8_t smem_raw[];
     // the 1024-byte aligned base, by pointer arithmetic on the shared array (so that every
@@ -197,8 +194,9 @@ __global__ void __launch_bounds__(kBlock, 1)
     uint64_t* bar_c = bar_a + 4;                  // [3] later products done
     uint64_t* bar_s = bar_c + 3;                  // [4] element-wise hand-overs (16 warps): c, ab, d, q
     uint64_t* bar_dk = bar_s + 4;                 // dk read from TMEM and staged (16 warps)
-    uint64_t* bar_kfree = bar_dk + 1;             // the item's stores have read their tiles (issuer)
-    uint64_t* bar_fin = bar_kfree + 1;            // teardown after an abort
+    uint64_t* bar_pdfree = bar_dk + 1;            // the dq store has read the PD region (issuer)
+    uint64_t* bar_pub = bar_pdfree + 1;           // the next item is published (issuer)
+    uint64_t* bar_fin = bar_pub + 1;              // teardown after an abort
     uint32_t* s_tmem = (uint32_t*)(sm + L::Misc);
     volatile int* s_abort = (volatile int*)(sm + L::Misc + 4);
     volatile int* s_item = (volatile int*)(sm + L::Misc + 8);  // [item parity]: chunk-head, or -1
@@ -210,6 +208,9 @@ __global__ void __launch_bounds__(kBlock, 1)
     const bool hi = lane >= 16;                 // lanes 16-31: the hi tiles
     const int r = 16 * quad + (lane & 15);      // chunk row of this thread's tiles
     auto P = [&](int term) { return part + (term * 4 + cq) * 64; };
+    // K of item j (by parity: two tiles, so that the next item's K lands while this one's
+    // is still read)
+    auto k_tile = [&](int j) { return sm + ((j & 1) ? L::K1 : L::K); };
     const int cb = cq * 32 + (hi ? 16 : 0);     // first dVhat column of this thread
 
     // The issuer's copies of one operand group of the CTA's item j, chunk-head n.  The
@@ -242,13 +243,17 @@ __global__ void __launch_bounds__(kBlock, 1)
             mbar_expect_tx(&bar_ld[2], 4 * kHalf + 256);
             tma_load_4d(sm + L::Q, &tm_q, 0, it.h, it.t0, it.b, &bar_ld[2]);
             tma_load_4d(sm + L::Q + kHalf, &tm_q, 64, it.h, it.t0, it.b, &bar_ld[2]);
-            tma_load_4d(sm + L::K, &tm_k, 0, it.h, it.t0, it.b, &bar_ld[2]);
-            tma_load_4d(sm + L::K + kHalf, &tm_k, 64, it.h, it.t0, it.b, &bar_ld[2]);
+            tma_load_4d(k_tile(j), &tm_k, 0, it.h, it.t0, it.b, &bar_ld[2]);
+            tma_load_4d(k_tile(j) + kHalf, &tm_k, 64, it.h, it.t0, it.b, &bar_ld[2]);
             bulk_load(sm + L::Gs + (j & 1) * 256, a.G + (size_t)it.bh * TP + it.t0, 256, &bar_ld[2]);
-        } else {  // dS'^T (Delta dS'^T)
+        } else if (g == 3) {  // dS'^T (Delta dS'^T)
             mbar_expect_tx(&bar_ld[3], 2 * kTile);
             tma_load_2d(sm + L::dSt, &tm_dsc, 0, rowD, &bar_ld[3]);
             tma_load_2d(sm + L::dSt + kTile, &tm_dsc, 64, rowD, &bar_ld[3]);
+        } else {  // V, into the dv staging tile (rows past the piece's end read as zero)
+            mbar_expect_tx(&bar_ld[4], 2 * kHalf);
+            tma_load_4d(sm + L::dVs, &tm_v, 0, it.h, it.t0, it.b, &bar_ld[4]);
+            tma_load_4d(sm + L::dVs + kHalf, &tm_v, 64, it.h, it.t0, it.b, &bar_ld[4]);
         }
         pend |= 1u << g;
         pend_par = (pend_par & ~(1u << g)) | ((uint32_t)(j & 1) << g);
@@ -278,7 +283,7 @@ __global__ void __launch_bounds__(kBlock, 1)
 
     // ---------------- the issuer
     if (tid == kIss) {
-        const uint32_t q = smem_u32(sm + L::Q), k = smem_u32(sm + L::K), dob = smem_u32(sm + L::dO);
+        const uint32_t q = smem_u32(sm + L::Q), dob = smem_u32(sm + L::dO);
         const uint32_t dt = smem_u32(sm + L::Dt), ddt = smem_u32(sm + L::dDt), tb = smem_u32(sm + L::Tb);
         const uint32_t dst = smem_u32(sm + L::dSt);
         constexpr uint32_t idKK = idesc_bf16(64, 64, false, false);
@@ -300,11 +305,11 @@ __global__ void __launch_bounds__(kBlock, 1)
             iwait(&bar_ld[g], (uint32_t)(j & 1));
             if (ok) pend &= ~(1u << g);
         };
-        auto store_dk = [&](int n) {  // rows past the piece's end are clipped
+        auto store_dk = [&](int n, int j) {  // from item j's K tile; rows past the piece's end are clipped
             const Item it = item_of(a, n);
             if (ok) {
-                tma_store_4d(&tm_dk, sm + L::dKs, 0, it.h, it.t0, it.b);
-                tma_store_4d(&tm_dk, sm + L::dKs + kHalf, 64, it.h, it.t0, it.b);
+                tma_store_4d(&tm_dk, k_tile(j), 0, it.h, it.t0, it.b);
+                tma_store_4d(&tm_dk, k_tile(j) + kHalf, 64, it.h, it.t0, it.b);
             }
             bulk_commit();
         };
@@ -324,13 +329,14 @@ __global__ void __launch_bounds__(kBlock, 1)
         int prev = -1, last_j = 0;
         for (int j = 0; cur >= 0; ++j) {
             const uint32_t ph = (uint32_t)(j & 1);
-            // the next item, published for the element-wise warps (they read it after the
-            // hand-over kfree of this item; its slot was last read for item j - 1 before the
-            // hand-over dk of j - 2, waited below in item j - 1)
+            // the next item, published for the element-wise warps (its slot was last read for
+            // item j - 1 in item j - 2, before the hand-over s_q of j - 2)
             const int next = take_item();
             s_item[(j + 1) & 1] = next;
+            mbar_arrive(bar_pub);
             const bool has_next = next >= 0;
             const Item it = item_of(a, cur);
+            const uint32_t k = smem_u32(k_tile(j));
             // dO [Delta^T | S^T]: one N = 192 product, dO Delta^T into lo [64, 128) and dO S^T
             // into lo [128, 256) (Delta^T and S^T lie 16 KB apart in smem); item j-1's dq
             // there was read before its hand-over s_q, waited below for j-1
@@ -363,7 +369,7 @@ __global__ void __launch_bounds__(kBlock, 1)
             // it, then Delta dS'^T of item j into hi [128, 256)
             if (j > 0) {
                 iwait(bar_dk, ph ^ 1u);
-                store_dk(prev);
+                store_dk(prev, j - 1);
             }
             ld_wait(3, j);
             if (ok) {
@@ -406,14 +412,20 @@ __global__ void __launch_bounds__(kBlock, 1)
                 }
             }
             mma_commit(&bar_c[1]);
-            // the next item's dDelta^T, T, dO, Delta^T, S^T: every product reading those tiles
-            // (and the dVhat written over dDelta^T) is done once [dA | dKhat] is, and the
-            // element-wise reads of S^T came before the hand-over s_ab
+            // the next item's operands but dS'^T, once every product reading their tiles is done
+            // (F K, F^T Q, issued last, complete after the others) and the element-wise reads
+            // of S^T and Q came before the hand-over s_ab: dDelta^T (the dVhat written over it
+            // is read), T, dO, Delta^T, S^T, Q and G (item j-1's G was read before its hand-over
+            // dk); V lands in the dv staging tile and K in item j-1's K tile, whose dk was
+            // stored, once the stores of item j-1's dk and item j's dv have read their tiles
             if (has_next) {
-                iwait(&bar_c[0], ph);
+                iwait(&bar_c[1], ph);
+                bulk_wait_read<0>();
                 if (ok) {
                     load_group(0, next, j + 1);
                     load_group(1, next, j + 1);
+                    load_group(4, next, j + 1);
+                    load_group(2, next, j + 1);
                 }
             }
             // dKp = diag(beta gamma) dKhat + (E + E^T) K once E + E^T and the scaled dKhat are written
@@ -429,29 +441,23 @@ __global__ void __launch_bounds__(kBlock, 1)
             mma_commit(&bar_c[2]);
             // the next item's dS'^T: E, written over it, has been consumed
             if (has_next && ok) load_group(3, next, j + 1);
-            // dq, staged in the Q tile (rows past the piece's end are clipped)
+            // dq, staged in the PD region (rows past the piece's end are clipped)
             iwait(&bar_s[3], ph);
             if (ok) {
-                tma_store_4d(&tm_dq, sm + L::Q, 0, it.h, it.t0, it.b);
-                tma_store_4d(&tm_dq, sm + L::Q + kHalf, 64, it.h, it.t0, it.b);
+                tma_store_4d(&tm_dq, sm + L::PD, 0, it.h, it.t0, it.b);
+                tma_store_4d(&tm_dq, sm + L::PD + kHalf, 64, it.h, it.t0, it.b);
             }
             bulk_commit();
-            // the dv and dq stores of item j and the dk store of item j-1 have read their tiles
-            bulk_wait_read<0>();
-            mbar_arrive(bar_kfree);  // releases the s_item write above too
-            if (has_next) {
-                p_dvhat(j + 1);  // runs behind (E + E^T) K
-                // the next item's Q, K, G once (E + E^T) K has read K (F^T Q read Q before it)
-                iwait(&bar_c[2], ph);
-                if (ok) load_group(2, next, j + 1);
-            }
+            if (has_next) p_dvhat(j + 1);  // runs behind (E + E^T) K
+            bulk_wait_read<0>();  // the next item's dP .* P may go to the PD region
+            mbar_arrive(bar_pdfree);
             prev = cur;
             cur = next;
             last_j = j;
         }
         if (prev >= 0) {
             iwait(bar_dk, (uint32_t)(last_j & 1));
-            store_dk(prev);
+            store_dk(prev, last_j);
         }
         if (!ok) *s_abort = 1;
     } else if (warp < 16) {
@@ -472,20 +478,14 @@ __global__ void __launch_bounds__(kBlock, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar);
         };
-        // beta of this thread's row, and the 16 columns of V's row r this thread takes in the
-        // dVhat stage, loaded one item ahead
-        auto pre_load = [&](int n, float& bp, uint4* vp) {
+        // beta of this thread's row in chunk-head n, loaded one item ahead
+        auto beta_of = [&](int n) {
+            if (n < 0) return 0.f;
             const Item it = item_of(a, n);
-            const bool in = r < min(kChunk, a.T - it.t0);
-            bp = in ? ldg_nc_f32(a.beta + tok_index(a, it.b, it.t0 + r, it.h)) : 0.f;
-            const __nv_bfloat16* src = (const __nv_bfloat16*)a.v + tok_index(a, it.b, it.t0 + r, it.h) * kD + cb;
-            vp[0] = in ? ldg_nc_v4(src) : make_uint4(0, 0, 0, 0);
-            vp[1] = in ? ldg_nc_v4(src + 8) : make_uint4(0, 0, 0, 0);
+            return r < min(kChunk, a.T - it.t0) ? ldg_nc_f32(a.beta + tok_index(a, it.b, it.t0 + r, it.h)) : 0.f;
         };
-        float bpre = 0.f;
-        uint4 vpre[2] = {};
         int ecur = s_item[0];  // this item's chunk-head
-        if (ecur >= 0) pre_load(ecur, bpre, vpre);
+        float bpre = beta_of(ecur);
         for (int j = 0; ecur >= 0; ++j) {
             const uint32_t ph = (uint32_t)(j & 1);
             const float* Gs = (const float*)(sm + L::Gs) + (j & 1) * 64;
@@ -496,8 +496,12 @@ __global__ void __launch_bounds__(kBlock, 1)
             // K-major A of [dA | dKhat].  The dv staging tile was read by the last item's store
             // (its release was waited at the end of that item).
             wait_flag(&bar_a[0], ph, kErrTimeoutMma);
+            wait_flag(&bar_ld[4], ph, kErrTimeoutTma);  // V in the dv staging tile
             tc_fence_after();
             {
+                uint8_t* vrow = sm + L::dVs + (cb >> 6) * kHalf;
+                const uint4 vpre[2] = {*(const uint4*)(vrow + sw128(r, (cb & 63) >> 3)),
+                                       *(const uint4*)(vrow + sw128(r, ((cb & 63) >> 3) + 1))};
                 float x[32], y[16];
                 tmem_ld32(c256 + lane_base + cq * 32, x);
                 tmem_ld_wait();
@@ -518,18 +522,24 @@ __global__ void __launch_bounds__(kBlock, 1)
                 }
 #pragma unroll
                 for (int q = 0; q < 16; ++q) dv[q] = br * y[q];
-                put_row(sm + L::dVs + (cb >> 6) * kHalf, r, (cb & 63) >> 3, dv, 16);
+                put_row(vrow, r, (cb & 63) >> 3, dv, 16);  // over the V values this thread read
                 put_row(sm + L::dDt + (cb >> 6) * kHalf, r, (cb & 63) >> 3, y, 16);
                 vd += __shfl_xor_sync(0xffffffffu, vd, 16);
+                if (j > 0 && warp >= 3) named_sync(2, kThreads);  // the last epilogue has read the sums
                 if (!hi) P(P_DB_LO)[r] = vd;
             }
             hand_over(&bar_s[0]);
+            // the next item (published at the issuer's start of this one) and its beta
+            wait_flag(bar_pub, ph, kErrTimeoutMma);
+            const int enext = s_item[(j + 1) & 1];
+            const float bnext = beta_of(enext);
             // (a) P, dP, F on columns [16 cq, 16 cq + 16): lane l < 16 holds (Q K^T)[r] and
             // (dO Delta^T)[r]; it finishes the first 8 columns and hands the last 8 to
             // lane l + 16.  A warp whose columns all lie past its rows (cq > quad) writes
             // the zeros without reading the products.
             wait_flag(&bar_ld[2], ph, kErrTimeoutTma);  // G, Q, K are read below
             wait_flag(&bar_a[2], ph, kErrTimeoutMma);
+            if (j > 0) wait_flag(bar_pdfree, ph ^ 1u, kErrTimeoutTma);  // the last dq store read PD
             tc_fence_after();
             const float Gr = Gs[r];
             float rowpart;
@@ -578,7 +588,7 @@ __global__ void __launch_bounds__(kBlock, 1)
                 float x[32];
                 tmem_ld32(c128 + lane_base + cq * 32, x);
                 tmem_ld_wait();
-                const float dot = dot_row32(sm + (hi ? L::K : L::Q) + (cq >> 1) * kHalf, r, (cq & 1) * 4, x);
+                const float dot = dot_row32((hi ? k_tile(j) : sm + L::Q) + (cq >> 1) * kHalf, r, (cq & 1) * 4, x);
                 float scale, lastpart = 0.f;
                 if (!hi) {
                     scale = __expf(Gr);
@@ -669,7 +679,7 @@ __global__ void __launch_bounds__(kBlock, 1)
 #pragma unroll
                     for (int q = 0; q < 32; ++q) x[q] = -x[q];
                     const float gam = __expf(Gr);
-                    const float kd = dot_row32(sm + L::K + (cq >> 1) * kHalf, r, (cq & 1) * 4, x);
+                    const float kd = dot_row32(k_tile(j) + (cq >> 1) * kHalf, r, (cq & 1) * 4, x);
                     P(P_DB_HI)[r] = gam * kd;
                     P(P_DG_HI)[r] += br * gam * kd;  // set in (b) by this thread
 #pragma unroll
@@ -697,15 +707,16 @@ __global__ void __launch_bounds__(kBlock, 1)
                 csp[g * 64 + col] = s;
             }
             hand_over(&bar_s[2]);
-            // dq (lanes 0-15 of lo [128, 256)) is final once F K has run: its rows into the Q tile
-            // (read by F^T Q, done by then) for the store
+            // dq (lanes 0-15 of lo [128, 256)) is final once F K has run: its rows into the PD
+            // region for the store, once every warp's column sums have read PD
             wait_flag(&bar_c[1], ph, kErrTimeoutMma);
+            named_sync(1, kThreads);
             tc_fence_after();
             {
                 float x[32];
                 tmem_ld32(c128 + lane_base + cq * 32, x);
                 tmem_ld_wait();
-                if (!hi) put_row(sm + L::Q + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);
+                if (!hi) put_row(sm + L::PD + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);
             }
             hand_over(&bar_s[3]);
             named_sync(1, kThreads);  // the per-row partial sums and column sums of every warp
@@ -750,17 +761,16 @@ __global__ void __launch_bounds__(kBlock, 1)
                     a.dbeta[tok_index(a, b, t0 + rr, h)] = db;
                 }
             }
-            // the sums above are read before the next item's stages write them again
-            named_sync(1, kThreads);
+            // the sums above are read before the next item's stages write them again: the
+            // warps that read them arrive on barrier 2, the others wait on it before their
+            // first write of the next item, in (c) (no arrival after the last item)
+            if (warp < 3 && enext >= 0) named_arrive(2, kThreads);
             // dk = dK (hi [128, 256)) + dKp (hi [320, 448)), columns [32 cq, 32 cq + 32), staged
-            // once the last item's dk store has read the staging tile; the hand-over lets the
-            // issuer store it and reuse those TMEM columns
+            // in this item's K tile (read for the last time by (E + E^T) K, and by every warp
+            // before the dq stage's barrier); the hand-over lets the issuer store it and reuse
+            // those TMEM columns
             wait_flag(&bar_c[2], ph, kErrTimeoutMma);
             tc_fence_after();
-            wait_flag(bar_kfree, ph, kErrTimeoutTma);
-            // the next item (published before kfree) and its beta and V row
-            const int enext = s_item[(j + 1) & 1];
-            if (enext >= 0) pre_load(enext, bpre, vpre);
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 float x[16], y[16];
@@ -770,11 +780,12 @@ __global__ void __launch_bounds__(kBlock, 1)
                 if (hi) {
 #pragma unroll
                     for (int q = 0; q < 16; ++q) x[q] += y[q];
-                    put_row(sm + L::dKs + (cq >> 1) * kHalf, r, (cq & 1) * 4 + hf * 2, x, 16);
+                    put_row(k_tile(j) + (cq >> 1) * kHalf, r, (cq & 1) * 4 + hf * 2, x, 16);
                 }
             }
             hand_over(bar_dk);
             ecur = enext;
+            bpre = bnext;
         }
     }
     __syncthreads();
@@ -824,13 +835,13 @@ cudaError_t launch_grad_fused_tc(const Args& a, cudaStream_t s) {
     if (BH == 0 || a.NC == 0) return cudaSuccess;
     const uint64_t rows = (uint64_t)BH * a.NC * kD, rowsC = (uint64_t)BH * a.NC * kChunk;
     CUtensorMap tm_q{}, tm_k{}, tm_do{}, tm_t{}, tm_dt{}, tm_ddt{}, tm_sc{}, tm_dsc{};
-    CUtensorMap tm_dq{}, tm_dk{}, tm_dv{};
+    CUtensorMap tm_dq{}, tm_dk{}, tm_dv{}, tm_v{};
     const bool ok = tmap_tokens(&tm_q, a.q, a, kD) && tmap_tokens(&tm_k, a.k, a, kD) &&
                     tmap_tokens(&tm_do, a.dO, a, kD) && tmap_2d(&tm_t, a.Tm, 64, rowsC, 64) &&
                     tmap_2d(&tm_dt, a.Dt, 64, rows, 128) && tmap_2d(&tm_ddt, a.dDt, 64, rows, 128) &&
                     tmap_2d(&tm_sc, a.Sc, kD, rows, 128) && tmap_2d(&tm_dsc, a.dSc, kD, rows, 128) &&
                     tmap_tokens(&tm_dq, a.dq, a, kD) && tmap_tokens(&tm_dk, a.dk_, a, kD) &&
-                    tmap_tokens(&tm_dv, a.dv_, a, kD);
+                    tmap_tokens(&tm_dv, a.dv_, a, kD) && tmap_tokens(&tm_v, a.v, a, kD);
     if (!ok) return cudaErrorInvalidValue;
     const size_t smem = FusedSmem::Size + 1024;
     cudaError_t e = cudaFuncSetAttribute(grad_fused_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -844,7 +855,7 @@ cudaError_t launch_grad_fused_tc(const Args& a, cudaStream_t s) {
                                       : std::max(sms + a.grad_sms, sms / 2);
     const int ctas = std::min(a.NC * BH, budget);
     grad_fused_tc_kernel<<<ctas, kBlock, smem, s>>>(tm_q, tm_k, tm_do, tm_t, tm_dt, tm_ddt, tm_sc, tm_dsc, tm_dq,
-                                                     tm_dk, tm_dv, a);
+                                                     tm_dk, tm_dv, tm_v, a);
     e = cudaGetLastError();
     timing_end(KK_GRAD_FUSED, s);
     return e;

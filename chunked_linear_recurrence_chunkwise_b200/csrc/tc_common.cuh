@@ -58,6 +58,12 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 __device__ __forceinline__ void named_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
+// Arrival on named barrier `id` without waiting; the threads that wait use named_sync
+// with the same count, and the arrival orders this thread's earlier accesses before
+// their later ones.
+__device__ __forceinline__ void named_arrive(int id, int n) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 // Waits for phase `parity` of `bar` to complete; false if kWaitCycles elapse first.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     const long long t0 = clock64();
