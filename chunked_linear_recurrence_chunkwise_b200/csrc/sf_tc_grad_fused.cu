@@ -108,8 +108,9 @@ struct FusedSmem {
     static constexpr int Gs = PD + 64 * 65 * 4;   // [item parity][64] fp32
     static constexpr int csp = Gs + 512;          // fp32 [8][64]: column sums of PD over 8-row groups
     static constexpr int part = csp + 8 * 256;    // fp32 [P_COUNT][4][64]
-    static constexpr int red = part + P_COUNT * 4 * 256;  // fp32 [32]: per-warp <S, dS'>, last-row sums
-    static constexpr int Bar = red + 128;
+    static constexpr int red = part + P_COUNT * 4 * 256;  // fp32 [32]: per-warp <S, dS'>, last-row sums;
+                                                          // [32]: the dG sum of rows 32-63
+    static constexpr int Bar = red + 256;
     static constexpr int Misc = Bar + kNBar * 8;
     static constexpr int Size = Misc + 16;
 };
@@ -218,11 +219,10 @@ __global__ void __launch_bounds__(kBlock, 1)
     // marks the groups whose armed phase the issuer has not yet seen complete, and
     // `pend_par` that phase's parity.
     uint32_t pend = 0, pend_par = 0;
-    // the next chunk-head of this CTA (the issuer takes them), or -1 once none is left
-    auto take_item = [&]() {
-        const int n = (int)atomicAdd(a.ticket, 1u);
-        return n < total ? n : -1;
-    };
+    // the next ticket of this CTA (the issuer takes them): chunk-head `ticket` while it is
+    // below `total`
+    auto take_item = [&]() { return atomicAdd(a.ticket, 1u); };
+    auto item_or_none = [&](unsigned t) { return t < (unsigned)total ? (int)t : -1; };
     int cur = -1;  // the issuer's current chunk-head
     auto load_group = [&](int g, int n, int j) {
         const Item it = item_of(a, n);
@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(kBlock, 1)
             mbar_init(bar_ld + i, hand ? 16 : 1);
         }
         *s_abort = 0;
-        cur = take_item();
+        cur = item_or_none(take_item());
         s_item[0] = cur;
         fence_barrier_init();
         if (cur >= 0)
@@ -327,13 +327,21 @@ __global__ void __launch_bounds__(kBlock, 1)
         };
         if (cur >= 0) p_dvhat(0);
         int prev = -1, last_j = 0;
+        // the ticket after the next one is taken an item ahead, so that the counter's round
+        // trip overlaps an item's work (its value is first looked at in the next item)
+        unsigned nxt = cur >= 0 ? take_item() : ~0u;
         for (int j = 0; cur >= 0; ++j) {
             const uint32_t ph = (uint32_t)(j & 1);
             // the next item, published for the element-wise warps (its slot was last read for
             // item j - 1 in item j - 2, before the hand-over s_q of j - 2)
-            const int next = take_item();
+            const int next = item_or_none(nxt);
             s_item[(j + 1) & 1] = next;
             mbar_arrive(bar_pub);
+            if (j > 0) {  // item j-1's dq store has read the PD region: this item's dP .* P may go there
+                bulk_wait_read<0>();
+                mbar_arrive(bar_pdfree);
+            }
+            nxt = next >= 0 ? take_item() : ~0u;
             const bool has_next = next >= 0;
             const Item it = item_of(a, cur);
             const uint32_t k = smem_u32(k_tile(j));
@@ -415,9 +423,10 @@ __global__ void __launch_bounds__(kBlock, 1)
             // the next item's operands but dS'^T, once every product reading their tiles is done
             // (F K, F^T Q, issued last, complete after the others) and the element-wise reads
             // of S^T and Q came before the hand-over s_ab: dDelta^T (the dVhat written over it
-            // is read), T, dO, Delta^T, S^T, Q and G (item j-1's G was read before its hand-over
-            // dk); V lands in the dv staging tile and K in item j-1's K tile, whose dk was
-            // stored, once the stores of item j-1's dk and item j's dv have read their tiles
+            // is read), T, dO, Delta^T, S^T, Q and G (item j-1's epilogue read its G before item
+            // j's hand-over s_ab); V lands in the dv staging tile and K in item j-1's K tile,
+            // whose dk was stored, once the stores of item j-1's dk and item j's dv have read
+            // their tiles
             if (has_next) {
                 iwait(&bar_c[1], ph);
                 bulk_wait_read<0>();
@@ -449,8 +458,6 @@ __global__ void __launch_bounds__(kBlock, 1)
             }
             bulk_commit();
             if (has_next) p_dvhat(j + 1);  // runs behind (E + E^T) K
-            bulk_wait_read<0>();  // the next item's dP .* P may go to the PD region
-            mbar_arrive(bar_pdfree);
             prev = cur;
             cur = next;
             last_j = j;
@@ -486,10 +493,61 @@ __global__ void __launch_bounds__(kBlock, 1)
         };
         int ecur = s_item[0];  // this item's chunk-head
         float bpre = beta_of(ecur);
+        // Epilogue of chunk-head n, the CTA's item jj, by warps 0-3: dg and dbeta from the
+        // per-row partial sums and column sums.  It runs in the next item while that one
+        // waits for its first products (or after the last item).
+        auto epilogue = [&](int n, int jj) {
+            const Item it = item_of(a, n);
+            const int b = it.b, h = it.h, t0 = it.t0, Lr = min(kChunk, a.T - t0);
+            const float* Gp = (const float*)(sm + L::Gs) + (jj & 1) * 64;
+            if (warp == 0 || warp == 3) {
+                // dG of row rr (warp 0: rows 0-31, warp 3: rows 32-63) and dg = its reverse
+                // in-chunk cumsum; warp 3 hands the sum of its rows to warp 0 on barrier 3
+                const int rr = (warp == 0 ? 0 : 32) + lane;
+                float g = 0.f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) g -= csp[i * 64 + rr];
+#pragma unroll
+                for (int pi = 0; pi < kDgTerms * 4; ++pi) g += part[pi * 64 + rr];
+                if (warp == 3) {
+                    // the last row's terms: sum_w <S, dS'>_w (lanes 0-15) and the last-row
+                    // sums (lanes 16-31)
+                    float v = red[lane];
+#pragma unroll
+                    for (int off = 8; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                    const float sdot = __shfl_sync(0xffffffffu, v, 0);
+                    if (rr == kChunk - 1) g += v + __expf(Gp[kChunk - 1]) * sdot;
+                }
+                float incl = g;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_down_sync(0xffffffffu, incl, off);
+                    if (lane + off < 32) incl += y;
+                }
+                if (warp == 3) {
+                    if (lane == 0) red[32] = incl;
+                    named_arrive(3, 64);
+                } else {
+                    named_sync(3, 64);
+                    incl += red[32];
+                }
+                if (a.g && rr < Lr) a.dg[tok_index(a, b, t0 + rr, h)] = incl;
+            } else if (warp == 1 || warp == 2) {  // dbeta
+                const int rr = tid - 32;
+                if (rr < Lr) {
+                    float db = 0.f;
+#pragma unroll
+                    for (int pi = kDgTerms * 4; pi < P_COUNT * 4; ++pi) db += part[pi * 64 + rr];
+                    a.dbeta[tok_index(a, b, t0 + rr, h)] = db;
+                }
+            }
+        };
+        int eprev = -1, last_j = 0;  // the last item's chunk-head and index
         for (int j = 0; ecur >= 0; ++j) {
             const uint32_t ph = (uint32_t)(j & 1);
             const float* Gs = (const float*)(sm + L::Gs) + (j & 1) * 64;
             const float br = bpre;
+            float vdr;  // <V_r, dVhat_r> (lanes 0-15), set down in (a)
             // (c) dVhat (lo [256, 384), columns [32 cq, 32 cq + 32)): lane l < 16 reads row r and
             // hands columns 16-31 of its 32 to lane l + 16, so each thread takes 16 columns from
             // cb: dv = beta_r dVhat for its store, <V_r, dVhat_r>, and dVhat in bf16 as the
@@ -525,14 +583,21 @@ __global__ void __launch_bounds__(kBlock, 1)
                 put_row(vrow, r, (cb & 63) >> 3, dv, 16);  // over the V values this thread read
                 put_row(sm + L::dDt + (cb >> 6) * kHalf, r, (cb & 63) >> 3, y, 16);
                 vd += __shfl_xor_sync(0xffffffffu, vd, 16);
-                if (j > 0 && warp >= 3) named_sync(2, kThreads);  // the last epilogue has read the sums
-                if (!hi) P(P_DB_LO)[r] = vd;
+                vdr = vd;
             }
             hand_over(&bar_s[0]);
             // the next item (published at the issuer's start of this one) and its beta
             wait_flag(bar_pub, ph, kErrTimeoutMma);
             const int enext = s_item[(j + 1) & 1];
             const float bnext = beta_of(enext);
+            // the last item's epilogue (warps 0-3); once all four have read the sums (barrier
+            // 4) they arrive on barrier 2, on which the other warps wait before their first
+            // write of the sums, in (a)
+            if (j > 0 && warp < 4) {
+                epilogue(eprev, j - 1);
+                named_sync(4, 128);
+                named_arrive(2, kThreads);
+            }
             // (a) P, dP, F on columns [16 cq, 16 cq + 16): lane l < 16 holds (Q K^T)[r] and
             // (dO Delta^T)[r]; it finishes the first 8 columns and hands the last 8 to
             // lane l + 16.  A warp whose columns all lie past its rows (cq > quad) writes
@@ -540,6 +605,8 @@ __global__ void __launch_bounds__(kBlock, 1)
             wait_flag(&bar_ld[2], ph, kErrTimeoutTma);  // G, Q, K are read below
             wait_flag(&bar_a[2], ph, kErrTimeoutMma);
             if (j > 0) wait_flag(bar_pdfree, ph ^ 1u, kErrTimeoutTma);  // the last dq store read PD
+            if (j > 0 && warp >= 4) named_sync(2, kThreads);  // the last epilogue has read the sums
+            if (!hi) P(P_DB_LO)[r] = vdr;
             tc_fence_after();
             const float Gr = Gs[r];
             float rowpart;
@@ -708,7 +775,8 @@ __global__ void __launch_bounds__(kBlock, 1)
             }
             hand_over(&bar_s[2]);
             // dq (lanes 0-15 of lo [128, 256)) is final once F K has run: its rows into the PD
-            // region for the store, once every warp's column sums have read PD
+            // region for the store, once every warp's column sums have read PD (the barrier
+            // also completes every warp's partial sums for the epilogue)
             wait_flag(&bar_c[1], ph, kErrTimeoutMma);
             named_sync(1, kThreads);
             tc_fence_after();
@@ -719,52 +787,6 @@ __global__ void __launch_bounds__(kBlock, 1)
                 if (!hi) put_row(sm + L::PD + (cq >> 1) * kHalf, r, (cq & 1) * 4, x, 32);
             }
             hand_over(&bar_s[3]);
-            named_sync(1, kThreads);  // the per-row partial sums and column sums of every warp
-            // ---------------- epilogue: dg and dbeta while (E + E^T) K runs, then dk
-            const Item it = item_of(a, ecur);
-            const int b = it.b, h = it.h, t0 = it.t0, Lr = min(kChunk, a.T - t0);
-            if (warp == 0) {  // dG and dg = reverse in-chunk cumsum
-                float sdot = 0.f, last = 0.f;
-#pragma unroll
-                for (int w = 0; w < 16; ++w) {
-                    sdot += red[w];
-                    last += red[16 + w];
-                }
-                float v2[2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int rr = 2 * lane + e;
-                    float g = 0.f;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) g -= csp[i * 64 + rr];
-#pragma unroll
-                    for (int pi = 0; pi < kDgTerms * 4; ++pi) g += part[pi * 64 + rr];
-                    if (rr == kChunk - 1) g += last + __expf(Gs[kChunk - 1]) * sdot;
-                    v2[e] = g;
-                }
-                float incl = v2[0] + v2[1];
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float y = __shfl_down_sync(0xffffffffu, incl, off);
-                    if (lane + off < 32) incl += y;
-                }
-                if (a.g) {
-                    if (2 * lane < Lr) a.dg[tok_index(a, b, t0 + 2 * lane, h)] = incl;
-                    if (2 * lane + 1 < Lr) a.dg[tok_index(a, b, t0 + 2 * lane + 1, h)] = incl - v2[0];
-                }
-            } else if (warp == 1 || warp == 2) {  // dbeta
-                const int rr = tid - 32;
-                if (rr < Lr) {
-                    float db = 0.f;
-#pragma unroll
-                    for (int pi = kDgTerms * 4; pi < P_COUNT * 4; ++pi) db += part[pi * 64 + rr];
-                    a.dbeta[tok_index(a, b, t0 + rr, h)] = db;
-                }
-            }
-            // the sums above are read before the next item's stages write them again: the
-            // warps that read them arrive on barrier 2, the others wait on it before their
-            // first write of the next item, in (c) (no arrival after the last item)
-            if (warp < 3 && enext >= 0) named_arrive(2, kThreads);
             // dk = dK (hi [128, 256)) + dKp (hi [320, 448)), columns [32 cq, 32 cq + 32), staged
             // in this item's K tile (read for the last time by (E + E^T) K, and by every warp
             // before the dq stage's barrier); the hand-over lets the issuer store it and reuse
@@ -784,9 +806,12 @@ __global__ void __launch_bounds__(kBlock, 1)
                 }
             }
             hand_over(bar_dk);
+            eprev = ecur;
             ecur = enext;
             bpre = bnext;
+            last_j = j;
         }
+        if (eprev >= 0 && warp < 4) epilogue(eprev, last_j);
     }
     __syncthreads();
     if (tid == kIss) {
