@@ -83,7 +83,7 @@ enum PartTerm {
 constexpr int kDgTerms = P_DB_LO;  // terms [0, kDgTerms) go to dG, the rest to dbeta
 
 // Barriers: kLoads copy groups; commits a0 (T^T dDelta), a1 (dO [Delta^T | S^T]),
-// a2 (Q K^T, K K^T), a3 (Delta dS'^T), c0 ([dA | dKhat]), c1 (F K, F^T Q),
+// a2 (Q K^T), a3 (Delta dS'^T), c0 (K K^T, [dA | dKhat]), c1 (F K, F^T Q),
 // c2 ((E + E^T) K); hand-overs s_c, s_ab, s_d, s_q and dk (16 arrivals); pdfree
 // (the issuer: the dq store has read the PD region); pub (the issuer: the next
 // item is published); fin.
@@ -366,11 +366,6 @@ __global__ void __launch_bounds__(kBlock, 1)
                     const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
                     mma_bf16(c0, sdesc(q + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);  // Q K^T
                 }
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
-                    mma_bf16(c384, sdesc(k + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);  // K K^T
-                }
             }
             mma_commit(&bar_a[2]);
             // item j-1's dk has been read from hi [128, 256) and [320, 448) and staged: store
@@ -388,6 +383,15 @@ __global__ void __launch_bounds__(kBlock, 1)
                              idMM2, ks > 0);  // Delta dS'^T
             }
             mma_commit(&bar_a[3]);
+            // K K^T, read in (d) after the commit of [dA | dKhat]; issued here so that the
+            // commits that (a) and (b) wait on come before it
+            if (ok) {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
+                    mma_bf16(c384, sdesc(k + o, 16, 1024), sdesc(k + o, 16, 1024), idKK, ks > 0);
+                }
+            }
             // dVhat is staged in bf16 (and dv for its store): [dA | dKhat] = -dVhat [Delta^T | S^T]
             // (the sign is taken by the element-wise warps), N = 192 into hi [256, 448)
             iwait(&bar_s[0], ph);
@@ -432,8 +436,8 @@ __global__ void __launch_bounds__(kBlock, 1)
                 bulk_wait_read<0>();
                 if (ok) {
                     load_group(0, next, j + 1);
-                    load_group(1, next, j + 1);
                     load_group(4, next, j + 1);
+                    load_group(1, next, j + 1);
                     load_group(2, next, j + 1);
                 }
             }
