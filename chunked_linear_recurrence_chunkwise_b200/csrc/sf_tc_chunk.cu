@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(kIntraThreads)
     using L = IntraSmem<kP>;
     constexpr bool kKK = kDelta || kP;  // a K K^T (or [Q;K] K^T) product is needed
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // 1024-aligned, shared window
     float* Gs = (float*)(sm + L::Gs);
     float* Bs = (float*)(sm + L::Bs);
     float* BGs = (float*)(sm + L::BGs);
@@ -517,7 +517,7 @@ __global__ void __launch_bounds__(128)
                      const __grid_constant__ CUtensorMap tm_o, const Args a) {
     using L = OutSmem;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // 1024-aligned, shared window
     float* Gs = (float*)(sm + L::Gs);
     const float* Eg = (const float*)(sm + L::Eg);
     uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);
@@ -676,7 +676,7 @@ __global__ void __launch_bounds__(128)
                        const __grid_constant__ CUtensorMap tm_o, const Args a) {
     using L = OutPSmem;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // 1024-aligned, shared window
     const float* Eg = (const float*)(sm + L::Eg);
     uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);
     uint64_t* bar_mma = bar_ld + 1;

@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(256, 1)
                         const Args a) {
     using L = GradSmem;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // 1024-aligned, shared window
     float* Gs = (float*)(sm + L::Gs);
     float* PD = (float*)(sm + L::PD);
     float* dGp = (float*)(sm + L::dGp);
