@@ -220,9 +220,10 @@ def kernel_units(name: str, w, mode: str = "keep") -> dict:
 # A kernel whose source has changed since reports traffic null.
 NCU_TRAFFIC_2048 = {
     # name: (bytes per 2048 chunk-heads, source file, sha256[:16]); profiles/<kernel>_*.md
-    "grad_fused": (437198336, "sf_tc_grad_fused.cu", "f75f206f17a7051b"),
+    "grad_fused": (431823360, "sf_tc_grad_fused.cu", "614da071aa2a2620"),
     "grad_attn": (321572096, "sf_tc_grad.cu", "5803a1b053b95f97"),
-    "state_fwd": (162895104, "sf_tc_state.cu", "c25118f738eb4316"),
+    "state_fwd": (163520512, "sf_tc_state.cu", "209eb1524f9f1ceb"),
+    "state_bwd": (224162304, "sf_tc_state.cu", "209eb1524f9f1ceb"),
 }
 KERNEL_SOURCE = {
     "grad_fused": "sf_tc_grad_fused.cu", "state_fwd": "sf_tc_state.cu", "state_bwd": "sf_tc_state.cu",
