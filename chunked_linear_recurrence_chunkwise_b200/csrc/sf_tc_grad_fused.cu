@@ -877,11 +877,16 @@ cudaError_t launch_grad_fused_tc(const Args& a, cudaStream_t s) {
                                          (int)smem);
     if (e != cudaSuccess) return e;
     timing_begin(KK_GRAD_FUSED, s);
-    // one CTA per SM it may hold (a.grad_sms < 0: all but that many, and at least half);
-    // the CTAs take the chunk-heads from the work counter
+    // One CTA per SM it may hold; the CTAs take the chunk-heads from the work counter.
+    // a.grad_sms < 0 asks to leave that many SMs to a reverse pass running beside the
+    // launch (one CTA per batch-head).  That pays while the pass holds at most a quarter
+    // of the SMs: with 32 heads of 148 SMs the pass and the launch take about as long
+    // (132 and 139 us per 4096-token piece), while with 64 heads the pass ends long
+    // before the launch, which is then faster on every SM.
     const int sms = sm_count();
-    const int budget = a.grad_sms > 0 ? std::min(a.grad_sms, sms)
-                                      : std::max(sms + a.grad_sms, sms / 2);
+    const int budget = a.grad_sms > 0                       ? std::min(a.grad_sms, sms)
+                       : (a.grad_sms < 0 && -4 * a.grad_sms <= sms) ? sms + a.grad_sms
+                                                                     : sms;
     const int ctas = std::min(a.NC * BH, budget);
     grad_fused_tc_kernel<<<ctas, kBlock, smem, s>>>(tm_q, tm_k, tm_do, tm_t, tm_dt, tm_ddt, tm_sc, tm_dsc, tm_dq,
                                                      tm_dk, tm_dv, tm_v, a);
