@@ -158,14 +158,17 @@ __device__ __forceinline__ void put_row(uint8_t* tile, int row, int q0, const fl
     }
 }
 
-// Work item n of a launch over NC chunks of every batch-head: the chunk fastest.
+// Work item n of a launch over NC chunks of every batch-head, the batch-head fastest: the
+// chunk-heads in flight at once then cover every head of a few chunks, and their
+// token-major loads take whole token rows.
 struct Item {
     int c, bh, b, h, t0;
 };
 __device__ __forceinline__ Item item_of(const Args& a, int n) {
     Item it;
-    it.c = n % a.NC;
-    it.bh = n / a.NC;
+    const int BH = a.B * a.H;
+    it.c = n / BH;
+    it.bh = n - it.c * BH;
     it.b = it.bh / a.H;
     it.h = it.bh - it.b * a.H;
     it.t0 = it.c * kChunk;
