@@ -220,7 +220,7 @@ def kernel_units(name: str, w, mode: str = "keep") -> dict:
 # A kernel whose source has changed since reports traffic null.
 NCU_TRAFFIC_2048 = {
     # name: (bytes per 2048 chunk-heads, source file, sha256[:16]); profiles/<kernel>_*.md
-    "grad_fused": (431823360, "sf_tc_grad_fused.cu", "614da071aa2a2620"),
+    "grad_fused": (432559104, "sf_tc_grad_fused.cu", "a4b03b30901bce81"),
     "grad_attn": (321560320, "sf_tc_grad.cu", "30dfb7b4600a540a"),
     "state_fwd": (163520512, "sf_tc_state.cu", "209eb1524f9f1ceb"),
     "state_bwd": (224162304, "sf_tc_state.cu", "209eb1524f9f1ceb"),
