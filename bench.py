@@ -215,15 +215,15 @@ def kernel_units(name: str, w, mode: str = "keep") -> dict:
 
 
 # DRAM bytes (read + write) per launch of one 4096-token piece of the 32-head, d = 128
-# workload (2048 chunk-heads) from an ncu capture, per kernel, with the sha256 (first 16
-# hex digits) of the source file the kernel was built from at the time of the capture.
-# A kernel whose source has changed since reports traffic null.
+# workload (2048 chunk-heads) from an ncu capture, per kernel, with `source_sha` of the
+# source file the kernel was built from at the time of the capture (its code, comments
+# left out).  A kernel whose code has changed since reports traffic null.
 NCU_TRAFFIC_2048 = {
-    # name: (bytes per 2048 chunk-heads, source file, sha256[:16]); profiles/<kernel>_*.md
-    "grad_fused": (432559104, "sf_tc_grad_fused.cu", "a4b03b30901bce81"),
-    "grad_attn": (321560320, "sf_tc_grad.cu", "30dfb7b4600a540a"),
-    "state_fwd": (163520512, "sf_tc_state.cu", "209eb1524f9f1ceb"),
-    "state_bwd": (224162304, "sf_tc_state.cu", "209eb1524f9f1ceb"),
+    # name: (bytes per 2048 chunk-heads, source file, source_sha); profiles/<kernel>_*.md
+    "grad_fused": (432559104, "sf_tc_grad_fused.cu", "1eb9c2de37a51998"),
+    "grad_attn": (321560320, "sf_tc_grad.cu", "48e6df666c2d3748"),
+    "state_fwd": (163520512, "sf_tc_state.cu", "bcaa1eef5ea3178a"),
+    "state_bwd": (224162304, "sf_tc_state.cu", "bcaa1eef5ea3178a"),
 }
 KERNEL_SOURCE = {
     "grad_fused": "sf_tc_grad_fused.cu", "state_fwd": "sf_tc_state.cu", "state_bwd": "sf_tc_state.cu",
@@ -232,12 +232,38 @@ KERNEL_SOURCE = {
 }
 
 
+def code_of(text: str) -> str:
+    """C/CUDA source without its comments, whitespace runs collapsed to one space
+    (string and character literals kept as written)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        ch = text[i]
+        if ch in "\"'":
+            j = i + 1
+            while j < n and text[j] != ch:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(ch)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_sha(fname: str) -> str | None:
+    """sha256 (first 16 hex digits) of a kernel source's code, comments left out, so
+    that the traffic of a capture stays attached to its code through comment edits."""
     import hashlib
     path = os.path.join(ROOT, "chunked_linear_recurrence_chunkwise_b200", "csrc", fname)
     try:
-        with open(path, "rb") as f:
-            return hashlib.sha256(f.read()).hexdigest()[:16]
+        with open(path, encoding="utf-8") as f:
+            return hashlib.sha256(code_of(f.read()).encode()).hexdigest()[:16]
     except OSError:
         return None
 

@@ -1,7 +1,8 @@
 // Fused per-chunk gradient kernel of the gated delta rule (sm_100a).
 //
-// One CTA per chunk-head computes dq, dk, dv, dbeta and dg from one load of
-// its inputs.  The chunkwise backward of the delta rule, with S the state
+// For each chunk-head (64 tokens of one batch-head) the kernel computes dq, dk,
+// dv, dbeta and dg from one load of its inputs.  The chunkwise backward of the
+// delta rule, with S the state
 // entering the chunk, dS' the gradient of the state leaving it, T = (I + A)^-1
 // the chunk's UT inverse and Delta = U - W S its corrected values:
 //   P = (Q K^T) .* Gamma,  dP = (dO Delta^T) .* lower,  F = dP .* Gamma
@@ -32,13 +33,13 @@
 //
 // One CTA per SM takes chunk-heads (work items) from a counter until none are
 // left, so that CTAs which start late (the SM was busy) take fewer, and
-// overlaps them: one thread of a seventeenth warp issues the copies, the stores and every
-// UMMA, each as soon as its operands are in place and the tiles or TMEM
-// columns it overwrites are dead; the next item's copies go out as the current
-// item's products finish with their tiles (dDelta^T, T, dO, Delta^T and S^T
-// once [dA | dKhat] has run, dS'^T once E is consumed, Q and K once the last
-// product has read K and the dq store has read Q), and its first product
-// T^T dDelta runs behind the current item's last one.  Sixteen warps share the
+// overlaps them: one thread of a seventeenth warp issues the copies, the stores
+// and every UMMA, each as soon as its operands are in place and the tiles or
+// TMEM columns it overwrites are dead.  The next item's copies go out as the
+// current item's products finish with their tiles: dDelta^T, T, dO, Delta^T,
+// S^T, Q, G and V once F K and F^T Q have run (K into the other of two K tiles),
+// dS'^T once E, written over it, is consumed; its first product T^T dDelta runs
+// behind the current item's last one.  Sixteen warps share the
 // element-wise work (warp w reads TMEM lane quadrant w % 4 and a quarter of
 // the columns, w / 4); they hand each stage over through an mbarrier (one
 // arrival per warp) and wait for the products they read on the commit
@@ -46,7 +47,8 @@
 // dependent chain first: dVhat -> dv, dbeta's V term and dVhat in bf16 ->
 // [dA | dKhat] -> E, dKp -> (E + E^T) K -> dk; the attention side (P, dP, F,
 // the rescaled dO S^T and Delta dS'^T, then F K and F^T Q -> dq) fills the
-// gaps.  dv, dq and dk leave through TMA stores from staging tiles.
+// gaps.  dv, dq and dk leave through TMA stores from staging tiles (dv over V,
+// dq in the PD region, dk in its item's K tile).
 
 #include <cuda.h>
 

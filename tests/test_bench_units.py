@@ -54,3 +54,13 @@ def test_step_roofline_of_the_bench_workload():
     assert abs(s["tflops"] - 417792 * th / 5e-3 / 1e12) < 0.01
     assert abs(s["hbm_floor_ms"] - 2840 * th / 6550.1e9 * 1e3) < 1e-3
     assert abs(s["hbm_floor_frac"] - s["hbm_floor_ms"] / 5.0) < 1e-3
+
+
+def test_source_hash_ignores_comments_only():
+    import bench
+    a = 'int x = 1; // one\n/* block\n comment */ const char* s = "a // b";\n'
+    b = 'int   x = 1;\nconst char* s = "a // b";  // another note\n'
+    c = 'int x = 2; const char* s = "a // b";'
+    assert bench.code_of(a) == bench.code_of(b)
+    assert bench.code_of(a) != bench.code_of(c)
+    assert '"a // b"' in bench.code_of(a)  # string literals are kept whole
