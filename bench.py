@@ -45,6 +45,9 @@ def parse_args(argv=None):
     p.add_argument("--no-other-mode", action="store_true",
                    help="do not time the other driver form beside the headline one")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-graph", action="store_true",
+                   help="time the driver calls launched eagerly instead of a CUDA-graph replay of them "
+                        "(the eager time is reported beside the graph one otherwise)")
     p.add_argument("--memory-study", default=None, metavar="T1,T2,...",
                    help="instead of the bench line: the layer's device memory and step time for these "
                         "sequence lengths at a fixed piece length of 4096 tokens (one JSON line)")
@@ -515,6 +518,19 @@ def workspace(torch, nbytes: int, dev):
     return ws
 
 
+def capture_graph(torch, fn, dev):
+    """A CUDA graph of one step's driver calls: fn(stream) issues them with `stream` as
+    their main stream (captured on a side stream; the drivers' aux and critical streams
+    join the capture through their event waits)."""
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.graph(g, stream=s):
+        fn(s)
+    torch.cuda.synchronize(dev)
+    return g
+
+
 def time_planned_cut(args, sf, torch, sh, lens, x, timing, dev, main, aux, outs):
     """Device time of the keep drivers on the cut sf_plan_cut picks from the measured costs."""
     n_chunks = sum(-(-n // 64) for n in lens)
@@ -532,16 +548,23 @@ def time_planned_cut(args, sf, torch, sh, lens, x, timing, dev, main, aux, outs)
     ws_b = workspace(torch, sf.sf_seq_workspace_bytes(sh, plan, sf.SF_OP_BWD), dev)
     keep = torch.empty(sf.sf_keep_bytes(sh, plan), dtype=torch.uint8, device=dev)
 
-    def step():
+    def step(sm=None):
+        sm = sm or main
         sf.sf_fwd_seq_keep(sh, plan, x["q"], x["k"], x["v"], x["g"], x["beta"], None, outs["o"],
-                           outs["S_out"], keep, ws_f, stream_main=main, stream_aux=aux)
+                           outs["S_out"], keep, ws_f, stream_main=sm, stream_aux=aux)
         sf.sf_bwd_seq_keep(sh, plan, x["q"], x["k"], x["v"], x["g"], x["beta"], keep, x["dO"], None,
                            outs["dq"], outs["dk"], outs["dv"], outs["dg"], outs["dbeta"], outs["dS_in"],
-                           ws_b, stream_main=main, stream_aux=aux)
+                           ws_b, stream_main=sm, stream_aux=aux)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    if not args.no_graph:  # timed as the headline is: a CUDA-graph replay of the two calls
+        g = capture_graph(torch, step, dev)
+
+        def step():
+            with torch.cuda.stream(main):
+                g.replay()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(main)
     for _ in range(args.steps):
@@ -587,21 +610,22 @@ def run_sf(args, w, rank, world, local_rank):
     outs_main = {"o": o, "dq": dq, "dk": dk, "dv": dv, "S_out": S_out, "dS_in": dS_in, "dg": dg,
                  "dbeta": db}
 
-    def step(src, serial=False, mode=None, out=None):
-        sa = main if serial else aux
+    def step(src, serial=False, mode=None, out=None, sm=None):
+        sm = sm or main
+        sa = sm if serial else aux
         r = out or outs_main
         if (mode or args.mode) == "keep":
             sf.sf_fwd_seq_keep(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], None, r["o"],
-                               r["S_out"], keep, ws_f, stream_main=main, stream_aux=sa)
+                               r["S_out"], keep, ws_f, stream_main=sm, stream_aux=sa)
             sf.sf_bwd_seq_keep(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], keep,
                                src["dO"], None, r["dq"], r["dk"], r["dv"], r["dg"], r["dbeta"], r["dS_in"],
-                               ws_b, stream_main=main, stream_aux=sa)
+                               ws_b, stream_main=sm, stream_aux=sa)
             return
         sf.sf_fwd_seq(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], None, r["o"],
-                      r["S_out"], S_saved, ws_f, stream_main=main, stream_aux=sa)
+                      r["S_out"], S_saved, ws_f, stream_main=sm, stream_aux=sa)
         sf.sf_bwd_seq(sh, lens, src["q"], src["k"], src["v"], src["g"], src["beta"], S_saved,
                       src["dO"], None, r["dq"], r["dk"], r["dv"], r["dg"], r["dbeta"], r["dS_in"], ws_b,
-                      stream_main=main, stream_aux=sa)
+                      stream_main=sm, stream_aux=sa)
 
     def barrier():
         if world > 1:
@@ -613,16 +637,43 @@ def run_sf(args, w, rank, world, local_rank):
     sf.sf_check(ws_f, main)
     sf.sf_check(ws_b, main)
 
+    # ---- the eager driver calls, timed (reported beside the headline, or as it)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(main)
+    for _ in range(args.steps):
+        step(x)
+    e1.record(main)
+    torch.cuda.synchronize()
+    barrier()
+    ms_eager = reduce_max(e0.elapsed_time(e1) / args.steps, device=dev)
+    sf.sf_check(ws_f, main)
+    sf.sf_check(ws_b, main)
+
+    # ---- the headline: one step's two driver calls captured into a CUDA graph and
+    # replayed (the same kernels in the same order; launch gaps shrink)
+    graph = None
+    if not args.no_graph:
+        graph = capture_graph(torch, lambda s: step(x, sm=s), dev)
+        for _ in range(args.warmup):
+            with torch.cuda.stream(main):
+                graph.replay()
+        torch.cuda.synchronize()
+
     # ---- device-timed region (inputs resident in HBM; they exceed L2, so no flush)
     clk = ClockSampler(local_rank)
     barrier()
     torch.cuda.synchronize()
     clk.start()
     time.sleep(0.3)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(main)
     for _ in range(args.steps):
-        step(x)
+        if graph is not None:
+            with torch.cuda.stream(main):
+                graph.replay()
+        else:
+            step(x)
     e1.record(main)
     torch.cuda.synchronize()
     clocks = clk.stop()
@@ -631,6 +682,7 @@ def run_sf(args, w, rank, world, local_rank):
     ms_max = reduce_max(ms, device=dev)
     sf.sf_check(ws_f, main)
     sf.sf_check(ws_b, main)
+    del graph
 
     # ---- the other driver form, timed the same way (reported beside the headline)
     other = "recompute" if args.mode == "keep" else "keep"
@@ -736,9 +788,12 @@ def run_sf(args, w, rank, world, local_rank):
             "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
             "data": "synthetic",
-            "config": bench_config(w, lens, world, args.mode),
+            "config": dict(bench_config(w, lens, world, args.mode),
+                           launch="eager" if args.no_graph else "cuda_graph"),
             "modes": {args.mode: {"ms_per_step": round(ms_max, 4),
                                   "value": round(job_tokens_per_s(world, B, T, ms_max), 1)},
+                      args.mode + "_eager": {"ms_per_step": round(ms_eager, 4),
+                                             "value": round(job_tokens_per_s(world, B, T, ms_eager), 1)},
                       other: None if ms_other is None else
                       {"ms_per_step": round(ms_other, 4),
                        "value": round(job_tokens_per_s(world, B, T, ms_other), 1)}},

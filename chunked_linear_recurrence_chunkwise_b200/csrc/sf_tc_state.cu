@@ -127,7 +127,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         const __grid_constant__ CUtensorMap tm_dt, const Args a) {
     using L = FwdSmem;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // 1024-aligned, shared window
+    // the 1024-aligned base by integer rounding: with the pointer arithmetic of the other
+    // kernels the reverse pass, run right after the forward pass on the same stream, gave
+    // up a bounded wait a few times in a thousand steps (the cause is not known)
+    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     float* Eds = (float*)(sm + L::Ed);
     uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);  // [kStages], count 1
     uint64_t* bar_x = bar_ld + kStages;           // count 1 (commits)
@@ -410,7 +413,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         const Args a) {
     using L = BwdSmem;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // 1024-aligned, shared window
+    // the 1024-aligned base by integer rounding: with the pointer arithmetic of the other
+    // kernels the reverse pass, run right after the forward pass on the same stream, gave
+    // up a bounded wait a few times in a thousand steps (the cause is not known)
+    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     float* Eds = (float*)(sm + L::Ed);
     uint64_t* bar_ld = (uint64_t*)(sm + L::Bar);  // [kBStages], count 1
     uint64_t* bar_y = bar_ld + kBStages;          // count 1 (commits and the copy thread)

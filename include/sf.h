@@ -112,7 +112,10 @@ size_t sf_seq_workspace_bytes(const sf_shape* shape, int n_sub, const int* lens,
  * is scheduled ahead of the parallel work (the first such call on a device
  * creates that stream; make it before any stream capture).  On return all
  * work is ordered before later work on stream_main.  stream_aux may equal
- * stream_main (no overlap, everything on stream_main). */
+ * stream_main (no overlap, everything on stream_main).  The drivers may be
+ * captured into a CUDA graph by capturing stream_main (stream_aux and the
+ * internal stream join the capture through the drivers' event waits); a
+ * replay runs the same kernels on the same pointers and gives the same bits. */
 sf_status sf_fwd_seq(const sf_shape* shape, int n_sub, const int* lens, const void* q,
                      const void* k, const void* v, const float* g, const float* beta,
                      const float* S_in, void* o, float* S_out, float* S_saved, void* ws,
