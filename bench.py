@@ -525,7 +525,9 @@ def capture_graph(torch, fn, dev):
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize(dev)
-    with torch.cuda.graph(g, stream=s):
+    # thread-local: other threads of the process (a process group's watchdog) may keep
+    # making CUDA calls while this thread captures
+    with torch.cuda.graph(g, stream=s, capture_error_mode="thread_local"):
         fn(s)
     torch.cuda.synchronize(dev)
     return g
