@@ -562,11 +562,18 @@ def time_planned_cut(args, sf, torch, sh, lens, x, timing, dev, main, aux, outs)
         step()
     torch.cuda.synchronize()
     if not args.no_graph:  # timed as the headline is: a CUDA-graph replay of the two calls
-        g = capture_graph(torch, step, dev)
+        try:
+            g = capture_graph(torch, step, dev)
 
-        def step():
-            with torch.cuda.stream(main):
-                g.replay()
+            def step():
+                with torch.cuda.stream(main):
+                    g.replay()
+
+            for _ in range(args.warmup):
+                step()
+        except RuntimeError:
+            pass
+        torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(main)
     for _ in range(args.steps):
@@ -655,9 +662,15 @@ def run_sf(args, w, rank, world, local_rank):
 
     # ---- the headline: one step's two driver calls captured into a CUDA graph and
     # replayed (the same kernels in the same order; launch gaps shrink)
-    graph = None
+    graph, launch = None, "eager"
     if not args.no_graph:
-        graph = capture_graph(torch, lambda s: step(x, sm=s), dev)
+        try:
+            graph = capture_graph(torch, lambda s: step(x, sm=s), dev)
+            launch = "cuda_graph"
+        except RuntimeError as e:  # time the eager step instead, and say so
+            torch.cuda.synchronize()
+            launch = f"eager (graph capture failed: {str(e)[:120]})"
+    if graph is not None:
         for _ in range(args.warmup):
             with torch.cuda.stream(main):
                 graph.replay()
@@ -790,8 +803,7 @@ def run_sf(args, w, rank, world, local_rank):
             "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
             "data": "synthetic",
-            "config": dict(bench_config(w, lens, world, args.mode),
-                           launch="eager" if args.no_graph else "cuda_graph"),
+            "config": dict(bench_config(w, lens, world, args.mode), launch=launch),
             "modes": {args.mode: {"ms_per_step": round(ms_max, 4),
                                   "value": round(job_tokens_per_s(world, B, T, ms_max), 1)},
                       args.mode + "_eager": {"ms_per_step": round(ms_eager, 4),
