@@ -552,6 +552,7 @@ __global__ void __launch_bounds__(kBlock, 1)
             }
         };
         int eprev = -1, last_j = 0;  // the last item's chunk-head and index
+        bool gave_up = false;        // the same in every element-wise warp
         for (int j = 0; ecur >= 0; ++j) {
             const uint32_t ph = (uint32_t)(j & 1);
             const float* Gs = (const float*)(sm + L::Gs) + (j & 1) * 64;
@@ -785,9 +786,16 @@ __global__ void __launch_bounds__(kBlock, 1)
             hand_over(&bar_s[2]);
             // dq (lanes 0-15 of lo [128, 256)) is final once F K has run: its rows into the PD
             // region for the store, once every warp's column sums have read PD (the barrier
-            // also completes every warp's partial sums for the epilogue)
+            // also completes every warp's partial sums for the epilogue).  At this barrier the
+            // warps also agree on whether a wait of the CTA gave up, and then all leave the
+            // loop here: a warp whose wait for the published next item gave up may have read
+            // a stale one, and warps that went on to different items would never meet at
+            // their named barriers again.
             wait_flag(&bar_c[1], ph, kErrTimeoutMma);
-            named_sync(1, kThreads);
+            if (named_sync_or(1, kThreads, *s_abort != 0)) {
+                gave_up = true;
+                break;
+            }
             tc_fence_after();
             {
                 float x[32];
@@ -820,7 +828,7 @@ __global__ void __launch_bounds__(kBlock, 1)
             bpre = bnext;
             last_j = j;
         }
-        if (eprev >= 0 && warp < 4) epilogue(eprev, last_j);
+        if (!gave_up && eprev >= 0 && warp < 4) epilogue(eprev, last_j);
     }
     __syncthreads();
     if (tid == kIss) {
